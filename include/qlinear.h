@@ -1,0 +1,156 @@
+/*
+ * qlinear.h -- C ABI of the group-wise affine W4 g64 quantized linear layer (sm_100a).
+ *
+ * The packed format (aimarketly "Ideogram-4-IQ4_M", intro: one f16 scale and one
+ * f16 bias per 64 weights on top of 4-bit codes, 4.5 bits per weight;
+ * huggingface "SceneWorks/ideogram-4-mlx", Versions: group-wise affine, group
+ * size 64) and its uniform affine grid w = scale * q + bias (aimarketly
+ * "Ideogram-4-IQ4_M", "What IQ4 means here").
+ *
+ * Layout of every tensor (all row-major, dense, no padding):
+ *   x       bf16     [M][K]      activations
+ *   codes   uint32   [N][K/8]    code (n, k) = (codes[n][k/8] >> 4*(k%8)) & 0xF, low nibble first
+ *   scales  f16      [N][K/64]   group scale  s(n, k/64)
+ *   biases  f16      [N][K/64]   group bias   b(n, k/64)
+ *   y       bf16     [M][N]      y[m][n] = sum_k x[m][k] * (s * q(n, k) + b)
+ * W is logically [N][K] (a PyTorch Linear weight): y = x . W^T.
+ *
+ * Conventions shared by every entry point:
+ *   - Ownership: the caller owns every buffer.  Tensor arguments are DEVICE
+ *     pointers on the current CUDA device.  The library allocates no device
+ *     memory; scratch comes from the caller's workspace.
+ *   - Asynchrony: work is enqueued on `stream` (0 = legacy default stream).
+ *     QL_OK means "validated and launched"; launch failures return QL_ERR_CUDA.
+ *     Faults detected inside kernels (non-finite pack input, a bounded wait that
+ *     expired) are recorded in a per-device status word read by
+ *     qlinear_get_device_status().
+ *   - Validation happens before any launch; on any error nothing is launched.
+ *     Required: group == 64 (else QL_ERR_UNSUPPORTED); K % 64 == 0, N % 8 == 0,
+ *     M >= 1, K >= 64, N >= 8, non-null tensors (else QL_ERR_INVALID_ARG); every
+ *     pointer 16-byte aligned (else QL_ERR_ALIGNMENT); outputs must not overlap
+ *     inputs (else QL_ERR_INVALID_ARG).
+ *   - Non-finite activations or parameters propagate through the arithmetic
+ *     IEEE-style.
+ *   - Thread safety: calls are reentrant; the last-dispatch record is
+ *     thread-local.
+ */
+#ifndef QLINEAR_H
+#define QLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QL_OK = 0,
+    QL_ERR_INVALID_ARG = 1,     /* bad size, null pointer, overlap, non-finite pack input */
+    QL_ERR_ALIGNMENT = 2,       /* a pointer is not 16-byte aligned */
+    QL_ERR_UNSUPPORTED = 3,     /* group != 64, or a feature not built (see each call) */
+    QL_ERR_WORKSPACE = 4,       /* workspace missing or smaller than qlinear_workspace_size() */
+    QL_ERR_CUDA = 5,            /* a CUDA runtime call or kernel launch failed */
+    QL_ERR_DEVICE_TIMEOUT = 6,  /* a bounded wait inside a kernel expired; the kernel returned early */
+    QL_ERR_BOUNDS = 7           /* a kernel's own index check failed (debug builds) */
+} ql_status;
+
+typedef enum { QL_F32 = 0, QL_BF16 = 1 } ql_dtype;
+
+/* Kernel paths of qlinear_forward, for qlinear_forward_config() and qlinear_last_dispatch(). */
+typedef enum {
+    QL_PATH_AUTO = 0,       /* per-shape choice of the dispatcher */
+    QL_PATH_GEMV = 1,       /* CUDA-core split-K weight streaming (any M; meant for M <= 4) */
+    QL_PATH_TC_SKINNY = 2,  /* tcgen05 weight streaming for small M: integer codes as bf16,
+                               per-group scale/bias applied to fp32 partials; M <= 32 */
+    QL_PATH_TC_FUSED = 3    /* tcgen05 fused-dequant GEMM for large M: fp16 operands,
+                               fp32 TMEM accumulators */
+} ql_path;
+
+/*
+ * Bytes of device workspace qlinear_forward() needs for this shape (0 is
+ * possible).  Returns (size_t)-1 when the shape is invalid.
+ */
+size_t qlinear_workspace_size(int64_t M, int64_t K, int64_t N, int32_t group);
+
+/*
+ * y = x . W^T for the packed W (the layer the pages describe: bf16
+ * activations, fp32 accumulation, bf16 output).  Preconditions and errors as in
+ * the conventions above; additionally `workspace` must hold at least
+ * qlinear_workspace_size(M, K, N, group) bytes (QL_ERR_WORKSPACE otherwise)
+ * and must not overlap any tensor.  The dispatcher picks the kernel path from
+ * (M, K, N); qlinear_last_dispatch() reports the choice.
+ */
+ql_status qlinear_forward(const void* x, const uint32_t* codes, const void* scales,
+                          const void* biases, void* y, int64_t M, int64_t K, int64_t N,
+                          int32_t group, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream);
+
+/*
+ * qlinear_forward with the path and split-K factor forced (testing and tuning).
+ * path: a ql_path; split_k: 0 = the dispatcher's choice, else the number of K
+ * slices (must divide K/64 into non-empty slices; QL_ERR_INVALID_ARG otherwise).
+ * out_dtype: QL_BF16 = the layer's output; QL_F32 writes y as fp32 [M][N]
+ * (the same arithmetic without the final rounding, for numerical tests).
+ * A path that cannot run the shape returns QL_ERR_UNSUPPORTED.
+ */
+ql_status qlinear_forward_config(const void* x, const uint32_t* codes, const void* scales,
+                                 const void* biases, void* y, ql_dtype out_dtype,
+                                 int64_t M, int64_t K, int64_t N, int32_t group,
+                                 int32_t path, int32_t split_k,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes for qlinear_forward_config() with the same path and split_k. */
+size_t qlinear_workspace_size_config(int64_t M, int64_t K, int64_t N, int32_t group,
+                                     int32_t path, int32_t split_k);
+
+/*
+ * Standalone dequantization: out[n][k] = RN_fp32(s * q + b), rounded once more
+ * to bf16 (nearest even) when out_dtype == QL_BF16.  Bit-exact by definition:
+ * s*q + b is formed with one fused multiply-add.  out is [N][K] of out_dtype.
+ */
+ql_status qlinear_dequant(const uint32_t* codes, const void* scales, const void* biases,
+                          int64_t K, int64_t N, int32_t group, void* out, ql_dtype out_dtype,
+                          cudaStream_t stream);
+
+/*
+ * Quantize fp32 w [N][K] into codes/scales/biases.
+ * imatrix == NULL: min/max round-to-nearest (MLX's own solution, candidate 0
+ * of the search in aimarketly "Ideogram-4-IQ4_M", "What IQ4 means here"):
+ * per group of 64, s = RN32(RN32(max-min)/15), scale = RN_f16(s),
+ * bias = RN_f16(min), q = clamp(rint(RN32(RN32(w-bias)/scale)), 0, 15)
+ * (ties to even), q = 0 when scale == 0.  Deterministic: equal inputs give
+ * equal bytes.
+ * imatrix != NULL (importance-weighted fit): QL_ERR_UNSUPPORTED in this build.
+ * A group holding a non-finite value or |w| > 65504 is written as codes 0,
+ * scale 0, bias 0, and the device status word records QL_ERR_INVALID_ARG.
+ */
+ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group,
+                       uint32_t* codes, void* scales, void* biases, cudaStream_t stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the current device's status word
+ * (the first error a kernel recorded since the last read).  Returns QL_OK when
+ * no kernel recorded anything, QL_ERR_CUDA if the synchronization fails.
+ */
+ql_status qlinear_get_device_status(cudaStream_t stream);
+
+/*
+ * Writes a NUL-terminated description of the calling thread's last
+ * qlinear_forward dispatch ("path=tc_fused tile=128x256 stages=4 splitk=1"),
+ * truncated to len bytes.  QL_ERR_INVALID_ARG if buf is NULL or len == 0.
+ */
+ql_status qlinear_last_dispatch(char* buf, size_t len);
+
+/* Static, human-readable name of a status code. */
+const char* qlinear_status_string(ql_status status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int32_t qlinear_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLINEAR_H */

@@ -1,0 +1,404 @@
+"""CPU oracle for the group-wise affine W4 g64 quantized linear layer.
+
+TEST INFRASTRUCTURE.  Only the tests, the smoke check and the benchmark's CPU
+baseline leg use this module.  The library's product path never imports, calls
+or links it, and it shares no code with the CUDA sources: it decodes the packed
+format, dequantizes, multiplies and quantizes with its own plain numpy code.
+
+What the layer computes, and where the pages say it:
+  * Format: 4-bit codes; every 64 consecutive weights along the input
+    dimension share one f16 scale and one f16 bias, which is the "+0.5 bit"
+    overhead on top of the 4-bit width (aimarketly "Ideogram-4-IQ4_M", intro;
+    huggingface "SceneWorks/ideogram-4-mlx", Versions: group-wise affine,
+    group size 64).
+  * Dequantization is the uniform affine grid w = scale * q + bias, the grid
+    the MLX quantized matmul reads (aimarketly "Ideogram-4-IQ4_M", "What IQ4
+    means here").
+  * The layer is y = x . W^T with bf16 activations, fp32 accumulation and bf16
+    output; here the product is formed in float64 from the fp32 dequantized
+    weights, the reference the CUDA path is measured against.
+  * Quantization: MLX's min/max round-to-nearest (RTN) solution, and an
+    importance-weighted least-squares fit searched with RTN as candidate 0, so
+    the fit is never worse than RTN on sum_j E[x_j^2] * dW_j^2 (aimarketly
+    "Ideogram-4-IQ4_M", "What IQ4 means here"); weights with no activation
+    statistics fall back to RTN (same page, "How the statistics were
+    collected").  The packer is deterministic ("byte-equivalent to load-time
+    quantization", huggingface "SceneWorks/ideogram-4-mlx", Provenance).
+
+Readings adopted where the pages are silent (each is also listed in the design
+notes of the repository):
+  R1 layout: W is [N][K] (a PyTorch Linear weight); codes are uint32 [N][K/8]
+     with code (n, k) = (codes[n][k/8] >> 4*(k%8)) & 0xF (low nibble first);
+     scales and biases are f16 [N][K/64].
+  R2 "fp32 dequant" is the correctly rounded binary32 value of the exact
+     s*q + b.
+  R3 RTN: per group of 64 fp32 weights, s = RN32(RN32(max - min) / 15),
+     scale = RN_f16(s), bias = RN_f16(min) (no zero snapping), and
+     q = clamp(round_half_even(RN32(RN32(w - bias) / scale)), 0, 15), q = 0
+     when scale == 0; codes are computed from the stored f16 parameters.
+  R4 imatrix fit: candidate grid, refits and the regularisation of
+     unobserved channels as documented on pack_imatrix().
+  R5 tolerance: bf16 output is gated on relative Frobenius error <= 4e-3 and
+     on max_i(|y_i - y_ref_i| - half_ulp_bf16(max(|y_i|, |y_ref_i|)))^+ <=
+     1.5e-2 * rms(y_ref); the literal max error is reported beside it.
+
+Parity status: the imatrix fit (pack_imatrix) is a search heuristic with no
+printed reference values; only its invariants are pinned ("never worse than
+RTN" per group, exact recovery of on-grid groups).  Everything else is pinned
+to closed forms, library conversions or brute force by the CPU tests.
+"""
+from __future__ import annotations
+
+import struct
+
+import numpy as np
+
+GROUP = 64
+F16_MAX = 65504.0
+
+
+# --------------------------------------------------------------------------
+# Format decoding (R1)
+# --------------------------------------------------------------------------
+
+def decode_f16(bits) -> np.ndarray:
+    """IEEE binary16 bit patterns -> float64, from the sign/exponent/fraction fields."""
+    b = np.asarray(bits).astype(np.uint16).astype(np.int64)
+    sign = np.where((b >> 15) & 1, -1.0, 1.0)
+    e = (b >> 10) & 0x1F
+    f = (b & 0x3FF).astype(np.float64)
+    normal = np.ldexp(1024.0 + f, (e - 25).astype(np.int32))      # (1 + f/2^10) * 2^(e-15)
+    subnormal = np.ldexp(f, -24)                                  # f/2^10 * 2^-14
+    special = np.where(f == 0, np.inf, np.nan)
+    mag = np.where(e == 0, subnormal, np.where(e == 31, special, normal))
+    return sign * mag
+
+
+def f16_array_bits(a) -> np.ndarray:
+    """Bit patterns of an f16 array (a view; no conversion)."""
+    return np.ascontiguousarray(a).view(np.uint16)
+
+
+def decode_bf16(bits) -> np.ndarray:
+    """bf16 bit patterns -> float64: a bf16 value is the upper half of a binary32."""
+    b = np.asarray(bits).astype(np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def unpack_codes(codes, K: int) -> np.ndarray:
+    """uint32 [N][K/8] -> int64 codes q [N][K], code k%8 in bits 4*(k%8) .. 4*(k%8)+3."""
+    c = np.asarray(codes, dtype=np.uint32).astype(np.int64)
+    N = c.shape[0]
+    assert c.shape[1] * 8 == K
+    shifts = 4 * np.arange(8, dtype=np.int64)
+    q = (c[:, :, None] >> shifts[None, None, :]) & 0xF
+    return q.reshape(N, K)
+
+
+def pack_codes(q) -> np.ndarray:
+    """int codes [N][K] in [0, 15] -> uint32 [N][K/8], low nibble first."""
+    q = np.asarray(q, dtype=np.uint64)
+    N, K = q.shape
+    assert K % 8 == 0 and q.max(initial=0) <= 15
+    shifts = 4 * np.arange(8, dtype=np.uint64)
+    words = (q.reshape(N, K // 8, 8) << shifts[None, None, :]).sum(axis=-1)
+    return words.astype(np.uint32)
+
+
+# --------------------------------------------------------------------------
+# Dequantization (R2)
+# --------------------------------------------------------------------------
+
+def dequant_exact(codes, scales, biases) -> np.ndarray:
+    """Exact w = s*q + b as float64 [N][K].
+
+    Exact because s and b are f16 values, i.e. integer multiples of 2^-24 below
+    2^16, and q <= 15: s*q + b = i * 2^-24 with |i| < 2^45, which float64 holds
+    without rounding (both the product and the sum are exact).
+    """
+    N, G = np.shape(scales)
+    K = G * GROUP
+    q = unpack_codes(codes, K).astype(np.float64)
+    s = np.repeat(decode_f16(f16_array_bits(scales)), GROUP, axis=1)
+    b = np.repeat(decode_f16(f16_array_bits(biases)), GROUP, axis=1)
+    return s * q + b
+
+
+def dequant_f32(codes, scales, biases) -> np.ndarray:
+    """fp32 dequant: RN_fp32 of the exact value (numpy's float64->float32 cast rounds to nearest even)."""
+    return dequant_exact(codes, scales, biases).astype(np.float32)
+
+
+def round_bf16(v) -> np.ndarray:
+    """Round float64 values to bf16 (8 significant bits, nearest, ties to even) -> uint16 bits.
+
+    Works from the exact value: v = f * 2^e with 0.5 <= |f| < 1, keep f * 2^8
+    rounded half-to-even.  Overflow goes to +-inf, NaN stays NaN.  (bf16
+    subnormals, |v| < 2^-126, are rounded on the subnormal grid 2^-133.)
+    """
+    v = np.asarray(v, dtype=np.float64)
+    f, e = np.frexp(v)
+    e = np.maximum(e, -125)                      # below 2^-126 the grid is fixed at 2^-133
+    m = np.rint(np.ldexp(v, 8 - e))             # integer significand, ties to even
+    r = np.ldexp(m, e - 8)
+    r = np.where(np.isnan(v), np.nan, r)
+    r = np.where(np.abs(r) >= 2.0 ** 128, np.copysign(np.inf, v), r)
+    r32 = r.astype(np.float32)                  # exact: r has <= 8 significant bits
+    return (r32.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def dequant_bf16(codes, scales, biases) -> np.ndarray:
+    """bf16 dequant = RN_bf16(fp32 dequant) as uint16 bits (the fp32 value is rounded again)."""
+    return round_bf16(dequant_f32(codes, scales, biases).astype(np.float64))
+
+
+# --------------------------------------------------------------------------
+# The layer y = x . W^T
+# --------------------------------------------------------------------------
+
+def forward_ref(x_bits, codes, scales, biases) -> np.ndarray:
+    """y_ref[m][n] = sum_k x[m][k] * w(n, k) in float64, w the fp32 dequant.
+
+    Every product x*w is exact in float64 (8 + 24 significant bits); the sum is
+    a float64 matrix product.
+    """
+    x = decode_bf16(x_bits)
+    w = dequant_f32(codes, scales, biases).astype(np.float64)
+    return x @ w.T
+
+
+def forward_rows(x_bits, codes, scales, biases, rows) -> np.ndarray:
+    """forward_ref restricted to the given rows of x (rows are independent)."""
+    x = decode_bf16(np.asarray(x_bits)[np.asarray(rows)])
+    w = dequant_f32(codes, scales, biases).astype(np.float64)
+    return x @ w.T
+
+
+def forward_triple_loop(x_bits, codes, scales, biases):
+    """Brute force: nibble, f16 and bf16 decoded inline per element, float64 sum in k order.
+
+    Pure Python; tiny shapes only.
+    """
+    x_bits = np.asarray(x_bits)
+    M, K = x_bits.shape
+    N = np.shape(codes)[0]
+    s_bits = f16_array_bits(scales)
+    b_bits = f16_array_bits(biases)
+    y = [[0.0] * N for _ in range(M)]
+    for m in range(M):
+        xs = [struct.unpack("<f", struct.pack("<I", int(x_bits[m, k]) << 16))[0] for k in range(K)]
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                word = int(codes[n, k // 8])
+                q = (word >> (4 * (k % 8))) & 0xF
+                s = struct.unpack("<e", struct.pack("<H", int(s_bits[n, k // GROUP])))[0]
+                b = struct.unpack("<e", struct.pack("<H", int(b_bits[n, k // GROUP])))[0]
+                w32 = struct.unpack("<f", struct.pack("<f", s * q + b))[0]   # RN to binary32
+                acc += xs[k] * w32
+            y[m][n] = acc
+    return np.array(y, dtype=np.float64)
+
+
+def half_ulp_bf16(v) -> np.ndarray:
+    """Half a bf16 unit in the last place at |v| (normal range)."""
+    _, e = np.frexp(np.abs(np.asarray(v, dtype=np.float64)))
+    return np.ldexp(1.0, np.maximum(e, -125) - 9)
+
+
+def tolerance(y, y_ref, bf16_output: bool = True) -> dict:
+    """Error metrics of reading R5.
+
+    relF     = ||y - y_ref||_F / ||y_ref||_F                (gate <= 4e-3)
+    max_rel  = max|y - y_ref| / rms(y_ref)                  (literal, reported)
+    max_gate = max(|y - y_ref| - half_ulp)^+ / rms(y_ref)   (gate <= 1.5e-2; half_ulp = 0 for fp32 output)
+    """
+    y = np.asarray(y, dtype=np.float64)
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    d = np.abs(y - y_ref)
+    rms = float(np.sqrt(np.mean(y_ref * y_ref)))
+    ref_norm = float(np.linalg.norm(y_ref))
+    relF = float(np.linalg.norm(y - y_ref) / ref_norm) if ref_norm > 0 else float(np.linalg.norm(y - y_ref))
+    allowance = half_ulp_bf16(np.maximum(np.abs(y), np.abs(y_ref))) if bf16_output else 0.0
+    excess = np.maximum(d - allowance, 0.0)
+    denom = rms if rms > 0 else 1.0
+    return {
+        "relF": relF,
+        "max_rel": float(d.max(initial=0.0) / denom),
+        "max_gate": float(excess.max(initial=0.0) / denom),
+        "rms": rms,
+        "ok": bool(relF <= 4e-3 and excess.max(initial=0.0) <= 1.5e-2 * denom),
+    }
+
+
+# --------------------------------------------------------------------------
+# RTN quantization (R3)
+# --------------------------------------------------------------------------
+
+def _check_packable(w: np.ndarray) -> None:
+    if not np.all(np.isfinite(w)):
+        raise ValueError("non-finite weight")
+    if np.any(np.abs(w) > F16_MAX):
+        raise ValueError("weight magnitude beyond the f16 range")
+
+
+def nearest_codes(w32, scale16, bias16) -> np.ndarray:
+    """q = clamp(round_half_even(RN32(RN32(w - b) / s)), 0, 15) per group; 0 where s == 0.
+
+    w32 float32 [N][G][64]; scale16, bias16 float16 [N][G].
+    """
+    s = scale16.astype(np.float32)[..., None]
+    b = bias16.astype(np.float32)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (w32 - b) / np.where(s == 0, np.float32(1), s)      # float32 subtract and divide
+    q = np.clip(np.rint(t), 0, 15)
+    q = np.where(s == 0, 0, q)
+    return q.astype(np.int64)
+
+
+def pack_rtn(w):
+    """Min/max round-to-nearest quantization of float32 W [N][K] -> (codes, scales f16, biases f16)."""
+    w = np.asarray(w, dtype=np.float32)
+    N, K = w.shape
+    assert K % GROUP == 0
+    _check_packable(w)
+    g = w.reshape(N, K // GROUP, GROUP)
+    mn = g.min(axis=-1)
+    mx = g.max(axis=-1)
+    s32 = (mx - mn) / np.float32(15.0)                            # float32: RN32(RN32(mx - mn) / 15)
+    scale16 = s32.astype(np.float16)
+    bias16 = mn.astype(np.float16)
+    q = nearest_codes(g, scale16, bias16)
+    return pack_codes(q.reshape(N, K)), scale16, bias16
+
+
+# --------------------------------------------------------------------------
+# Importance-weighted fit (R4)
+# --------------------------------------------------------------------------
+
+def imatrix_from_x(x_bits) -> np.ndarray:
+    """Per-input-channel mean squared activation E[x_j^2] over the rows of x, float64."""
+    x = decode_bf16(x_bits)
+    return np.mean(x * x, axis=0)
+
+
+def group_weighted_error(w, codes, scales, biases, imp) -> np.ndarray:
+    """E[n][g] = sum_{j in g} imp_j * (w_j - deq_j)^2 in float64, deq the fp32 dequant."""
+    w = np.asarray(w, dtype=np.float64)
+    N, K = w.shape
+    deq = dequant_f32(codes, scales, biases).astype(np.float64)
+    d2 = (w - deq) ** 2 * np.asarray(imp, dtype=np.float64)[None, :]
+    return d2.reshape(N, K // GROUP, GROUP).sum(axis=-1)
+
+
+FIT_SHRINK = tuple(0.025 * i for i in range(9))   # 0, 0.025, ..., 0.2
+FIT_REFITS = 2
+
+
+def pack_imatrix(w, imatrix, row_chunk: int = 256):
+    """Importance-weighted least-squares group fit, searched with RTN as candidate 0.
+
+    Objective per group: E = sum_j imp_j * (w_j - deq_j)^2 (float64), deq the fp32
+    dequant of the stored f16 triple.  imp = imatrix + 1e-6 * mean(imatrix), so a
+    channel no activation reached still counts a little.  imatrix None -> RTN.
+
+    Candidates, in order:
+      0   the RTN triple (pack_rtn);
+      1.. for each range shrink (a, b) in FIT_SHRINK^2 without (0, 0), in row-major
+          order: lo = mn + a*r, hi = mx - b*r (r = mx - mn, float64),
+          scale = RN_f16((hi - lo)/15), bias = RN_f16(lo), codes nearest (R3 rule);
+          then FIT_REFITS rounds of: weighted least squares for (s, b) with the codes
+          fixed (2x2 normal equations, float64; stop when the system is singular or
+          s <= 0), scale = RN_f16(s), bias = RN_f16(b), codes re-chosen nearest.
+    Every visited triple is scored; the lowest E wins, ties to the lowest index.
+    For fixed (s, b) the nearest code is optimal for any imp >= 0 because the
+    objective is a sum of independent non-negative terms.
+    """
+    w = np.asarray(w, dtype=np.float32)
+    if imatrix is None:
+        return pack_rtn(w)
+    N, K = w.shape
+    _check_packable(w)
+    imp = np.asarray(imatrix, dtype=np.float64)
+    imp = imp + 1e-6 * imp.mean()
+    codes = np.empty((N, K // 8), dtype=np.uint32)
+    scales = np.empty((N, K // GROUP), dtype=np.float16)
+    biases = np.empty((N, K // GROUP), dtype=np.float16)
+    for r0 in range(0, N, row_chunk):
+        r1 = min(N, r0 + row_chunk)
+        c, s, b = _fit_rows(w[r0:r1], imp)
+        codes[r0:r1], scales[r0:r1], biases[r0:r1] = c, s, b
+    return codes, scales, biases
+
+
+def _score(g64, imp_g, q, s16, b16):
+    """Weighted error of the triple (q, s16, b16) per group; deq = RN32(s*q + b)."""
+    deq = (s16.astype(np.float64)[..., None] * q + b16.astype(np.float64)[..., None]).astype(np.float32)
+    return np.sum(imp_g * (g64 - deq.astype(np.float64)) ** 2, axis=-1)
+
+
+def _fit_rows(w, imp):
+    n, K = w.shape
+    G = K // GROUP
+    g32 = w.reshape(n, G, GROUP)
+    g64 = g32.astype(np.float64)
+    imp_g = imp.reshape(1, G, GROUP)
+
+    c0, s0, b0 = pack_rtn(w)
+    best_q = unpack_codes(c0, K).reshape(n, G, GROUP)
+    best_s, best_b = s0.copy(), b0.copy()
+    best_e = _score(g64, imp_g, best_q, best_s, best_b)
+
+    def consider(q, s16, b16):
+        nonlocal best_q, best_s, best_b, best_e
+        e = _score(g64, imp_g, q, s16, b16)
+        better = e < best_e                      # strict: ties keep the earlier candidate
+        best_e = np.where(better, e, best_e)
+        best_s = np.where(better, s16, best_s)
+        best_b = np.where(better, b16, best_b)
+        best_q = np.where(better[..., None], q, best_q)
+
+    mn = g64.min(axis=-1)
+    mx = g64.max(axis=-1)
+    r = mx - mn
+    sw = imp_g.sum(axis=-1)                                 # sum imp
+    swx = (imp_g * g64).sum(axis=-1)                        # sum imp * w
+    for a in FIT_SHRINK:
+        for bb in FIT_SHRINK:
+            if a == 0 and bb == 0:
+                continue
+            lo = mn + a * r
+            hi = mx - bb * r
+            s16 = ((hi - lo) / 15.0).astype(np.float16)
+            b16 = lo.astype(np.float16)
+            q = nearest_codes(g32, s16, b16)
+            consider(q, s16, b16)
+            active = np.ones(s16.shape, dtype=bool)
+            for _ in range(FIT_REFITS):
+                qf = q.astype(np.float64)
+                swq = (imp_g * qf).sum(axis=-1)
+                swqq = (imp_g * qf * qf).sum(axis=-1)
+                swqx = (imp_g * qf * g64).sum(axis=-1)
+                det = swqq * sw - swq * swq
+                ok = active & (np.abs(det) > 1e-12 * np.maximum(swqq * sw, 1e-300))
+                with np.errstate(divide="ignore", invalid="ignore"):
+                    s_ls = (swqx * sw - swq * swx) / det
+                    b_ls = (swqq * swx - swq * swqx) / det
+                ok &= np.isfinite(s_ls) & np.isfinite(b_ls) & (s_ls > 0)
+                ok &= (np.abs(s_ls) <= F16_MAX) & (np.abs(b_ls) <= F16_MAX)
+                active = ok
+                if not ok.any():
+                    break
+                s_new = np.where(ok, s_ls, s16.astype(np.float64)).astype(np.float16)
+                b_new = np.where(ok, b_ls, b16.astype(np.float64)).astype(np.float16)
+                q_new = nearest_codes(g32, s_new, b_new)
+                s16 = np.where(ok, s_new, s16)
+                b16 = np.where(ok, b_new, b16)
+                q = np.where(ok[..., None], q_new, q)
+                e = _score(g64, imp_g, q, s16, b16)
+                better = ok & (e < best_e)
+                best_e = np.where(better, e, best_e)
+                best_s = np.where(better, s16, best_s)
+                best_b = np.where(better, b16, best_b)
+                best_q = np.where(better[..., None], q, best_q)
+    return pack_codes(best_q.reshape(n, K)), best_s.astype(np.float16), best_b.astype(np.float16)

@@ -1,0 +1,395 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Each test states what fixes the expected value: a library conversion, exact
+rational arithmetic, a closed form, brute force, or a number the pages print.
+"""
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import qlinear_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _random_layer(rng, M, K, N):
+    codes = rng.integers(0, 1 << 32, size=(N, K // 8), dtype=np.uint32)
+    s = np.exp(rng.uniform(np.log(1e-3), np.log(2e-2), size=(N, K // 64))).astype(np.float16)
+    b = (-7.5 * s.astype(np.float64) + 0.1 * s.astype(np.float64) * rng.standard_normal(s.shape)).astype(np.float16)
+    x = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(torch.bfloat16)
+    return x.view(torch.int16).numpy().view(np.uint16), codes, s, b
+
+
+# ---------------------------------------------------------------- decoding
+
+def test_decode_f16_all_patterns_match_numpy():
+    """All 65536 binary16 patterns: the bit-field decoder equals numpy's half->double conversion."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = O.decode_f16(bits)
+    lib = bits.view(np.float16).astype(np.float64)
+    both_nan = np.isnan(ours) & np.isnan(lib)
+    assert np.array_equal(ours[~both_nan], lib[~both_nan])
+    assert np.array_equal(np.isnan(ours), np.isnan(lib))
+
+
+def test_decode_bf16_all_patterns_match_torch():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = O.decode_bf16(bits)
+    lib = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    both_nan = np.isnan(ours) & np.isnan(lib)
+    assert np.array_equal(ours[~both_nan], lib[~both_nan])
+
+
+def test_round_bf16_from_f32_matches_torch():
+    """For binary32 inputs the oracle's bf16 rounding equals torch's float->bfloat16 cast."""
+    rng = _rng(1)
+    u = rng.integers(0, 1 << 32, size=200000, dtype=np.uint64).astype(np.uint32)
+    # include ties, near-ties and extremes
+    extra = np.array([0x3F808000, 0x3F818000, 0x3F80FFFF, 0x7F7FFFFF, 0x7F7F8000, 0x00000001,
+                      0x80000000, 0x00800000, 0x3F800000], dtype=np.uint32)
+    u = np.concatenate([u, extra])
+    f = u.view(np.float32)
+    finite = np.isfinite(f)
+    ours = O.round_bf16(f[finite].astype(np.float64))
+    lib = torch.from_numpy(f[finite]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, lib)
+
+
+def test_round_bf16_from_f64_is_nearest_with_ties_even():
+    """Brute force: compare with the nearer of the two bf16 neighbours (exact rationals)."""
+    rng = _rng(2)
+    v = rng.standard_normal(3000) * np.exp(rng.uniform(-20, 20, 3000))
+    got = O.decode_bf16(O.round_bf16(v))
+    for val, g in zip(v, got):
+        # neighbours: truncate the binary32 pattern of a value just below/above
+        f32 = np.float32(val)
+        cands = set()
+        for t in (np.nextafter(f32, np.float32(-np.inf)), f32, np.nextafter(f32, np.float32(np.inf))):
+            hi = (np.array([t], dtype=np.float32).view(np.uint32)[0] >> 16)
+            for d in (-1, 0, 1):
+                cands.add(int(hi) + d)
+        best = None
+        for c in sorted(cands):
+            cv = Fraction(float(O.decode_bf16(np.array([c & 0xFFFF]))[0]))
+            dist = abs(cv - Fraction(float(val)))
+            key = (dist, c & 1)           # ties: even significand
+            if best is None or key < best[0]:
+                best = (key, cv)
+        assert Fraction(float(g)) == best[1]
+
+
+def test_nibble_order_low_first():
+    """Reading R1: code k%8 sits in bits 4*(k%8)..; word 0x76543210 holds codes 0..7 in order."""
+    codes = np.array([[0x76543210, 0xFEDCBA98]], dtype=np.uint32)
+    q = O.unpack_codes(codes, 16)
+    assert q.tolist() == [list(range(16))]
+    assert np.array_equal(O.pack_codes(q), codes)
+
+
+def test_pack_unpack_roundtrip():
+    rng = _rng(3)
+    codes = rng.integers(0, 1 << 32, size=(7, 40), dtype=np.uint32)
+    assert np.array_equal(O.pack_codes(O.unpack_codes(codes, 320)), codes)
+
+
+def test_bits_per_weight_is_4_5_golden():
+    """Packed size = 4 bits/code + f16 scale + f16 bias per 64 = 4.5 bits/weight (the pages' figure)."""
+    g = json.load(open(os.path.join(GOLDEN, "format_constants.json")))
+    group = g["group_size"]["value"]
+    bpw = g["code_bits"]["value"] + g["overhead_bits_per_weight"]["value"]
+    K, N = 4608, 13824
+    w = np.zeros((N, K), dtype=np.float32)
+    w[:, ::2] = 1.0
+    codes, s, b = O.pack_rtn(w[:64])          # small pack: check the per-row layout sizes
+    assert codes.shape == (64, K // 8) and s.shape == (64, K // group) and b.shape == (64, K // group)
+    row_bytes = codes[0].nbytes + s[0].nbytes + b[0].nbytes
+    assert row_bytes * 8 == bpw * K
+    assert row_bytes * N == 35_831_808
+
+
+# ---------------------------------------------------------------- dequant
+
+def _edge_f16():
+    vals = [0x0000, 0x8000, 0x0001, 0x8001, 0x03FF, 0x0400, 0x3C00, 0xBC00, 0x7BFF, 0xFBFF,
+            0x1400, 0x2E66, 0xC000, 0x3555, 0x0200, 0x8200]
+    return np.array(vals, dtype=np.uint16)
+
+
+def test_dequant_exact_equals_rational_arithmetic():
+    """s*q + b computed with exact rationals equals dequant_exact for every code and edge f16 value."""
+    e = _edge_f16()
+    S, B = np.meshgrid(e, e, indexing="ij")
+    S = S.reshape(-1, 1)
+    B = B.reshape(-1, 1)
+    N = S.shape[0]
+    # one group per row, codes 0..15 repeated 4 times
+    q = np.tile(np.arange(16), 4)[None, :].repeat(N, 0)
+    codes = O.pack_codes(q)
+    got = O.dequant_exact(codes, S.view(np.float16), B.view(np.float16))
+    for n in range(N):
+        s = Fraction(float(np.array(S[n]).view(np.float16)[0]))
+        b = Fraction(float(np.array(B[n]).view(np.float16)[0]))
+        for k in range(16):
+            assert Fraction(float(got[n, k])) == s * k + b
+
+
+def test_dequant_f32_is_correctly_rounded():
+    """fp32 dequant = binary32 nearest (ties even) to the exact rational s*q + b."""
+    rng = _rng(4)
+    x, codes, s, b = _random_layer(rng, 1, 256, 64)
+    w32 = O.dequant_f32(codes, s, b)
+    q = O.unpack_codes(codes, 256)
+    for n in range(0, 64, 7):
+        for k in range(0, 256, 5):
+            exact = Fraction(float(s[n, k // 64])) * int(q[n, k]) + Fraction(float(b[n, k // 64]))
+            got = Fraction(float(w32[n, k]))
+            # neighbours of got in binary32
+            lo = Fraction(float(np.nextafter(w32[n, k], np.float32(-np.inf))))
+            hi = Fraction(float(np.nextafter(w32[n, k], np.float32(np.inf))))
+            assert abs(got - exact) <= abs(lo - exact) and abs(got - exact) <= abs(hi - exact)
+
+
+def test_dequant_bf16_is_bf16_of_f32_dequant():
+    rng = _rng(5)
+    _, codes, s, b = _random_layer(rng, 1, 128, 32)
+    w32 = O.dequant_f32(codes, s, b)
+    lib = torch.from_numpy(w32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.dequant_bf16(codes, s, b), lib)
+
+
+# ---------------------------------------------------------------- forward
+
+@pytest.mark.parametrize("M,K,N", [(1, 64, 8), (3, 128, 16), (16, 256, 40), (5, 192, 64)])
+def test_forward_equals_triple_loop(M, K, N):
+    rng = _rng(M * 1000 + K + N)
+    x, codes, s, b = _random_layer(rng, M, K, N)
+    y = O.forward_ref(x, codes, s, b)
+    yt = O.forward_triple_loop(x, codes, s, b)
+    xa = np.abs(O.decode_bf16(x))
+    wa = np.abs(O.dequant_f32(codes, s, b).astype(np.float64))
+    bound = 1e-14 * (xa @ wa.T) + 1e-300
+    assert np.all(np.abs(y - yt) <= bound)
+
+
+def test_forward_constant_codes_closed_form():
+    """All codes c, scale 1, bias 0 -> y[m][n] = c * sum_k x[m][k]."""
+    rng = _rng(6)
+    M, K, N = 4, 192, 16
+    x = _random_layer(rng, M, K, N)[0]
+    for c in (0, 1, 7, 15):
+        codes = O.pack_codes(np.full((N, K), c))
+        s = np.ones((N, K // 64), dtype=np.float16)
+        b = np.zeros((N, K // 64), dtype=np.float16)
+        y = O.forward_ref(x, codes, s, b)
+        xs = O.decode_bf16(x).sum(axis=1)
+        assert np.allclose(y, (c * xs)[:, None], rtol=1e-13, atol=1e-13)
+
+
+def test_forward_constant_codes_per_group_affine():
+    """Constant codes c per group with scale s_g, bias b_g -> y = sum_g (s_g*c + b_g) * sum_{k in g} x_k."""
+    rng = _rng(7)
+    M, K, N = 3, 256, 8
+    x = _random_layer(rng, M, K, N)[0]
+    s = np.array(rng.uniform(0.01, 0.1, (N, 4)), dtype=np.float16)
+    b = np.array(rng.uniform(-0.5, 0.5, (N, 4)), dtype=np.float16)
+    c = 11
+    codes = O.pack_codes(np.full((N, K), c))
+    y = O.forward_ref(x, codes, s, b)
+    xs = O.decode_bf16(x).reshape(M, 4, 64).sum(axis=2)        # [M][G]
+    w_g = s.astype(np.float64) * c + b.astype(np.float64)      # [N][G]
+    expect = xs @ w_g.T
+    assert np.allclose(y, expect, rtol=1e-12, atol=1e-12)
+
+
+def test_forward_one_hot_selects_weight_column():
+    """x = e_k -> y[:, n] = w(n, k) exactly, and its bf16 rounding is the bf16 dequant."""
+    rng = _rng(8)
+    K, N = 128, 24
+    _, codes, s, b = _random_layer(rng, 1, K, N)
+    one = np.uint16(0x3F80)     # bf16 1.0
+    x = np.zeros((K, K), dtype=np.uint16)
+    x[np.arange(K), np.arange(K)] = one
+    y = O.forward_ref(x, codes, s, b)
+    w32 = O.dequant_f32(codes, s, b)
+    assert np.array_equal(y, w32.T.astype(np.float64))
+    assert np.array_equal(O.round_bf16(y), O.dequant_bf16(codes, s, b).T)
+
+
+def test_forward_power_of_two_linearity_exact():
+    rng = _rng(9)
+    x, codes, s, b = _random_layer(rng, 4, 128, 16)
+    x2 = (x.astype(np.uint32) + (1 << 7)).astype(np.uint16)     # exponent + 1 -> 2x (no overflow here)
+    y1 = O.forward_ref(x, codes, s, b)
+    y2 = O.forward_ref(x2, codes, s, b)
+    assert np.array_equal(y2, 2.0 * y1)
+
+
+def test_forward_transposed_operand_would_fail():
+    """A non-square case distinguishes W from W^T: the brute-force loop indexes W[n][k] explicitly."""
+    rng = _rng(10)
+    x, codes, s, b = _random_layer(rng, 2, 64, 8)
+    y = O.forward_ref(x, codes, s, b)
+    assert y.shape == (2, 8)
+    w = O.dequant_f32(codes, s, b).astype(np.float64)
+    assert np.allclose(y[1, 3], np.dot(O.decode_bf16(x)[1], w[3]), rtol=1e-14)
+
+
+# ---------------------------------------------------------------- tolerance
+
+def test_half_ulp_bf16_values():
+    assert O.half_ulp_bf16(1.0) == 2.0 ** -8
+    assert O.half_ulp_bf16(1.99) == 2.0 ** -8
+    assert O.half_ulp_bf16(2.0) == 2.0 ** -7
+    assert O.half_ulp_bf16(-0.75) == 2.0 ** -9
+
+
+def test_tolerance_metrics_basic():
+    y_ref = np.array([1.0, -2.0, 3.0, 0.5])
+    t = O.tolerance(y_ref, y_ref)
+    assert t["relF"] == 0 and t["max_gate"] == 0 and t["ok"]
+    # exact result rounded to bf16 is always within the half-ulp allowance
+    rng = _rng(11)
+    r = rng.standard_normal(10000) * 3
+    yb = O.decode_bf16(O.round_bf16(r))
+    t = O.tolerance(yb, r)
+    assert t["max_gate"] == 0.0 and t["ok"]
+    bad = r * (1 + 1e-2)
+    assert not O.tolerance(bad, r)["ok"]
+
+
+# ---------------------------------------------------------------- RTN pack
+
+def _rtn_case(seed, N=16, K=256):
+    rng = _rng(seed)
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    return w
+
+
+def test_rtn_codes_are_nearest_grid_point():
+    """Brute force over the 16 grid points: each RTN code is (one of) the nearest."""
+    w = _rtn_case(12)
+    codes, s, b = O.pack_rtn(w)
+    N, K = w.shape
+    q = O.unpack_codes(codes, K)
+    sf = s.astype(np.float64)
+    bf = b.astype(np.float64)
+    for n in range(N):
+        for k in range(K):
+            g = k // 64
+            grid = sf[n, g] * np.arange(16) + bf[n, g]
+            d = np.abs(grid - float(w[n, k]))
+            assert d[q[n, k]] <= d.min() + 4e-7 * max(abs(float(w[n, k])), 1e-3)
+
+
+def test_rtn_reconstructs_group_extremes():
+    """Reading R3 bounds: deq(code of min) within half an f16 ulp of min; max within 15*ulp(s)/2 + ulp(min)/2."""
+    w = _rtn_case(13, N=32, K=512)
+    codes, s, b = O.pack_rtn(w)
+    deq = O.dequant_f32(codes, s, b).astype(np.float64).reshape(32, 8, 64)
+    g = w.astype(np.float64).reshape(32, 8, 64)
+
+    def half_ulp_f16(v):
+        _, e = np.frexp(np.abs(v))
+        return np.ldexp(1.0, np.maximum(e, -13) - 12)
+
+    i_min = g.argmin(-1)
+    i_max = g.argmax(-1)
+    mn = np.take_along_axis(g, i_min[..., None], -1)[..., 0]
+    mx = np.take_along_axis(g, i_max[..., None], -1)[..., 0]
+    d_min = np.take_along_axis(deq, i_min[..., None], -1)[..., 0]
+    d_max = np.take_along_axis(deq, i_max[..., None], -1)[..., 0]
+    eps = 2.0 ** -23 * np.maximum(np.abs(mn), np.abs(mx))
+    sf = s.astype(np.float64)
+    assert np.all(np.abs(d_min - mn) <= half_ulp_f16(mn) + eps)
+    assert np.all(np.abs(d_max - mx) <= 15 * half_ulp_f16(sf) + half_ulp_f16(mn) + eps)
+
+
+def test_rtn_constant_group():
+    w = np.full((2, 128), 0.3, dtype=np.float32)
+    w[1, 64:] = -1.25
+    codes, s, b = O.pack_rtn(w)
+    assert np.all(O.unpack_codes(codes, 128) == 0)
+    assert np.all(s == 0)
+    assert np.array_equal(O.dequant_f32(codes, s, b), np.repeat(b.astype(np.float32), 64, axis=1))
+
+
+def test_rtn_monotone_code_map():
+    w = _rtn_case(14, N=8, K=128)
+    codes, s, b = O.pack_rtn(w)
+    q = O.unpack_codes(codes, 128).reshape(8, 2, 64)
+    g = w.reshape(8, 2, 64)
+    for n in range(8):
+        for j in range(2):
+            order = np.argsort(g[n, j], kind="stable")
+            assert np.all(np.diff(q[n, j][order]) >= 0)
+
+
+def test_rtn_on_grid_group_is_exact():
+    """A group that already lies on an f16 affine grid spanning codes 0..15 is reproduced exactly."""
+    s = np.float16(0.0078125 * 1.25)
+    b = np.float16(-0.0625)
+    q = np.tile(np.arange(16), 4)
+    w = (np.float64(s) * q + np.float64(b)).astype(np.float32)[None, :]
+    codes, s2, b2 = O.pack_rtn(w)
+    assert s2[0, 0] == s and b2[0, 0] == b
+    assert np.array_equal(O.unpack_codes(codes, 64)[0], q)
+
+
+def test_rtn_rejects_non_finite_and_out_of_range():
+    w = np.zeros((1, 64), dtype=np.float32)
+    w[0, 3] = np.nan
+    with pytest.raises(ValueError):
+        O.pack_rtn(w)
+    w[0, 3] = 70000.0
+    with pytest.raises(ValueError):
+        O.pack_rtn(w)
+
+
+# ---------------------------------------------------------------- imatrix fit
+
+def test_fit_never_worse_than_rtn_per_group():
+    """The pages: RTN is candidate 0 of the search, so the fit is never worse by the weighted objective."""
+    rng = _rng(15)
+    N, K = 48, 512
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    x = torch.from_numpy((rng.standard_normal((64, K)) * np.exp(rng.standard_normal(K))).astype(np.float32))
+    xb = x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    imp = O.imatrix_from_x(xb)
+    cf, sf, bf = O.pack_imatrix(w, imp)
+    cr, sr, br = O.pack_rtn(w)
+    impr = imp + 1e-6 * imp.mean()
+    ef = O.group_weighted_error(w, cf, sf, bf, impr)
+    er = O.group_weighted_error(w, cr, sr, br, impr)
+    assert np.all(ef <= er)
+    assert ef.sum() < er.sum()          # the search does find better triples on Gaussian weights
+
+
+def test_fit_without_statistics_is_rtn():
+    w = _rtn_case(16)
+    a = O.pack_imatrix(w, None)
+    r = O.pack_rtn(w)
+    for u, v in zip(a, r):
+        assert np.array_equal(u, v)
+
+
+def test_fit_on_grid_group_has_zero_error():
+    s = np.float16(0.01)
+    b = np.float16(-0.07)
+    q = np.tile(np.arange(16), 4)
+    w = (np.float64(s) * q + np.float64(b)).astype(np.float32)[None, :]
+    imp = np.linspace(0.1, 3.0, 64)
+    c, s2, b2 = O.pack_imatrix(w, imp)
+    assert O.group_weighted_error(w, c, s2, b2, imp).max() == 0.0
+
+
+def test_imatrix_is_mean_square():
+    x = np.array([[0x3F80, 0x4000], [0xBF80, 0x0000]], dtype=np.uint16)   # [[1, 2], [-1, 0]]
+    assert np.array_equal(O.imatrix_from_x(x), np.array([1.0, 2.0]))
