@@ -1,0 +1,36 @@
+"""B200-native group-wise affine W4 g64 quantized linear layer.
+
+Python binding of the C ABI declared in include/qlinear.h: argument
+marshalling only.  Every step of the computation runs in the CUDA kernels of
+libqlinear.so; there is no CPU fallback and no other backend.  Importing this
+package does not load the library; the first call does, and fails loudly if
+the library is missing or no GPU is visible.
+
+Tensors follow the ABI layout:
+    x       torch.bfloat16 [M][K]
+    codes   torch.int32    [N][K/8]   (uint32 bit patterns, 8 codes per word, low nibble first)
+    scales  torch.float16  [N][K/64]
+    biases  torch.float16  [N][K/64]
+    y       torch.bfloat16 [M][N]     (y = x . W^T, W[n][k] = scale * code + bias)
+"""
+from __future__ import annotations
+
+from ._lib import (  # noqa: F401
+    GROUP,
+    PATH_AUTO,
+    PATH_GEMV,
+    PATH_TC_FUSED,
+    PATH_TC_SKINNY,
+    QLinearError,
+    STATUS,
+    dequant,
+    device_status,
+    forward,
+    last_dispatch,
+    lib,
+    library_path,
+    pack,
+    set_profile_events,
+    version,
+    workspace_size,
+)

@@ -1,0 +1,407 @@
+// C ABI of the qlinear library: argument validation, per-shape dispatch,
+// workspace layout, tensor-map encoding and launches.  Every kernel of the
+// library is included here so the whole library is one device module.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "ql_common.cuh"
+#include "ql_dequant.cuh"
+#include "ql_gemv.cuh"
+#include "ql_pack.cuh"
+#include "ql_prepass.cuh"
+#include "ql_tc_fused.cuh"
+
+namespace ql {
+namespace {
+
+constexpr int32_t kVersion = 100;   // 0.1.0
+constexpr int kMaxDevices = 64;
+
+thread_local char t_last_dispatch[192] = "none";
+thread_local cudaEvent_t t_prof_start = nullptr;
+thread_local cudaEvent_t t_prof_stop = nullptr;
+
+void prof_begin(cudaStream_t st) {
+    if (t_prof_start && t_prof_stop) cudaEventRecord(t_prof_start, st);
+}
+void prof_end(cudaStream_t st) {
+    if (t_prof_start && t_prof_stop) cudaEventRecord(t_prof_stop, st);
+}
+
+void set_dispatch(const char* fmt, ...) __attribute__((format(printf, 1, 2)));
+void set_dispatch(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_last_dispatch, sizeof(t_last_dispatch), fmt, ap);
+    va_end(ap);
+}
+
+struct DeviceInfo {
+    int sm_count = 0;
+    bool fused_attr_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+ql_status device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QL_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (d.sm_count == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return QL_ERR_CUDA;
+        d.sm_count = n;
+    }
+    if (!d.fused_attr_set) {
+        if (cudaFuncSetAttribute(fused::fused_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 fused::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(fused::fused_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 fused::kSmemBytes) != cudaSuccess) {
+            return QL_ERR_CUDA;
+        }
+        d.fused_attr_set = true;
+    }
+    *out = &d;
+    return QL_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+ql_status get_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+    std::call_once(g_encode_once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess) {
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        }
+    });
+    *fn = g_encode;
+    return g_encode ? QL_OK : QL_ERR_CUDA;
+}
+
+// 2-D row-major tensor map: inner extent `cols` elements, `rows` rows, row pitch in bytes.
+ql_status encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t cols, uint64_t rows,
+                    uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    if (get_encoder(&enc) != QL_OK) return QL_ERR_CUDA;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {pitch_bytes};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? QL_OK : QL_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return na > 0 && nb > 0 && x < y + nb && y < x + na;
+}
+
+ql_status launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ shapes and plans
+
+ql_status check_shape(int64_t M, int64_t K, int64_t N, int32_t group) {
+    if (group != kGroup) return QL_ERR_UNSUPPORTED;
+    if (M < 1 || K < kGroup || N < 8 || K % kGroup != 0 || N % 8 != 0) return QL_ERR_INVALID_ARG;
+    if (M > (1ll << 31) - 1 || K > (1ll << 30) || N > (1ll << 30)) return QL_ERR_INVALID_ARG;
+    return QL_OK;
+}
+
+struct Plan {
+    int path = QL_PATH_GEMV;
+    int split_k = 1;
+    size_t workspace = 0;
+    // fused path workspace carve-up
+    size_t off_xh = 0, off_rs = 0, off_sb = 0;
+};
+
+int auto_split(int64_t M, int64_t K, int64_t N, int sm_count) {
+    // Enough CTAs for ~4 waves of 8-row CTAs and K-slices of at least 4096.
+    const int64_t G = K / kGroup;
+    const int64_t ctas = N / kGemvWarps;
+    int s = 1;
+    while (ctas * s < 4 * sm_count && G / (2 * s) >= 64) s *= 2;
+    (void)M;
+    return s;
+}
+
+ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int sm_count, Plan* plan) {
+    const int64_t G = K / kGroup;
+    if (path == QL_PATH_AUTO) path = (M <= 64) ? QL_PATH_GEMV : QL_PATH_TC_FUSED;
+    plan->path = path;
+    if (path == QL_PATH_GEMV) {
+        int s = split_k > 0 ? split_k : auto_split(M, K, N, sm_count);
+        if (s > G || s > 65535) return QL_ERR_INVALID_ARG;
+        plan->split_k = s;
+        plan->workspace = s > 1 ? static_cast<size_t>(s) * M * N * sizeof(float) : 0;
+        return QL_OK;
+    }
+    if (path == QL_PATH_TC_FUSED) {
+        if (split_k > 1) return QL_ERR_UNSUPPORTED;
+        plan->split_k = 1;
+        plan->off_xh = 0;
+        plan->off_rs = round_up(static_cast<size_t>(M) * K * 2, 256);
+        plan->off_sb = plan->off_rs + round_up(static_cast<size_t>(M) * 4, 256);
+        plan->workspace = plan->off_sb + round_up(static_cast<size_t>(G) * N * 4, 256);
+        return QL_OK;
+    }
+    return QL_ERR_UNSUPPORTED;
+}
+
+// ------------------------------------------------------------------ launches
+
+ql_status run_gemv(const Plan& pl, const void* x, const uint32_t* codes, const void* scales, const void* biases,
+                   void* y, bool bf16_out, int64_t M, int64_t K, int64_t N, void* ws, cudaStream_t st,
+                   int sm_count) {
+    const dim3 grid(static_cast<unsigned>(N / kGemvWarps), static_cast<unsigned>(pl.split_k));
+    const bool partial = pl.split_k > 1;
+    void* out = partial ? ws : y;
+    auto xb = static_cast<const __nv_bfloat16*>(x);
+    auto sc = static_cast<const __half*>(scales);
+    auto bi = static_cast<const __half*>(biases);
+    prof_begin(st);
+    if (bf16_out)
+        gemv_kernel<true><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
+    else
+        gemv_kernel<false><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
+    prof_end(st);
+    if (partial) {
+        const int64_t count = M * N;
+        const int blocks = static_cast<int>(std::min<int64_t>((count / 4 + 255) / 256, 8 * sm_count));
+        if (bf16_out)
+            splitk_reduce_kernel<true><<<blocks, 256, 0, st>>>(static_cast<const float*>(ws), y, count, pl.split_k);
+        else
+            splitk_reduce_kernel<false><<<blocks, 256, 0, st>>>(static_cast<const float*>(ws), y, count, pl.split_k);
+    }
+    set_dispatch("path=gemv warps=%d splitk=%d launches=%d", kGemvWarps, pl.split_k, partial ? 2 : 1);
+    return launch_status();
+}
+
+ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const void* scales, const void* biases,
+                    void* y, bool bf16_out, int64_t M, int64_t K, int64_t N, void* ws, cudaStream_t st,
+                    int sm_count) {
+    const int64_t G = K / kGroup;
+    auto* base = static_cast<uint8_t*>(ws);
+    auto* xh = reinterpret_cast<__half*>(base + pl.off_xh);
+    auto* rs = reinterpret_cast<float*>(base + pl.off_rs);
+    auto* sb = reinterpret_cast<uint32_t*>(base + pl.off_sb);
+
+    CUtensorMap mx, mc, mp;
+    ql_status s;
+    if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xh, K, M, K * 2, fused::BK, fused::BM,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
+        return s;
+    if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K / 8, N, K / 2, fused::BK / 8, fused::BN,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+        return s;
+    if ((s = encode_2d(&mp, CU_TENSOR_MAP_DATA_TYPE_UINT32, sb, N, G, N * 4, fused::BN, 1,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+        return s;
+
+    convert_x_kernel<<<static_cast<unsigned>(M), kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), xh, rs,
+                                                                        static_cast<int>(K));
+    const dim3 tgrid(static_cast<unsigned>((G + 31) / 32), static_cast<unsigned>((N + 31) / 32));
+    transpose_params_kernel<<<tgrid, 256, 0, st>>>(static_cast<const __half*>(scales), static_cast<const __half*>(biases),
+                                                   sb, static_cast<int>(N), static_cast<int>(G));
+    fused::Params p;
+    p.rowscale = rs;
+    p.y = y;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.G = static_cast<int>(G);
+    p.num_m = static_cast<int>((M + fused::BM - 1) / fused::BM);
+    p.num_n = static_cast<int>((N + fused::BN - 1) / fused::BN);
+    const int tiles = p.num_m * p.num_n;
+    const int grid = std::min(tiles, sm_count);
+    prof_begin(st);
+    if (bf16_out)
+        fused::fused_gemm_kernel<true><<<grid, fused::kThreads, fused::kSmemBytes, st>>>(mx, mc, mp, p);
+    else
+        fused::fused_gemm_kernel<false><<<grid, fused::kThreads, fused::kSmemBytes, st>>>(mx, mc, mp, p);
+    prof_end(st);
+    set_dispatch("path=tc_fused tile=%dx%dx%d stages=%d/%d ctas=%d splitk=1 launches=3", fused::BM, fused::BN, fused::BK,
+                 fused::NS_T, fused::NS_B, grid);
+    (void)codes;
+    return launch_status();
+}
+
+ql_status forward_impl(const void* x, const uint32_t* codes, const void* scales, const void* biases, void* y,
+                       ql_dtype out_dtype, int64_t M, int64_t K, int64_t N, int32_t group, int32_t path,
+                       int32_t split_k, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    ql_status s = check_shape(M, K, N, group);
+    if (s != QL_OK) return s;
+    if (!x || !codes || !scales || !biases || !y) return QL_ERR_INVALID_ARG;
+    if (out_dtype != QL_BF16 && out_dtype != QL_F32) return QL_ERR_INVALID_ARG;
+    if (path < QL_PATH_AUTO || path > QL_PATH_TC_FUSED || split_k < 0) return QL_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(biases) || !aligned16(y))
+        return QL_ERR_ALIGNMENT;
+    const int64_t G = K / kGroup;
+    const size_t xb = static_cast<size_t>(M) * K * 2, cb = static_cast<size_t>(N) * K / 2,
+                 pb = static_cast<size_t>(N) * G * 2,
+                 yb = static_cast<size_t>(M) * N * (out_dtype == QL_BF16 ? 2 : 4);
+    if (overlap(y, yb, x, xb) || overlap(y, yb, codes, cb) || overlap(y, yb, scales, pb) || overlap(y, yb, biases, pb))
+        return QL_ERR_INVALID_ARG;
+    DeviceInfo* dev = nullptr;
+    if ((s = device_info(&dev)) != QL_OK) return s;
+    Plan pl;
+    if ((s = make_plan(M, K, N, path, split_k, dev->sm_count, &pl)) != QL_OK) return s;
+    if (pl.workspace > 0) {
+        if (!workspace || workspace_bytes < pl.workspace) return QL_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return QL_ERR_ALIGNMENT;
+        if (overlap(workspace, pl.workspace, x, xb) || overlap(workspace, pl.workspace, y, yb) ||
+            overlap(workspace, pl.workspace, codes, cb) || overlap(workspace, pl.workspace, scales, pb) ||
+            overlap(workspace, pl.workspace, biases, pb))
+            return QL_ERR_INVALID_ARG;
+    }
+    const bool bf16 = out_dtype == QL_BF16;
+    if (pl.path == QL_PATH_GEMV)
+        return run_gemv(pl, x, codes, scales, biases, y, bf16, M, K, N, workspace, stream, dev->sm_count);
+    return run_fused(pl, x, codes, scales, biases, y, bf16, M, K, N, workspace, stream, dev->sm_count);
+}
+
+size_t workspace_impl(int64_t M, int64_t K, int64_t N, int32_t group, int32_t path, int32_t split_k) {
+    if (check_shape(M, K, N, group) != QL_OK) return static_cast<size_t>(-1);
+    DeviceInfo* dev = nullptr;
+    int sms = 148;
+    if (device_info(&dev) == QL_OK) sms = dev->sm_count;
+    Plan pl;
+    if (make_plan(M, K, N, path, split_k, sms, &pl) != QL_OK) return static_cast<size_t>(-1);
+    return pl.workspace;
+}
+
+}  // namespace
+}  // namespace ql
+
+using namespace ql;
+
+extern "C" {
+
+size_t qlinear_workspace_size(int64_t M, int64_t K, int64_t N, int32_t group) {
+    return workspace_impl(M, K, N, group, QL_PATH_AUTO, 0);
+}
+
+size_t qlinear_workspace_size_config(int64_t M, int64_t K, int64_t N, int32_t group, int32_t path, int32_t split_k) {
+    return workspace_impl(M, K, N, group, path, split_k);
+}
+
+ql_status qlinear_forward(const void* x, const uint32_t* codes, const void* scales, const void* biases, void* y,
+                          int64_t M, int64_t K, int64_t N, int32_t group, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream) {
+    return forward_impl(x, codes, scales, biases, y, QL_BF16, M, K, N, group, QL_PATH_AUTO, 0, workspace,
+                        workspace_bytes, stream);
+}
+
+ql_status qlinear_forward_config(const void* x, const uint32_t* codes, const void* scales, const void* biases,
+                                 void* y, ql_dtype out_dtype, int64_t M, int64_t K, int64_t N, int32_t group,
+                                 int32_t path, int32_t split_k, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream) {
+    return forward_impl(x, codes, scales, biases, y, out_dtype, M, K, N, group, path, split_k, workspace,
+                        workspace_bytes, stream);
+}
+
+ql_status qlinear_dequant(const uint32_t* codes, const void* scales, const void* biases, int64_t K, int64_t N,
+                          int32_t group, void* out, ql_dtype out_dtype, cudaStream_t stream) {
+    ql_status s = check_shape(1, K, N, group);
+    if (s != QL_OK) return s;
+    if (!codes || !scales || !biases || !out) return QL_ERR_INVALID_ARG;
+    if (out_dtype != QL_BF16 && out_dtype != QL_F32) return QL_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(biases) || !aligned16(out)) return QL_ERR_ALIGNMENT;
+    const int64_t G = K / kGroup;
+    const size_t ob = static_cast<size_t>(N) * K * (out_dtype == QL_BF16 ? 2 : 4);
+    if (overlap(out, ob, codes, static_cast<size_t>(N) * K / 2) || overlap(out, ob, scales, static_cast<size_t>(N) * G * 2) ||
+        overlap(out, ob, biases, static_cast<size_t>(N) * G * 2))
+        return QL_ERR_INVALID_ARG;
+    DeviceInfo* dev = nullptr;
+    if ((s = device_info(&dev)) != QL_OK) return s;
+    const int64_t words = N * K / 8;
+    const int blocks = static_cast<int>(std::min<int64_t>((words + 255) / 256, 16 * dev->sm_count));
+    auto sc = static_cast<const __half*>(scales);
+    auto bi = static_cast<const __half*>(biases);
+    if (out_dtype == QL_BF16)
+        dequant_kernel<true><<<blocks, 256, 0, stream>>>(codes, sc, bi, out, words);
+    else
+        dequant_kernel<false><<<blocks, 256, 0, stream>>>(codes, sc, bi, out, words);
+    return launch_status();
+}
+
+ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group, uint32_t* codes,
+                       void* scales, void* biases, cudaStream_t stream) {
+    ql_status s = check_shape(1, K, N, group);
+    if (s != QL_OK) return s;
+    if (!w || !codes || !scales || !biases) return QL_ERR_INVALID_ARG;
+    if (imatrix != nullptr) return QL_ERR_UNSUPPORTED;
+    if (!aligned16(w) || !aligned16(codes) || !aligned16(scales) || !aligned16(biases)) return QL_ERR_ALIGNMENT;
+    const int64_t G = K / kGroup;
+    const size_t wb = static_cast<size_t>(N) * K * 4, cb = static_cast<size_t>(N) * K / 2,
+                 pb = static_cast<size_t>(N) * G * 2;
+    if (overlap(w, wb, codes, cb) || overlap(w, wb, scales, pb) || overlap(w, wb, biases, pb) ||
+        overlap(codes, cb, scales, pb) || overlap(codes, cb, biases, pb) || overlap(scales, pb, biases, pb))
+        return QL_ERR_INVALID_ARG;
+    DeviceInfo* dev = nullptr;
+    if ((s = device_info(&dev)) != QL_OK) return s;
+    const int64_t groups = N * G;
+    const int blocks = static_cast<int>(std::min<int64_t>((groups + 7) / 8, 32 * dev->sm_count));
+    pack_rtn_kernel<<<blocks, 256, 0, stream>>>(w, codes, static_cast<__half*>(scales), static_cast<__half*>(biases),
+                                                groups);
+    return launch_status();
+}
+
+ql_status qlinear_get_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return QL_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return QL_ERR_CUDA;
+    const unsigned int zero = 0;
+    if (v != 0 && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return QL_ERR_CUDA;
+    return static_cast<ql_status>(v);
+}
+
+ql_status qlinear_last_dispatch(char* buf, size_t len) {
+    if (!buf || len == 0) return QL_ERR_INVALID_ARG;
+    std::strncpy(buf, t_last_dispatch, len - 1);
+    buf[len - 1] = '\0';
+    return QL_OK;
+}
+
+ql_status qlinear_set_profile_events(cudaEvent_t start, cudaEvent_t stop) {
+    if ((start == nullptr) != (stop == nullptr)) return QL_ERR_INVALID_ARG;
+    t_prof_start = start;
+    t_prof_stop = stop;
+    return QL_OK;
+}
+
+const char* qlinear_status_string(ql_status status) {
+    switch (status) {
+        case QL_OK: return "QL_OK";
+        case QL_ERR_INVALID_ARG: return "QL_ERR_INVALID_ARG";
+        case QL_ERR_ALIGNMENT: return "QL_ERR_ALIGNMENT";
+        case QL_ERR_UNSUPPORTED: return "QL_ERR_UNSUPPORTED";
+        case QL_ERR_WORKSPACE: return "QL_ERR_WORKSPACE";
+        case QL_ERR_CUDA: return "QL_ERR_CUDA";
+        case QL_ERR_DEVICE_TIMEOUT: return "QL_ERR_DEVICE_TIMEOUT";
+        case QL_ERR_BOUNDS: return "QL_ERR_BOUNDS";
+    }
+    return "QL_ERR_UNKNOWN";
+}
+
+int32_t qlinear_version(void) { return kVersion; }
+
+}  // extern "C"

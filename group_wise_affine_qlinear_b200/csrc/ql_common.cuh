@@ -1,0 +1,46 @@
+// Shared device helpers of the qlinear library: status word, bounded waits,
+// conversions.  Everything here is compiled into one translation unit
+// (ql_api.cu includes every kernel header), so the status word below is a
+// single per-device object.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/qlinear.h"
+
+namespace ql {
+
+constexpr int kGroup = 64;
+
+// First error recorded by any kernel since the host last read it (0 = none).
+__device__ unsigned int g_device_status;
+
+__device__ __forceinline__ void record_status(unsigned int code) {
+    atomicCAS(&g_device_status, 0u, code);
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Every wait on another thread, warp or async unit gives up after this long,
+// records QL_ERR_DEVICE_TIMEOUT and lets the kernel unwind.
+constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;   // 1 s
+
+__device__ __forceinline__ uint32_t bits_of(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 half2_of(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+}  // namespace ql

@@ -1,0 +1,103 @@
+// Operand preparation for the fused tensor-core path (large M).
+//
+// 1) Activations: bf16 x[M][K] -> f16 xh[M][K] * 2^-e_m with one power of two
+//    per row chosen from the row's max |x| so that the largest magnitude lands
+//    in [2^15, 2^16) below the f16 maximum.  A bf16 value (8 significant bits)
+//    scaled by a power of two is exactly representable in f16 whenever it stays
+//    in the f16 normal range; only entries more than ~2^29 below the row
+//    maximum are rounded (to f16 subnormals).  rowscale[m] = 2^e_m undoes the
+//    scaling in the epilogue.  Within every 8 consecutive k the f16 copy is
+//    stored in the order (0,4,1,5,2,6,3,7), which matches the order the
+//    dequantizer produces code pairs in (codes j and j+4 share one 32-bit
+//    word); permuting both operands alike leaves every dot product unchanged.
+// 2) Group parameters: scales/biases [N][G] -> sb[G][N] of (scale, bias) f16
+//    pairs, so one K-step's parameters for a run of N rows are contiguous and
+//    can be fetched by the tensor memory accelerator.
+#pragma once
+
+#include "ql_common.cuh"
+
+namespace ql {
+
+constexpr int kPrepThreads = 256;
+
+// One CTA per row.  Pass 1 reads the row for max|x|, pass 2 re-reads (L2) and converts.
+__global__ void __launch_bounds__(kPrepThreads) convert_x_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                 __half* __restrict__ xh,
+                                                                 float* __restrict__ rowscale, int K) {
+    __shared__ float red[kPrepThreads / 32];
+    __shared__ int row_exp;
+    const int64_t m = blockIdx.x;
+    const uint4* src = reinterpret_cast<const uint4*>(x + m * K);   // 8 bf16 per uint4
+    uint4* dst = reinterpret_cast<uint4*>(xh + m * K);
+    const int n8 = K / 8;
+
+    float amax = 0.0f;
+    for (int i = threadIdx.x; i < n8; i += kPrepThreads) {
+        const uint4 v = __ldg(src + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            // bit-level |.|: NaN patterns compare above every finite value
+            amax = fmaxf(amax, fabsf(bf16_lo(w[j])));
+            amax = fmaxf(amax, fabsf(bf16_hi(w[j])));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float a = red[0];
+        for (int i = 1; i < kPrepThreads / 32; ++i) a = fmaxf(a, red[i]);
+        int e = 0;                         // zero, inf or nan rows: no scaling
+        if (a > 0.0f && a <= 3.4028235e38f) {
+            const int ea = static_cast<int>((__float_as_uint(a) >> 23) & 0xFF) - 127;   // floor(log2 a), a normal
+            e = max(ea, -100) - 15;
+        }
+        row_exp = e;
+        rowscale[m] = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);    // 2^e, e in [-115, 112]
+    }
+    __syncthreads();
+    const float inv = __uint_as_float(static_cast<uint32_t>(127 - row_exp) << 23);   // 2^-e, exact
+    for (int i = threadIdx.x; i < n8; i += kPrepThreads) {
+        const uint4 v = __ldg(src + i);
+        // source order 0..7 = (v.x lo, v.x hi, v.y lo, v.y hi, v.z lo, v.z hi, v.w lo, v.w hi)
+        const float f0 = bf16_lo(v.x) * inv, f1 = bf16_hi(v.x) * inv;
+        const float f2 = bf16_lo(v.y) * inv, f3 = bf16_hi(v.y) * inv;
+        const float f4 = bf16_lo(v.z) * inv, f5 = bf16_hi(v.z) * inv;
+        const float f6 = bf16_lo(v.w) * inv, f7 = bf16_hi(v.w) * inv;
+        uint4 o;
+        o.x = bits_of(__floats2half2_rn(f0, f4));
+        o.y = bits_of(__floats2half2_rn(f1, f5));
+        o.z = bits_of(__floats2half2_rn(f2, f6));
+        o.w = bits_of(__floats2half2_rn(f3, f7));
+        dst[i] = o;
+    }
+}
+
+// sb[g][n] = (scale[n][g], bias[n][g]); 32x32 tiles through shared memory.
+__global__ void __launch_bounds__(256) transpose_params_kernel(const __half* __restrict__ scales,
+                                                               const __half* __restrict__ biases,
+                                                               uint32_t* __restrict__ sb, int N, int G) {
+    __shared__ uint32_t tile[32][33];
+    const int g0 = blockIdx.x * 32, n0 = blockIdx.y * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;     // 8 rows per pass
+    for (int r = ty; r < 32; r += 8) {
+        const int n = n0 + r, g = g0 + tx;
+        uint32_t v = 0;
+        if (n < N && g < G) {
+            const int64_t i = static_cast<int64_t>(n) * G + g;
+            v = static_cast<uint32_t>(__half_as_ushort(scales[i])) |
+                (static_cast<uint32_t>(__half_as_ushort(biases[i])) << 16);
+        }
+        tile[r][tx] = v;
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {
+        const int g = g0 + r, n = n0 + tx;
+        if (g < G && n < N) sb[static_cast<int64_t>(g) * N + n] = tile[tx][r];
+    }
+}
+
+}  // namespace ql

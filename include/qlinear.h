@@ -41,6 +41,12 @@
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
+#if defined(__GNUC__)
+#define QL_API __attribute__((visibility("default")))
+#else
+#define QL_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -72,7 +78,7 @@ typedef enum {
  * Bytes of device workspace qlinear_forward() needs for this shape (0 is
  * possible).  Returns (size_t)-1 when the shape is invalid.
  */
-size_t qlinear_workspace_size(int64_t M, int64_t K, int64_t N, int32_t group);
+QL_API size_t qlinear_workspace_size(int64_t M, int64_t K, int64_t N, int32_t group);
 
 /*
  * y = x . W^T for the packed W (the layer the pages describe: bf16
@@ -82,7 +88,7 @@ size_t qlinear_workspace_size(int64_t M, int64_t K, int64_t N, int32_t group);
  * and must not overlap any tensor.  The dispatcher picks the kernel path from
  * (M, K, N); qlinear_last_dispatch() reports the choice.
  */
-ql_status qlinear_forward(const void* x, const uint32_t* codes, const void* scales,
+QL_API ql_status qlinear_forward(const void* x, const uint32_t* codes, const void* scales,
                           const void* biases, void* y, int64_t M, int64_t K, int64_t N,
                           int32_t group, void* workspace, size_t workspace_bytes,
                           cudaStream_t stream);
@@ -90,19 +96,20 @@ ql_status qlinear_forward(const void* x, const uint32_t* codes, const void* scal
 /*
  * qlinear_forward with the path and split-K factor forced (testing and tuning).
  * path: a ql_path; split_k: 0 = the dispatcher's choice, else the number of K
- * slices (must divide K/64 into non-empty slices; QL_ERR_INVALID_ARG otherwise).
+ * slices, 1 <= split_k <= K/64 (QL_ERR_INVALID_ARG otherwise); slice z covers the
+ * groups [z*G/split_k, (z+1)*G/split_k), G = K/64.
  * out_dtype: QL_BF16 = the layer's output; QL_F32 writes y as fp32 [M][N]
  * (the same arithmetic without the final rounding, for numerical tests).
  * A path that cannot run the shape returns QL_ERR_UNSUPPORTED.
  */
-ql_status qlinear_forward_config(const void* x, const uint32_t* codes, const void* scales,
+QL_API ql_status qlinear_forward_config(const void* x, const uint32_t* codes, const void* scales,
                                  const void* biases, void* y, ql_dtype out_dtype,
                                  int64_t M, int64_t K, int64_t N, int32_t group,
                                  int32_t path, int32_t split_k,
                                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Workspace bytes for qlinear_forward_config() with the same path and split_k. */
-size_t qlinear_workspace_size_config(int64_t M, int64_t K, int64_t N, int32_t group,
+QL_API size_t qlinear_workspace_size_config(int64_t M, int64_t K, int64_t N, int32_t group,
                                      int32_t path, int32_t split_k);
 
 /*
@@ -110,7 +117,7 @@ size_t qlinear_workspace_size_config(int64_t M, int64_t K, int64_t N, int32_t gr
  * to bf16 (nearest even) when out_dtype == QL_BF16.  Bit-exact by definition:
  * s*q + b is formed with one fused multiply-add.  out is [N][K] of out_dtype.
  */
-ql_status qlinear_dequant(const uint32_t* codes, const void* scales, const void* biases,
+QL_API ql_status qlinear_dequant(const uint32_t* codes, const void* scales, const void* biases,
                           int64_t K, int64_t N, int32_t group, void* out, ql_dtype out_dtype,
                           cudaStream_t stream);
 
@@ -126,7 +133,7 @@ ql_status qlinear_dequant(const uint32_t* codes, const void* scales, const void*
  * A group holding a non-finite value or |w| > 65504 is written as codes 0,
  * scale 0, bias 0, and the device status word records QL_ERR_INVALID_ARG.
  */
-ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group,
+QL_API ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group,
                        uint32_t* codes, void* scales, void* biases, cudaStream_t stream);
 
 /*
@@ -134,20 +141,30 @@ ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t 
  * (the first error a kernel recorded since the last read).  Returns QL_OK when
  * no kernel recorded anything, QL_ERR_CUDA if the synchronization fails.
  */
-ql_status qlinear_get_device_status(cudaStream_t stream);
+QL_API ql_status qlinear_get_device_status(cudaStream_t stream);
 
 /*
  * Writes a NUL-terminated description of the calling thread's last
- * qlinear_forward dispatch ("path=tc_fused tile=128x256 stages=4 splitk=1"),
+ * qlinear_forward dispatch, e.g. "path=tc_fused tile=128x256x64 stages=4/3 ctas=148
+ * splitk=1 launches=3" (launches = kernels that call enqueued),
  * truncated to len bytes.  QL_ERR_INVALID_ARG if buf is NULL or len == 0.
  */
-ql_status qlinear_last_dispatch(char* buf, size_t len);
+QL_API ql_status qlinear_last_dispatch(char* buf, size_t len);
+
+/*
+ * Measurement hook.  While set (both non-NULL), every qlinear_forward* call
+ * made by the calling thread records `start` on its stream immediately before
+ * its main kernel (the tensor-core GEMM or the weight-streaming kernel) and
+ * `stop` immediately after it, so the main kernel can be timed alone.  The
+ * caller owns both events; NULL, NULL turns the hook off.  Thread-local.
+ */
+QL_API ql_status qlinear_set_profile_events(cudaEvent_t start, cudaEvent_t stop);
 
 /* Static, human-readable name of a status code. */
-const char* qlinear_status_string(ql_status status);
+QL_API const char* qlinear_status_string(ql_status status);
 
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
-int32_t qlinear_version(void);
+QL_API int32_t qlinear_version(void);
 
 #ifdef __cplusplus
 }

@@ -147,6 +147,14 @@ def round_bf16(v) -> np.ndarray:
     return (r32.view(np.uint32) >> 16).astype(np.uint16)
 
 
+def dequant_f16(codes, scales, biases) -> np.ndarray:
+    """RN_f16 of the exact s*q + b (one rounding; numpy's float64->float16 cast rounds to nearest even).
+
+    The precision of the weight operand of the tensor-core path for large M.
+    """
+    return dequant_exact(codes, scales, biases).astype(np.float16)
+
+
 def dequant_bf16(codes, scales, biases) -> np.ndarray:
     """bf16 dequant = RN_bf16(fp32 dequant) as uint16 bits (the fp32 value is rounded again)."""
     return round_bf16(dequant_f32(codes, scales, biases).astype(np.float64))

@@ -1,0 +1,113 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point the header declares, and rejects bad arguments before any
+launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import group_wise_affine_qlinear_b200 as ql
+from group_wise_affine_qlinear_b200 import build as qb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    qb.build()
+    return ql.lib()
+
+
+def _declared():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            txt = open(os.path.join(inc, f)).read()
+            names += re.findall(r"QL_API\s+[\w\s\*]+?\b(qlinear_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for n in ("qlinear_forward", "qlinear_dequant", "qlinear_pack", "qlinear_workspace_size"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in _declared():
+        assert hasattr(L, n), n
+
+
+def test_version_and_status_strings(L):
+    assert ql.version() == 100
+    for code, name in ql.STATUS.items():
+        assert L.qlinear_status_string(code).decode() == name
+    assert L.qlinear_status_string(99).decode() == "QL_ERR_UNKNOWN"
+
+
+def test_last_dispatch_buffer_checks(L):
+    assert L.qlinear_last_dispatch(None, 10) == 1
+    buf = ctypes.create_string_buffer(4)
+    assert L.qlinear_last_dispatch(buf, 4) == 0
+    assert len(buf.value) <= 3
+
+
+FAKE = 0x10000000          # never dereferenced: validation rejects before any launch
+
+
+def _fwd(L, x=FAKE, c=FAKE + (1 << 24), s=FAKE + (2 << 24), b=FAKE + (3 << 24), y=FAKE + (4 << 24),
+         M=16, K=256, N=256, group=64):
+    return L.qlinear_forward(x, c, s, b, y, M, K, N, group, None, 0, None)
+
+
+def test_forward_rejects_bad_shapes(L):
+    assert _fwd(L, group=32) == 3
+    assert _fwd(L, group=128) == 3
+    assert _fwd(L, K=100) == 1
+    assert _fwd(L, K=0) == 1
+    assert _fwd(L, N=12) == 1
+    assert _fwd(L, M=0) == 1
+    assert _fwd(L, M=-3) == 1
+
+
+def test_forward_rejects_null_and_misaligned(L):
+    assert _fwd(L, x=0) == 1
+    assert _fwd(L, y=0) == 1
+    assert _fwd(L, c=FAKE + (1 << 24) + 4) == 2
+    assert _fwd(L, x=FAKE + 2) == 2
+
+
+def test_forward_rejects_output_aliasing(L):
+    assert _fwd(L, y=FAKE) == 1                     # y over x
+    assert _fwd(L, y=FAKE + (1 << 24) + 64) == 1    # y inside codes
+
+
+def test_forward_config_rejects_bad_path(L):
+    r = L.qlinear_forward_config(FAKE, FAKE + (1 << 24), FAKE + (2 << 24), FAKE + (3 << 24), FAKE + (4 << 24),
+                                 1, 16, 256, 256, 64, 9, 0, None, 0, None)
+    assert r == 1
+
+
+def test_dequant_and_pack_validation(L):
+    assert L.qlinear_dequant(FAKE, FAKE + (1 << 24), FAKE + (2 << 24), 256, 256, 32, FAKE + (3 << 24), 0, None) == 3
+    assert L.qlinear_dequant(FAKE, FAKE + (1 << 24), FAKE + (2 << 24), 256, 256, 64, FAKE, 0, None) == 1
+    assert L.qlinear_dequant(FAKE + 8, FAKE + (1 << 24), FAKE + (2 << 24), 256, 256, 64, FAKE + (3 << 24), 0, None) == 2
+    assert L.qlinear_pack(FAKE, FAKE, 256, 256, 64, FAKE + (1 << 24), FAKE + (2 << 24), FAKE + (3 << 24), None) == 3
+    assert L.qlinear_pack(FAKE, None, 256, 256, 64, FAKE, FAKE + (2 << 24), FAKE + (3 << 24), None) == 1
+
+
+def test_workspace_size_values(L):
+    # fused path: f16 activations + row scales + transposed (scale, bias) pairs, 256-byte aligned pieces
+    M, K, N = 4608, 4608, 13824
+    ws = ql.workspace_size(M, K, N, ql.PATH_TC_FUSED)
+    assert ws == M * K * 2 + M * 4 + (K // 64) * N * 4
+    assert ql.workspace_size(1, 4096, 64, ql.PATH_GEMV, 1) == 0
+    assert ql.workspace_size(2, 4096, 64, ql.PATH_GEMV, 4) == 4 * 2 * 64 * 4
+    assert L.qlinear_workspace_size(16, 100, 256, 64) == ctypes.c_size_t(-1).value
+
+
+def test_profile_events_pairing(L):
+    assert L.qlinear_set_profile_events(FAKE, None) == 1
+    assert L.qlinear_set_profile_events(None, None) == 0

@@ -1,0 +1,272 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle.
+
+Bit-exact where the result is integer or defined by a single rounding
+(dequant, RTN pack, one-hot forward); within the tolerance of reading R5
+(relative Frobenius <= 4e-3, half-ulp-adjusted max error <= 1.5e-2 * rms)
+for the forward pass.
+"""
+import numpy as np
+import pytest
+import torch
+
+import group_wise_affine_qlinear_b200 as ql
+from group_wise_affine_qlinear_b200 import synthetic as S
+from oracle import qlinear_oracle as O
+
+from ._helpers import bf16_bits, random_layer, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"gemv": ql.PATH_GEMV, "tc_fused": ql.PATH_TC_FUSED}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA GPU required for -m gpu tests")
+    ql.lib()
+    yield
+    assert ql.device_status() == 0
+
+
+def _dev(codes, s, b):
+    return to_dev_codes(codes), to_dev_f16(s), to_dev_f16(b)
+
+
+def _check_tol(y_dev, y_ref, bf16=True, limit_relF=4e-3, limit_max=1.5e-2):
+    y = O.decode_bf16(bf16_bits(y_dev)) if bf16 else y_dev.double().cpu().numpy()
+    t = O.tolerance(y, y_ref, bf16_output=bf16)
+    assert t["relF"] <= limit_relF and t["max_gate"] <= limit_max, t
+    return t
+
+
+# ------------------------------------------------------------------ dequant
+
+@pytest.mark.parametrize("name", ["tiny", "qkv"])
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+def test_dequant_bitexact(name, dt):
+    codes, s, b = S.WORKLOADS[name].w()
+    out = ql.dequant(*_dev(codes, s, b), out_dtype=dt)
+    torch.cuda.synchronize()
+    if dt == torch.float32:
+        ref = O.dequant_f32(codes, s, b)
+        assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+    else:
+        assert np.array_equal(bf16_bits(out), O.dequant_bf16(codes, s, b))
+
+
+def test_dequant_edge_values_bitexact():
+    """Every code x f16 edge values (zeros, subnormals, max normal, negatives) for scale and bias."""
+    e = np.array([0x0000, 0x8000, 0x0001, 0x8001, 0x03FF, 0x0400, 0x3C00, 0xBC00, 0x7BFF, 0xFBFF,
+                  0x1400, 0x2E66, 0xC000, 0x3555, 0x0200, 0x8200], dtype=np.uint16)
+    S_, B_ = np.meshgrid(e, e, indexing="ij")
+    N = S_.size
+    s = S_.reshape(N, 1).view(np.float16)
+    b = B_.reshape(N, 1).view(np.float16)
+    q = np.tile(np.arange(16), 4)[None, :].repeat(N, 0)
+    codes = O.pack_codes(q)
+    for dt in (torch.float32, torch.bfloat16):
+        out = ql.dequant(*_dev(codes, s, b), out_dtype=dt)
+        if dt == torch.float32:
+            got = out.cpu().numpy()
+            ref = O.dequant_f32(codes, s, b)
+            both_nan = np.isnan(got) & np.isnan(ref)
+            assert np.array_equal(got.view(np.uint32)[~both_nan], ref.view(np.uint32)[~both_nan])
+        else:
+            assert np.array_equal(bf16_bits(out), O.dequant_bf16(codes, s, b))
+
+
+# ------------------------------------------------------------------ pack
+
+def _pack_inputs(seed):
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_normal((96, 512)) * 0.02).astype(np.float32)
+    w[3, :64] = 0.125                        # constant group
+    w[4, 64:128] = np.float32(-65504.0)      # extreme but packable
+    w[4, 70] = 65504.0
+    w[5, :64] = rng.standard_normal(64).astype(np.float32) * 1e-7   # scale rounds to an f16 subnormal/zero
+    w[6, :] = np.round(w[6, :] * 1000) / 1000
+    return w
+
+
+def test_pack_rtn_bitexact():
+    w = _pack_inputs(1)
+    c, s, b = ql.pack(torch.from_numpy(w).cuda())
+    rc, rs, rb = O.pack_rtn(w)
+    assert np.array_equal(c.cpu().numpy().view(np.uint32), rc)
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), rs.view(np.uint16))
+    assert np.array_equal(b.cpu().numpy().view(np.uint16), rb.view(np.uint16))
+    assert ql.device_status() == 0
+
+
+def test_pack_rtn_bitexact_dit_weight():
+    w = S.dense_weight(2, 0, 512, 4608, 0.02)
+    c, s, b = ql.pack(torch.from_numpy(w).cuda())
+    rc, rs, rb = O.pack_rtn(w)
+    assert np.array_equal(c.cpu().numpy().view(np.uint32), rc)
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), rs.view(np.uint16))
+    assert np.array_equal(b.cpu().numpy().view(np.uint16), rb.view(np.uint16))
+
+
+def test_pack_nonfinite_reports_status():
+    w = np.zeros((8, 128), dtype=np.float32)
+    w[2, 5] = np.nan
+    w[5, 100] = 1e6
+    c, s, b = ql.pack(torch.from_numpy(w).cuda())
+    assert ql.device_status() == 1          # QL_ERR_INVALID_ARG
+    assert ql.device_status() == 0          # read clears
+    cs = c.cpu().numpy()
+    assert np.all(cs[2, :8] == 0) and np.all(cs[5, 8:] == 0)
+    with pytest.raises(ValueError):
+        O.pack_rtn(w)
+
+
+def test_pack_imatrix_unsupported():
+    w = torch.zeros((8, 64), dtype=torch.float32, device="cuda")
+    with pytest.raises(ql.QLinearError) as e:
+        ql.pack(w, imatrix=torch.ones(64, dtype=torch.float32, device="cuda"))
+    assert e.value.status == 3
+
+
+# ------------------------------------------------------------------ forward: small and ragged
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_forward_tiny(path, out):
+    w = S.WORKLOADS["tiny"]
+    x = w.x()
+    codes, s, b = w.w()
+    dt = torch.bfloat16 if out == "bf16" else torch.float32
+    y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=PATHS[path], out_dtype=dt)
+    _check_tol(y, O.forward_ref(x, codes, s, b), bf16=(out == "bf16"))
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_forward_one_hot_bitexact(path):
+    """x rows = unit vectors: y selects single weights, so the result is exact.
+
+    CUDA-core path: y = RN_bf16(fp32 dequant).  Tensor-core path (f16 operand): y = RN_bf16(RN_f16(w)).
+    """
+    rng = np.random.default_rng(3)
+    K, N = 320, 264
+    _, codes, s, b = random_layer(rng, 1, K, N)
+    ks = np.array([0, 1, 4, 7, 8, 63, 64, 65, 130, 200, 255, 256, 319] + list(range(9, 320, 23)))
+    x = np.zeros((ks.size, K), dtype=np.uint16)
+    x[np.arange(ks.size), ks] = 0x3F80
+    y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=PATHS[path])
+    got = bf16_bits(y)
+    if path == "gemv":
+        ref = O.dequant_bf16(codes, s, b)[:, ks].T
+    else:
+        ref = O.round_bf16(O.dequant_f16(codes, s, b).astype(np.float64))[:, ks].T
+    assert np.array_equal(got, ref)
+
+
+RAGGED_M = [1, 2, 3, 7, 8, 31, 32, 33, 127, 129, 255, 257, 513]
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("K,N", [(64, 8), (320, 264), (1024, 520)])
+def test_forward_ragged(path, K, N):
+    rng = np.random.default_rng(K + N)
+    for M in RAGGED_M:
+        if path == "gemv" and M > 129:
+            continue
+        x, codes, s, b = random_layer(rng, M, K, N)
+        y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=PATHS[path])
+        _check_tol(y, O.forward_ref(x, codes, s, b))
+
+
+@pytest.mark.parametrize("split", [1, 2, 3, 5, 16])
+def test_gemv_split_k(split):
+    rng = np.random.default_rng(split)
+    x, codes, s, b = random_layer(rng, 4, 1024, 64)
+    y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=ql.PATH_GEMV, split_k=split)
+    _check_tol(y, O.forward_ref(x, codes, s, b))
+
+
+def test_gemv_split_k_beyond_groups_rejected():
+    rng = np.random.default_rng(4)
+    x, codes, s, b = random_layer(rng, 4, 1024, 64)
+    with pytest.raises(ValueError):
+        ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=ql.PATH_GEMV, split_k=17)
+
+
+def test_forward_deterministic():
+    rng = np.random.default_rng(7)
+    x, codes, s, b = random_layer(rng, 300, 1024, 512)
+    args = (to_dev_bf16(x), *_dev(codes, s, b))
+    for path in PATHS.values():
+        a = bf16_bits(ql.forward(*args, path=path))
+        c = bf16_bits(ql.forward(*args, path=path))
+        assert np.array_equal(a, c)
+
+
+def test_dispatch_record():
+    rng = np.random.default_rng(8)
+    x, codes, s, b = random_layer(rng, 256, 256, 256)
+    ql.forward(to_dev_bf16(x), *_dev(codes, s, b))
+    assert ql.last_dispatch().startswith("path=tc_fused")
+    ql.forward(to_dev_bf16(x[:1]), *_dev(codes, s, b))
+    assert ql.last_dispatch().startswith("path=")
+
+
+def test_workspace_and_alignment_errors():
+    rng = np.random.default_rng(9)
+    x, codes, s, b = random_layer(rng, 256, 256, 256)
+    xd, cd, sd, bd = to_dev_bf16(x), *_dev(codes, s, b)
+    L = ql.lib()
+    y = torch.empty((256, 256), dtype=torch.bfloat16, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    need = ql.workspace_size(256, 256, 256)
+    assert need > 0
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    ok = L.qlinear_forward(xd.data_ptr(), cd.data_ptr(), sd.data_ptr(), bd.data_ptr(), y.data_ptr(),
+                           256, 256, 256, 64, ws.data_ptr(), need, st)
+    assert ok == 0
+    assert L.qlinear_forward(xd.data_ptr(), cd.data_ptr(), sd.data_ptr(), bd.data_ptr(), y.data_ptr(),
+                             256, 256, 256, 64, ws.data_ptr(), need - 1, st) == 4
+    assert L.qlinear_forward(xd.data_ptr(), cd.data_ptr(), sd.data_ptr(), bd.data_ptr(), y.data_ptr(),
+                             256, 256, 256, 64, None, 0, st) == 4
+    assert L.qlinear_forward(xd.data_ptr() + 2, cd.data_ptr(), sd.data_ptr(), bd.data_ptr(), y.data_ptr(),
+                             255, 256, 256, 64, ws.data_ptr(), need, st) == 2
+    # y aliasing x
+    assert L.qlinear_forward(xd.data_ptr(), cd.data_ptr(), sd.data_ptr(), bd.data_ptr(), xd.data_ptr(),
+                             256, 256, 256, 64, ws.data_ptr(), need, st) == 1
+    # workspace overlapping y
+    assert L.qlinear_forward(xd.data_ptr(), cd.data_ptr(), sd.data_ptr(), bd.data_ptr(), y.data_ptr(),
+                             256, 256, 256, 64, y.data_ptr(), need, st) == 1
+
+
+# ------------------------------------------------------------------ forward: the full workloads (sampled rows)
+
+def _full_case(name, M=None, path=ql.PATH_AUTO, fitted=None):
+    w = S.WORKLOADS[name]
+    M = w.M if M is None else M
+    x = w.x(M)
+    codes, s, b = w.w() if fitted is None else fitted
+    y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=path)
+    rows = sample_rows(M, n_random=48, seed=M)
+    y_ref = O.forward_rows(x, codes, s, b, rows)
+    got = bf16_bits(y)[rows]
+    t = O.tolerance(O.decode_bf16(got), y_ref)
+    assert t["ok"], (name, M, t)
+    return t
+
+
+@pytest.mark.parametrize("M", S.TEXT_PROJ_M)
+def test_full_text_proj(M):
+    _full_case("text_proj", M)
+
+
+def test_full_qkv():
+    _full_case("qkv")
+
+
+def test_full_mlp_down():
+    _full_case("mlp_down")
+
+
+@pytest.mark.parametrize("name", ["canvas2048_n4608", "canvas2048_n13824"])
+def test_full_canvas2048(name):
+    _full_case(name)

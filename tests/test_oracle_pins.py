@@ -157,6 +157,21 @@ def test_dequant_f32_is_correctly_rounded():
             assert abs(got - exact) <= abs(lo - exact) and abs(got - exact) <= abs(hi - exact)
 
 
+def test_dequant_f16_is_correctly_rounded():
+    """f16 operand = binary16 nearest to the exact rational s*q + b (checked against both neighbours)."""
+    rng = _rng(17)
+    _, codes, s, b = _random_layer(rng, 1, 128, 24)
+    w16 = O.dequant_f16(codes, s, b)
+    q = O.unpack_codes(codes, 128)
+    for n in range(24):
+        for k in range(0, 128, 3):
+            exact = Fraction(float(s[n, k // 64])) * int(q[n, k]) + Fraction(float(b[n, k // 64]))
+            got = Fraction(float(w16[n, k]))
+            lo = Fraction(float(np.nextafter(w16[n, k], np.float16(-np.inf))))
+            hi = Fraction(float(np.nextafter(w16[n, k], np.float16(np.inf))))
+            assert abs(got - exact) <= abs(lo - exact) and abs(got - exact) <= abs(hi - exact)
+
+
 def test_dequant_bf16_is_bf16_of_f32_dequant():
     rng = _rng(5)
     _, codes, s, b = _random_layer(rng, 1, 128, 32)
