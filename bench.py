@@ -58,6 +58,26 @@ def peaks():
     return 1590.0, 6650.0, "fallback"
 
 
+def kernel_source_hash() -> str:
+    import hashlib
+    d = os.path.join(ROOT, "group_wise_affine_qlinear_b200", "csrc")
+    src = open(os.path.join(d, "ql_tc_fused.cuh"), "rb").read() + open(os.path.join(d, "ql_ptx.cuh"), "rb").read()
+    return hashlib.sha256(src).hexdigest()[:12]
+
+
+def recorded_traffic(path: str, key: str):
+    """DRAM bytes per launch from the last ncu capture, if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    h = kernel_source_hash()
+    for ln in open(p):
+        f = ln.split()
+        if len(f) == 4 and f[0] == path and f[1] == key and f[2] == h:
+            return int(f[3])
+    return None
+
+
 # ---------------------------------------------------------------------------- CPU oracle timing
 
 def oracle_rate(w: S.Workload, M: int, seconds: float, x_bits=None, weights=None):
@@ -270,12 +290,7 @@ def main():
     e2e_value = world * flops / (mean_e2e * 1e-3) / 1e12
     peak_tf, peak_gbs, peak_kind = peaks()
     main_tf = flops / (mean_main * 1e-3) / 1e12
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof):
-        tj = json.load(open(prof))
-        key = f"{dispatch.split()[0]}:{w.name}:M={M}"
-        traffic = tj.get(key)
+    traffic = recorded_traffic(dispatch.split()[0], f"{w.name}:M={M}")
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K_, "warmup": a.warmup,
