@@ -26,6 +26,7 @@ from ._lib import (  # noqa: F401
     dequant,
     device_status,
     forward,
+    forward_noalloc,
     last_dispatch,
     lib,
     library_path,

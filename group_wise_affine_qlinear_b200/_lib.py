@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
         L.qlinear_get_device_status.restype = ctypes.c_int
         L.qlinear_last_dispatch.argtypes = [ctypes.c_char_p, sz]
         L.qlinear_last_dispatch.restype = ctypes.c_int
+        L.qlinear_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp]
+        L.qlinear_forward_noalloc.restype = ctypes.c_int
         L.qlinear_set_profile_events.argtypes = [vp, vp]
         L.qlinear_set_profile_events.restype = ctypes.c_int
         L.qlinear_status_string.argtypes = [ctypes.c_int]
@@ -139,6 +141,24 @@ def forward(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: 
                                      out.data_ptr(), _BF16 if out_dtype == torch.bfloat16 else _F32,
                                      M, K, N, GROUP, path, split_k, ws_ptr, ws_bytes, st)
     _check(s, "qlinear_forward")
+    return out
+
+
+def forward_noalloc(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+                    out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Small-M forward that allocates nothing on the device (qlinear_forward_noalloc in include/qlinear.h)."""
+    L = lib()
+    N, K = _weights_shape(codes, scales)
+    M = x.shape[0]
+    _need_cuda(x, "x", torch.bfloat16, (M, K))
+    _need_cuda(codes, "codes", torch.int32, (N, K // 8))
+    _need_cuda(scales, "scales", torch.float16, (N, K // GROUP))
+    _need_cuda(biases, "biases", torch.float16, (N, K // GROUP))
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need_cuda(out, "out", torch.bfloat16, (M, N))
+    _check(L.qlinear_forward_noalloc(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), biases.data_ptr(),
+                                     out.data_ptr(), M, K, N, GROUP, _stream_handle(stream)), "qlinear_forward_noalloc")
     return out
 
 

@@ -2,8 +2,8 @@
 
     python -m group_wise_affine_qlinear_b200.build [--verbose-ptxas]
 
-The library is one CUDA translation unit (csrc/ql_api.cu includes every
-kernel), linked with the static CUDA runtime so it loads without a GPU driver
+The library is two CUDA translation units (csrc/ql_api.cu, which includes
+every kernel header, and csrc/ql_noalloc.cu), linked with the static CUDA runtime so it loads without a GPU driver
 present; the driver is only needed when a call is made.
 """
 from __future__ import annotations
@@ -16,7 +16,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SRC = os.path.join(HERE, "csrc", "ql_api.cu")
+SRCS = [os.path.join(HERE, "csrc", f) for f in ("ql_api.cu", "ql_noalloc.cu")]
 OUT = os.path.join(HERE, "libqlinear.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -46,7 +46,7 @@ def build(force: bool = False, verbose_ptxas: bool = False, extra: list[str] | N
         return OUT
     cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "--cudart", "static",
-           "-I", os.path.join(ROOT, "include"), SRC, "-o", OUT + ".tmp"]
+           "-I", os.path.join(ROOT, "include"), *SRCS, "-o", OUT + ".tmp"]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
     if extra:

@@ -134,22 +134,12 @@ struct Plan {
     size_t off_xh = 0, off_rs = 0, off_sb = 0;
 };
 
-int auto_split(int64_t M, int64_t K, int64_t N, int sm_count) {
-    // Enough CTAs for ~4 waves of 8-row CTAs and K-slices of at least 4096.
-    const int64_t G = K / kGroup;
-    const int64_t ctas = N / kGemvWarps;
-    int s = 1;
-    while (ctas * s < 4 * sm_count && G / (2 * s) >= 64) s *= 2;
-    (void)M;
-    return s;
-}
-
 ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int sm_count, Plan* plan) {
     const int64_t G = K / kGroup;
     if (path == QL_PATH_AUTO) path = (M <= 64) ? QL_PATH_GEMV : QL_PATH_TC_FUSED;
     plan->path = path;
     if (path == QL_PATH_GEMV) {
-        int s = split_k > 0 ? split_k : auto_split(M, K, N, sm_count);
+        int s = split_k > 0 ? split_k : gemv_auto_split(K, N, sm_count);
         if (s > G || s > 65535) return QL_ERR_INVALID_ARG;
         plan->split_k = s;
         plan->workspace = s > 1 ? static_cast<size_t>(s) * M * N * sizeof(float) : 0;

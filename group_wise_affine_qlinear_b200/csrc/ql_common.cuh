@@ -1,7 +1,5 @@
 // Shared device helpers of the qlinear library: status word, bounded waits,
-// conversions.  Everything here is compiled into one translation unit
-// (ql_api.cu includes every kernel header), so the status word below is a
-// single per-device object.
+// conversions.
 #pragma once
 
 #include <cstdint>
@@ -16,7 +14,9 @@ namespace ql {
 constexpr int kGroup = 64;
 
 // First error recorded by any kernel since the host last read it (0 = none).
-__device__ unsigned int g_device_status;
+// One per translation unit and device; qlinear_get_device_status() reads the
+// one of ql_api.cu, whose kernels are the ones that record errors.
+static __device__ unsigned int g_device_status;
 
 __device__ __forceinline__ void record_status(unsigned int code) {
     atomicCAS(&g_device_status, 0u, code);

@@ -15,8 +15,9 @@ constexpr int kGemvMChunk = 4;         // activation rows per register accumulat
 
 // grid: (N / kGemvWarps, S).  Slice z covers groups [z*G/S, (z+1)*G/S) (balanced, non-empty for S <= G).
 // out: partial[z][M][N] fp32 when split_k > 1, else y (bf16 or fp32) directly.
+// The body is a device function so more than one kernel entry can share it.
 template <bool kBf16Out>
-__global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(
+__device__ __forceinline__ void gemv_body(
     const __nv_bfloat16* __restrict__ x, const uint32_t* __restrict__ codes,
     const __half* __restrict__ scales, const __half* __restrict__ biases,
     void* __restrict__ out, int M, int K, int N, bool partial_out) {
@@ -89,11 +90,19 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(
     }
 }
 
+template <bool kBf16Out>
+__global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(
+    const __nv_bfloat16* __restrict__ x, const uint32_t* __restrict__ codes,
+    const __half* __restrict__ scales, const __half* __restrict__ biases,
+    void* __restrict__ out, int M, int K, int N, bool partial_out) {
+    gemv_body<kBf16Out>(x, codes, scales, biases, out, M, K, N, partial_out);
+}
+
 // y[i] = sum_{z=0}^{S-1} partial[z][i] in that fixed order (deterministic), four
 // elements per thread.  count = M*N is a multiple of 8.
 template <bool kBf16Out>
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ partial,
-                                                            void* __restrict__ y, int64_t count, int S) {
+__device__ __forceinline__ void splitk_reduce_body(const float* __restrict__ partial, void* __restrict__ y,
+                                                   int64_t count, int S) {
     const int64_t n4 = count / 4;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
@@ -111,6 +120,22 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
             reinterpret_cast<float4*>(y)[i] = a;
         }
     }
+}
+
+template <bool kBf16Out>
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ partial,
+                                                            void* __restrict__ y, int64_t count, int S) {
+    splitk_reduce_body<kBf16Out>(partial, y, count, S);
+}
+
+// Split factor of the weight-streaming path: double it while the grid has fewer
+// than four waves of 8-row CTAs and every slice keeps at least 64 groups.
+inline int gemv_auto_split(int64_t K, int64_t N, int sm_count) {
+    const int64_t G = K / kGroup;
+    const int64_t ctas = N / kGemvWarps;
+    int s = 1;
+    while (ctas * s < 4 * sm_count && G / (2 * s) >= 64) s *= 2;
+    return s;
 }
 
 }  // namespace ql

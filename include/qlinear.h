@@ -152,6 +152,32 @@ QL_API ql_status qlinear_get_device_status(cudaStream_t stream);
 QL_API ql_status qlinear_last_dispatch(char* buf, size_t len);
 
 /*
+ * Allocation-free forward for small M.  The pages have no counterpart of this
+ * call; it exists for callers that cannot allocate device memory where they
+ * run the layer (a plugin living inside another engine's fixed memory pool, a
+ * serving loop that must not allocate after start-up, a runtime that passes
+ * only inputs and outputs and no workspace).
+ *
+ * Same arithmetic and arguments as qlinear_forward (bf16 y), restricted to
+ * M <= QL_NOALLOC_MAX_M (QL_ERR_UNSUPPORTED above), and it allocates nothing:
+ * its split-K partials live in a fixed scratch array of
+ * QL_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that
+ * loads the library holds until the process exits.  A shape whose partials
+ * would not fit returns QL_ERR_WORKSPACE.  The first call on a device looks up
+ * that device's address of the array (cudaGetSymbolAddress with the device
+ * current), so make the first call on each device before any stream capture.
+ * All calls share the one array and it keeps the last call's contents: calls
+ * that overlap on the GPU (other streams or host threads) race and must be
+ * serialized by the caller.  No cudaMalloc, cudaFree or allocating library
+ * routine is called.
+ */
+#define QL_NOALLOC_SCRATCH_BYTES (4u << 20)
+#define QL_NOALLOC_MAX_M 64
+QL_API ql_status qlinear_forward_noalloc(const void* x, const uint32_t* codes, const void* scales,
+                                         const void* biases, void* y, int64_t M, int64_t K, int64_t N,
+                                         int32_t group, cudaStream_t stream);
+
+/*
  * Measurement hook.  While set (both non-NULL), every qlinear_forward* call
  * made by the calling thread records `start` on its stream immediately before
  * its main kernel (the tensor-core GEMM or the weight-streaming kernel) and
