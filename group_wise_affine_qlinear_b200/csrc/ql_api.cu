@@ -60,10 +60,11 @@ ql_status device_info(DeviceInfo** out) {
         d.sm_count = n;
     }
     if (!d.fused_attr_set) {
-        if (cudaFuncSetAttribute(fused::fused_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 fused::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(fused::fused_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 fused::kSmemBytes) != cudaSuccess) {
+        using FC = fused::DefaultCfg;
+        if (cudaFuncSetAttribute(fused::fused_gemm_kernel<true, FC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 FC::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(fused::fused_gemm_kernel<false, FC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 FC::kSmemBytes) != cudaSuccess) {
             return QL_ERR_CUDA;
         }
         d.fused_attr_set = true;
@@ -197,14 +198,18 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
 
     CUtensorMap mx, mc, mp;
     ql_status s;
-    if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xh, K, M, K * 2, fused::BK, fused::BM,
+    if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xh, K, M, K * 2, fused::BK, fused::BT,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
-    if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K / 8, N, K / 2, fused::BK / 8, fused::BN,
+    if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K / 8, N, K / 2, fused::BK / 8, fused::BW,
                        CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
         return s;
-    if ((s = encode_2d(&mp, CU_TENSOR_MAP_DATA_TYPE_UINT32, sb, N, G, N * 4, fused::BN, 1,
+    if ((s = encode_2d(&mp, CU_TENSOR_MAP_DATA_TYPE_UINT32, sb, N, G, N * 4, fused::BW, 1,
                        CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+        return s;
+    CUtensorMap my;
+    if ((s = encode_2d(&my, bf16_out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, y, N, M,
+                       N * (bf16_out ? 2 : 4), 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
         return s;
 
     convert_x_kernel<<<static_cast<unsigned>(M), kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), xh, rs,
@@ -218,18 +223,19 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(N);
     p.G = static_cast<int>(G);
-    p.num_m = static_cast<int>((M + fused::BM - 1) / fused::BM);
-    p.num_n = static_cast<int>((N + fused::BN - 1) / fused::BN);
-    const int tiles = p.num_m * p.num_n;
+    p.num_t = static_cast<int>((M + fused::BT - 1) / fused::BT);
+    p.num_w = static_cast<int>((N + fused::BW - 1) / fused::BW);
+    const int tiles = p.num_t * p.num_w;
     const int grid = std::min(tiles, sm_count);
+    using FC = fused::DefaultCfg;
     prof_begin(st);
     if (bf16_out)
-        fused::fused_gemm_kernel<true><<<grid, fused::kThreads, fused::kSmemBytes, st>>>(mx, mc, mp, p);
+        fused::fused_gemm_kernel<true, FC><<<grid, fused::kThreads, FC::kSmemBytes, st>>>(mx, mc, mp, my, p);
     else
-        fused::fused_gemm_kernel<false><<<grid, fused::kThreads, fused::kSmemBytes, st>>>(mx, mc, mp, p);
+        fused::fused_gemm_kernel<false, FC><<<grid, fused::kThreads, FC::kSmemBytes, st>>>(mx, mc, mp, my, p);
     prof_end(st);
-    set_dispatch("path=tc_fused tile=%dx%dx%d stages=%d/%d ctas=%d splitk=1 launches=3", fused::BM, fused::BN, fused::BK,
-                 fused::NS_T, fused::NS_B, grid);
+    set_dispatch("path=tc_fused tile=%dw x %dt x %dk stages=x%d/c%d/a%d ctas=%d splitk=1 launches=3", fused::BW,
+                 fused::BT, fused::BK, FC::kNX, FC::kNC, fused::NA, grid);
     (void)codes;
     return launch_status();
 }

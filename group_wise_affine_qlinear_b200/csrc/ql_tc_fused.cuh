@@ -1,25 +1,42 @@
-// Fused-dequant tensor-core GEMM for large M (tcgen05, TMEM accumulators).
+// Fused-dequant tensor-core GEMM for large M (tcgen05, TMEM operands and accumulators).
 //
 // y[m][n] = rowscale[m] * sum_k xh[m][k] * wh(n, k)
 //   xh    f16 activations prescaled per row by a power of two (prepass)
 //   wh    RN_f16(s * q + b): the affine grid of aimarketly "Ideogram-4-IQ4_M",
 //         "What IQ4 means here", formed by one fused f16x2 multiply-add from the
 //         exact code q, i.e. rounded once
-// Operands are f16 (both A and B must share a type in kind::f16); the
-// accumulator is fp32 in tensor memory.  One K-step is exactly one 64-wide
-// quantization group, so every weight row needs one (scale, bias) pair per step.
+// Operands are f16 (A and B must share a type in kind::f16); the accumulator is
+// fp32 in tensor memory.  One K-step is exactly one 64-wide quantization group,
+// so every weight row needs one (scale, bias) pair per step.
 //
-// Tile: 128 tokens (TMEM lanes) x 256 weight rows (TMEM columns) x 64 k.
-// Warp roles of one persistent CTA per SM:
-//   warps 0-7   dequantizers: one weight row each per K-step; read the 32 code
-//               bytes and the (scale, bias) pair TMA brought in, write the f16
-//               B tile in the K-major 128-byte-swizzle layout the MMA reads
-//   warp 8      TMA producer: activation tile (swizzled), code tile, parameter tile
+// The MMA computes the transposed tile D[n][m] = sum_k wh(n, k) xh(m, k), for
+// two groups of 128 weight rows that share one activation tile:
+//   A = dequantized weights, 128 rows x 64 k per group, written by the
+//       dequantizers straight into tensor memory (tcgen05.st), never into
+//       shared memory;
+//   B = activations, 192 tokens x 64 k, TMA-loaded into shared memory with the
+//       128-byte swizzle, read by both groups' MMAs;
+//   D = per group 128 lanes (weight rows) x 192 columns (tokens), fp32.
+// Keeping the dequantized tiles out of shared memory leaves shared memory to the
+// activation stream, and serving 256 weight rows from each activation tile
+// halves the L2 -> SM traffic per FLOP compared with one group.  TMEM holds the
+// two accumulators (2 x 192 columns) and two A stages of 2 x 32 columns: all
+// 512 columns, so each accumulator is single-buffered; the MMA of the next tile
+// waits only for its own group to be drained, which overlaps half the epilogue.
+//
+// Warp roles of one persistent CTA per SM (512 threads):
+//   warps 0-7   dequantizers: warp w owns TMEM lanes 32*(w%4).. of group w/4,
+//               one weight row per thread, every K-step
+//   warp 8      TMA producer of activation tiles
 //   warp 9      TMEM allocator and single-thread MMA issuer
-//   warps 10-13 epilogue: TMEM -> registers -> rowscale -> bf16/fp32 -> global
-// Two rings decouple the roles: the TMA ring (activations, codes, parameters)
-// and the B ring (dequantized tiles).  Two TMEM accumulators (2 x 256 columns)
-// let the epilogue of one tile overlap the main loop of the next.
+//   warp 10     TMA producer of code and parameter tiles
+//   warp 11     idle
+//   warps 12-15 epilogue: TMEM -> registers -> rowscale -> bf16/fp32 -> a 32x32
+//               staging block in shared memory -> TMA tensor store (which also
+//               clips the ragged edges of y)
+// Rings: X (activation tiles, freed by MMA completion), C (codes + parameters,
+// freed once read by the dequantizers), A (TMEM weight stages, freed by MMA
+// completion); accumulators are freed per group by the epilogue.
 #pragma once
 
 #include "ql_ptx.cuh"
@@ -27,48 +44,59 @@
 namespace ql {
 namespace fused {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BWG = 128;                // weight rows per group (MMA M, TMEM lanes)
+constexpr int NG = 2;                   // groups per tile
+constexpr int BW = NG * BWG;            // weight rows per tile
+constexpr int BT = 192;                 // tokens per tile (MMA N, TMEM columns)
 constexpr int BK = 64;
 constexpr int UK = 16;
-constexpr int NS_T = 4;
-constexpr int NS_B = 3;
-constexpr int kDequantWarps = BN / 32;                  // one row per thread
-constexpr int kWarpTma = kDequantWarps;                 // 8
-constexpr int kWarpMma = kDequantWarps + 1;             // 9
-constexpr int kWarpEpi0 = kDequantWarps + 2;            // 10..13 (ids % 4 = 2,3,0,1: every TMEM quarter once)
-constexpr int kThreads = (kDequantWarps + 2 + 4) * 32;  // 448
-constexpr uint32_t kTmemCols = 2 * BN;                  // 512
+constexpr int kDequantWarps = 8;
+constexpr int kWarpTmaX = 8;
+constexpr int kWarpMma = 9;
+constexpr int kWarpTmaC = 10;
+constexpr int kWarpEpi0 = 12;           // 12..15: quarters 0..3
+constexpr int kThreads = 16 * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCol = 0;         // accumulator of group g at columns [g*BT, (g+1)*BT)
+constexpr uint32_t kAStageCol = NG * BT;// A stage s, group g at columns [384 + 64 s + 32 g, +32)
+constexpr int NA = 2;                   // TMEM weight stages
+static_assert(kAStageCol + NA * NG * 32 <= kTmemCols, "tensor memory budget");
 
-constexpr uint32_t kABytes = BM * BK * 2;               // 16 KB
-constexpr uint32_t kBBytes = BN * BK * 2;               // 32 KB
-constexpr uint32_t kCBytes = BN * BK / 2;               // 8 KB of codes
-constexpr uint32_t kPBytes = BN * 4;                    // 1 KB of (scale, bias)
-constexpr uint32_t kTxBytes = kABytes + kCBytes + kPBytes;
+constexpr uint32_t kXBytes = BT * BK * 2;   // 24 KB
+constexpr uint32_t kCBytes = BW * BK / 2;   // 8 KB of codes
+constexpr uint32_t kPBytes = BW * 4;        // 1 KB of (scale, bias)
+constexpr uint32_t kStageBytes = 32 * 32 * 4;   // one epilogue staging block (fp32 worst case)
+constexpr uint32_t kEpiBytes = 4 * 2 * kStageBytes;   // 4 warps x 2 buffers
 
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffB = kOffA + NS_T * kABytes;
-constexpr uint32_t kOffC = kOffB + NS_B * kBBytes;
-constexpr uint32_t kOffP = kOffC + NS_T * kCBytes;
-constexpr uint32_t kOffBar = kOffP + NS_T * kPBytes;
-constexpr uint32_t kNumBars = 2 * NS_T + 2 * NS_B + 4 + 1;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+template <int NX, int NC>
+struct Cfg {
+    static constexpr int kNX = NX, kNC = NC;
+    static constexpr uint32_t kOffX = 0;
+    static constexpr uint32_t kOffC = kOffX + NX * kXBytes;
+    static constexpr uint32_t kOffP = kOffC + NC * kCBytes;
+    static constexpr uint32_t kOffEpi = kOffP + NC * kPBytes;
+    static constexpr uint32_t kOffBar = kOffEpi + kEpiBytes;
+    static constexpr uint32_t kNumBars = 2 * NX + 2 * NC + 2 * NA + 1 + NG + 1;
+    static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
+    static_assert(kXBytes % 1024 == 0, "swizzle atoms need 1 KB alignment");
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
-static_assert(kOffB % 1024 == 0 && kBBytes % 1024 == 0 && kABytes % 1024 == 0, "swizzle atoms need 1 KB alignment");
+using DefaultCfg = Cfg<5, 6>;
 
 struct Params {
     float* rowscale;      // [M] 2^e_m
     void* y;              // [M][N] bf16 or fp32
     int M, N, G;
-    int num_m, num_n;
+    int num_t, num_w;     // token tiles, weight tiles
 };
 
-__device__ __forceinline__ void tile_coords(int t, int num_n, int& m_blk, int& n_blk) {
-    // n fastest: a wave of CTAs shares a few activation row-blocks (streamed from HBM
-    // once) and sweeps the whole (L2-resident) packed weight.
-    m_blk = t / num_n;
-    n_blk = t - m_blk * num_n;
+__device__ __forceinline__ void tile_coords(int t, int num_w, int& t_blk, int& w_blk) {
+    // weight tiles fastest: a wave of CTAs shares one or two activation row blocks
+    // (streamed from HBM once) and sweeps the whole (L2-resident) packed weight.
+    t_blk = t / num_w;
+    w_blk = t - t_blk * num_w;
 }
 
 // Dequantize one code word (8 codes, k order 0..7) into 4 f16x2 words holding the
@@ -77,7 +105,7 @@ __device__ __forceinline__ void tile_coords(int t, int num_n, int& m_blk, int& n
 // 4-7 / 20-23 ORed into 64.0 (0x5400, unit 1/16) gives 64 + q exactly.
 // Subtracting the magic leaves q exactly; one fused f16x2 FMA then forms
 // RN_f16(s*q + b).
-__device__ __forceinline__ uint4 dequant_word(uint32_t v, __half2 s2, __half2 b2) {
+__device__ __forceinline__ void dequant_word(uint32_t v, __half2 s2, __half2 b2, uint32_t* o) {
     const uint32_t v8 = v >> 8;
     uint32_t p0, p1, p2, p3;
     asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(p0) : "r"(v));
@@ -86,45 +114,60 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t v, __half2 s2, __half2 b2
     asm("lop3.b32 %0, %1, 0x00F000F0, 0x54005400, 0xEA;" : "=r"(p3) : "r"(v8));
     const __half2 m1024 = half2_of(0x64006400u);
     const __half2 m64 = half2_of(0x54005400u);
-    uint4 o;
-    o.x = bits_of(__hfma2(__hsub2(half2_of(p0), m1024), s2, b2));
-    o.y = bits_of(__hfma2(__hsub2(half2_of(p1), m64), s2, b2));
-    o.z = bits_of(__hfma2(__hsub2(half2_of(p2), m1024), s2, b2));
-    o.w = bits_of(__hfma2(__hsub2(half2_of(p3), m64), s2, b2));
-    return o;
+    o[0] = bits_of(__hfma2(__hsub2(half2_of(p0), m1024), s2, b2));
+    o[1] = bits_of(__hfma2(__hsub2(half2_of(p1), m64), s2, b2));
+    o[2] = bits_of(__hfma2(__hsub2(half2_of(p2), m1024), s2, b2));
+    o[3] = bits_of(__hfma2(__hsub2(half2_of(p3), m64), s2, b2));
 }
 
-template <bool kBf16Out>
+// Position in a ring of N stages for the i-th use overall.
+template <int N>
+__device__ __forceinline__ void ring_pos(uint32_t i, int& stage, uint32_t& phase) {
+    stage = static_cast<int>(i % N);
+    phase = (i / N) & 1u;
+}
+
+template <bool kBf16Out, class C>
 __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
     const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
-    const __grid_constant__ CUtensorMap map_params, const Params p) {
+    const __grid_constant__ CUtensorMap map_params, const __grid_constant__ CUtensorMap map_y, const Params p) {
+    constexpr int NX = C::kNX, NC = C::kNC;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint64_t* tfull = bars;
-    uint64_t* tempty = tfull + NS_T;
-    uint64_t* bfull = tempty + NS_T;
-    uint64_t* bempty = bfull + NS_B;
-    uint64_t* afull = bempty + NS_B;
-    uint64_t* aempty = afull + 2;
-    uint64_t* drain = aempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint64_t* x_full = bars;
+    uint64_t* x_empty = x_full + NX;
+    uint64_t* c_full = x_empty + NX;
+    uint64_t* c_empty = c_full + NC;
+    uint64_t* a_full = c_empty + NC;
+    uint64_t* a_empty = a_full + NA;
+    uint64_t* acc_full = a_empty + NA;          // one per tile
+    uint64_t* acc_empty = acc_full + 1;         // one per group
+    uint64_t* drain = acc_empty + NG;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int num_tiles = p.num_m * p.num_n;
+    const int num_tiles = p.num_t * p.num_w;
+    // K-steps this CTA runs in total (its tiles times G); every ring position is a function of the step index.
+    const uint32_t my_tiles = blockIdx.x < static_cast<unsigned>(num_tiles)
+                                  ? (static_cast<uint32_t>(num_tiles) - 1u - blockIdx.x) / gridDim.x + 1u : 0u;
+    const uint32_t total_steps = my_tiles * static_cast<uint32_t>(p.G);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NS_T; ++i) { ptx::mbar_init(&tfull[i], 1); ptx::mbar_init(&tempty[i], 1); }
-        for (int i = 0; i < NS_B; ++i) { ptx::mbar_init(&bfull[i], kDequantWarps); ptx::mbar_init(&bempty[i], 1); }
-        for (int i = 0; i < 2; ++i) { ptx::mbar_init(&afull[i], 1); ptx::mbar_init(&aempty[i], 4); }
+        for (int i = 0; i < NX; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], 1); }
+        for (int i = 0; i < NC; ++i) { ptx::mbar_init(&c_full[i], 1); ptx::mbar_init(&c_empty[i], kDequantWarps); }
+        for (int i = 0; i < NA; ++i) { ptx::mbar_init(&a_full[i], kDequantWarps); ptx::mbar_init(&a_empty[i], 1); }
+        ptx::mbar_init(&acc_full[0], 1);
+        for (int g = 0; g < NG; ++g) ptx::mbar_init(&acc_empty[g], 4);
         ptx::mbar_init(drain, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == kWarpTma && lane == 0) {
-        ptx::prefetch_tensormap(&map_x);
+    if (warp == kWarpTmaX && lane == 0) ptx::prefetch_tensormap(&map_x);
+    if (warp == kWarpEpi0 && lane == 0) ptx::prefetch_tensormap(&map_y);
+    if (warp == kWarpTmaC && lane == 0) {
         ptx::prefetch_tensormap(&map_codes);
         ptx::prefetch_tensormap(&map_params);
     }
@@ -139,146 +182,178 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
 
     if (warp < kDequantWarps) {
         // ---------------------------------------------------------------- dequantizers
-        const int r = threadIdx.x;                 // weight row within the tile
-        int ts = 0, bs = 0;
-        uint32_t tph = 0, bph = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-            for (int kb = 0; kb < p.G; ++kb) {
-                bool got = ptx::mbar_wait(&tfull[ts], tph, abort_flag);
-                got = got && ptx::mbar_wait(&bempty[bs], bph ^ 1, abort_flag);
-                if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
-                const uint4* crow = reinterpret_cast<const uint4*>(smem + kOffC + ts * kCBytes + r * 32);
-                const uint4 c0 = crow[0], c1 = crow[1];
-                const uint32_t sb = reinterpret_cast<const uint32_t*>(smem + kOffP + ts * kPBytes)[r];
-                const __half2 sb2 = half2_of(sb);
-                const __half2 s2 = __low2half2(sb2);
-                const __half2 b2 = __high2half2(sb2);
-                uint8_t* brow = smem + kOffB + bs * kBBytes + r * 128;
-                const uint32_t sw = static_cast<uint32_t>(r & 7);
-                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const int grp = warp >> 2;                 // weight-row group
+        const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
+        const int r = grp * BWG + quarter * 32 + lane;   // weight row within the tile
+        // Rows whose bit 2 is set read their two 16-byte halves in the opposite order,
+        // so each group of 8 lanes touches 8 distinct 16-byte bank groups.
+        const int h = (r >> 2) & 1;
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        for (uint32_t i = 0; i < total_steps; ++i) {
+            int cs, as;
+            uint32_t cph, aph;
+            ring_pos<NC>(i, cs, cph);
+            ring_pos<NA>(i, as, aph);
+            bool got = ptx::mbar_wait(&c_full[cs], cph, abort_flag);
+            got = got && ptx::mbar_wait(&a_empty[as], aph ^ 1, abort_flag);
+            if (!__all_sync(0xFFFFFFFFu, got)) break;
+            ptx::tc_fence_after_sync();
+            const uint4* crow = reinterpret_cast<const uint4*>(smem + C::kOffC + cs * kCBytes + r * 32);
+            const uint4 first = crow[h];
+            const uint4 second = crow[h ^ 1];
+            const uint32_t sb = reinterpret_cast<const uint32_t*>(smem + C::kOffP + cs * kPBytes)[r];
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&c_empty[cs]);     // codes and parameters are in registers
+            const uint4 c0 = h ? second : first;
+            const uint4 c1 = h ? first : second;
+            const __half2 sb2 = half2_of(sb);
+            const __half2 s2 = __low2half2(sb2);
+            const __half2 b2 = __high2half2(sb2);
+            const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            uint32_t a[32];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    *reinterpret_cast<uint4*>(brow + ((c ^ sw) << 4)) = dequant_word(words[c], s2, b2);
-                }
-                ptx::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&bfull[bs]);
-                if (++ts == NS_T) { ts = 0; tph ^= 1; }
-                if (++bs == NS_B) { bs = 0; bph ^= 1; }
-            }
+            for (int c = 0; c < 8; ++c) dequant_word(words[c], s2, b2, &a[4 * c]);
+            ptx::tmem_st_32x32b_x32(tmem_base + lane_addr + kAStageCol + 64u * as + 32u * grp, a);
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&a_full[as]);
         }
-    } else if (warp == kWarpTma) {
-        // ---------------------------------------------------------------- TMA producer
+    } else if (warp == kWarpTmaX || warp == kWarpTmaC) {
+        // ---------------------------------------------------------------- TMA producers
         if (lane == 0) {
-            int ts = 0;
-            uint32_t tph = 0;
-            uint32_t issued[NS_T] = {};
+            const bool is_x = warp == kWarpTmaX;
+            const int depth = is_x ? NX : NC;
+            uint64_t* full = is_x ? x_full : c_full;
+            uint64_t* empty = is_x ? x_empty : c_empty;
+            uint32_t i = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                int m_blk, n_blk;
-                tile_coords(t, p.num_n, m_blk, n_blk);
-                for (int kb = 0; kb < p.G; ++kb) {
-                    if (!ptx::mbar_wait(&tempty[ts], tph ^ 1, abort_flag)) { ok = false; break; }
-                    ptx::mbar_arrive_expect_tx(&tfull[ts], kTxBytes);
-                    ptx::tma_load_2d(smem + kOffA + ts * kABytes, &map_x, &tfull[ts], kb * BK, m_blk * BM);
-                    ptx::tma_load_2d(smem + kOffC + ts * kCBytes, &map_codes, &tfull[ts], kb * (BK / 8), n_blk * BN);
-                    ptx::tma_load_2d(smem + kOffP + ts * kPBytes, &map_params, &tfull[ts], n_blk * BN, kb);
-                    ++issued[ts];
-                    if (++ts == NS_T) { ts = 0; tph ^= 1; }
+                int t_blk, w_blk;
+                tile_coords(t, p.num_w, t_blk, w_blk);
+                for (int kb = 0; kb < p.G; ++kb, ++i) {
+                    const int s = static_cast<int>(i % depth);
+                    const uint32_t ph = (i / depth) & 1u;
+                    if (!ptx::mbar_wait(&empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
+                    if (is_x) {
+                        ptx::mbar_arrive_expect_tx(&full[s], kXBytes);
+                        ptx::tma_load_2d(smem + C::kOffX + s * kXBytes, &map_x, &full[s], kb * BK, t_blk * BT);
+                    } else {
+                        ptx::mbar_arrive_expect_tx(&full[s], kCBytes + kPBytes);
+                        ptx::tma_load_2d(smem + C::kOffC + s * kCBytes, &map_codes, &full[s], kb * (BK / 8), w_blk * BW);
+                        ptx::tma_load_2d(smem + C::kOffP + s * kPBytes, &map_params, &full[s], w_blk * BW, kb);
+                    }
                 }
             }
-            // Never leave the CTA with bulk copies still landing in its shared memory.
-            for (int i = 0; i < NS_T; ++i) {
-                if (issued[i] > 0) ptx::mbar_wait(&tfull[i], (issued[i] - 1) & 1, nullptr);
+            // Never leave the CTA with bulk copies still landing in its shared memory:
+            // wait for the most recent load of every stage that received one.
+            const uint32_t issued = i;
+            for (uint32_t j = (issued > static_cast<uint32_t>(depth) ? issued - depth : 0u); j < issued; ++j) {
+                ptx::mbar_wait(&full[j % depth], (j / depth) & 1u, nullptr);
             }
         }
     } else if (warp == kWarpMma) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_f16(BM, BN, false);
-            int ts = 0, bs = 0;
-            uint32_t tph = 0, bph = 0;
+            constexpr uint32_t idesc = ptx::idesc_f16(BWG, BT, false);
+            uint32_t i = 0;
             bool ok = true;
             int j = 0;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++j) {
-                const int a = j & 1;
-                if (!ptx::mbar_wait(&aempty[a], ((j >> 1) & 1) ^ 1, abort_flag)) break;
-                ptx::tc_fence_after_sync();
-                const uint32_t d = tmem_base + static_cast<uint32_t>(a * BN);
-                for (int kb = 0; kb < p.G; ++kb) {
-                    if (!ptx::mbar_wait(&tfull[ts], tph, abort_flag)) { ok = false; break; }
-                    if (!ptx::mbar_wait(&bfull[bs], bph, abort_flag)) { ok = false; break; }
+                for (int kb = 0; kb < p.G; ++kb, ++i) {
+                    int xs, as;
+                    uint32_t xph, aph;
+                    ring_pos<NX>(i, xs, xph);
+                    ring_pos<NA>(i, as, aph);
+                    if (!ptx::mbar_wait(&x_full[xs], xph, abort_flag)) { ok = false; break; }
+                    if (!ptx::mbar_wait(&a_full[as], aph, abort_flag)) { ok = false; break; }
                     ptx::tc_fence_after_sync();
-                    const uint32_t a_addr = ptx::smem_addr(smem + kOffA + ts * kABytes);
-                    const uint32_t b_addr = ptx::smem_addr(smem + kOffB + bs * kBBytes);
+                    const uint32_t x_addr = ptx::smem_addr(smem + C::kOffX + xs * kXBytes);
 #pragma unroll
-                    for (int u = 0; u < BK / UK; ++u) {
-                        ptx::mma_f16_ss(d, ptx::sdesc_sw128(a_addr + u * UK * 2), ptx::sdesc_sw128(b_addr + u * UK * 2),
-                                        idesc, (kb | u) != 0);
+                    for (int g = 0; g < NG; ++g) {
+                        if (kb == 0) {
+                            // the previous tile's group-g results must have been drained
+                            if (!ptx::mbar_wait(&acc_empty[g], (j & 1) ^ 1, abort_flag)) { ok = false; break; }
+                            ptx::tc_fence_after_sync();
+                        }
+                        const uint32_t d = tmem_base + kAccCol + static_cast<uint32_t>(g * BT);
+                        const uint32_t a_tm = tmem_base + kAStageCol + 64u * as + 32u * g;
+#pragma unroll
+                        for (int u = 0; u < BK / UK; ++u) {
+                            ptx::mma_f16_ts(d, a_tm + u * (UK / 2), ptx::sdesc_sw128(x_addr + u * UK * 2), idesc,
+                                            (kb | u) != 0);
+                        }
                     }
-                    ptx::mma_commit(&tempty[ts]);
-                    ptx::mma_commit(&bempty[bs]);
-                    if (++ts == NS_T) { ts = 0; tph ^= 1; }
-                    if (++bs == NS_B) { bs = 0; bph ^= 1; }
+                    if (!ok) break;
+                    ptx::mma_commit(&x_empty[xs]);
+                    ptx::mma_commit(&a_empty[as]);
                 }
-                if (ok) ptx::mma_commit(&afull[a]);
+                if (ok) ptx::mma_commit(&acc_full[0]);
             }
             // Wait until every MMA this thread issued has finished before TMEM is released.
             ptx::mma_commit(drain);
             ptx::mbar_wait(drain, 0, nullptr);
         }
-    } else {
+    } else if (warp >= kWarpEpi0) {
         // ---------------------------------------------------------------- epilogue
         const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
+        uint8_t* epi_stage = smem + C::kOffEpi + (warp - kWarpEpi0) * 2 * kStageBytes;
+        uint32_t nstore = 0;
         int j = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++j) {
-            const int a = j & 1;
-            const bool got = ptx::mbar_wait(&afull[a], (j >> 1) & 1, abort_flag);
+            int t_blk, w_blk;
+            tile_coords(t, p.num_w, t_blk, w_blk);
+            // Row scales of the tile's tokens, fetched before the accumulators are ready:
+            // rs[c] belongs to token t_blk*BT + 32c + lane.
+            float rs[BT / 32];
+#pragma unroll
+            for (int c = 0; c < BT / 32; ++c) {
+                const int m = t_blk * BT + 32 * c + lane;
+                rs[c] = (m < p.M) ? p.rowscale[m] : 0.0f;
+            }
+            const bool got = ptx::mbar_wait(&acc_full[0], j & 1, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
             ptx::tc_fence_after_sync();
-            int m_blk, n_blk;
-            tile_coords(t, p.num_n, m_blk, n_blk);
-            const int m = m_blk * BM + quarter * 32 + lane;
-            const float rs = (m < p.M) ? p.rowscale[m] : 0.0f;
-            const uint32_t taddr = tmem_base + static_cast<uint32_t>(a * BN) + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
-            for (int chunk = 0; chunk < BN / 32; ++chunk) {
-                uint32_t r[32];
-                ptx::tmem_ld_32x32b_x32(taddr + chunk * 32, r);
-                ptx::tmem_wait_ld();
-                const int n0 = n_blk * BN + chunk * 32;
-                if (m < p.M) {
-                    if constexpr (kBf16Out) {
-                        __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(m) * p.N;
+            for (int g = 0; g < NG; ++g) {
+                const int n_base = w_blk * BW + g * BWG + quarter * 32;   // this warp's 32 output columns
+                const uint32_t taddr = tmem_base + kAccCol + static_cast<uint32_t>(g * BT) +
+                                       (static_cast<uint32_t>(quarter * 32) << 16);
+                // Two register buffers: the TMEM load of chunk c+1 is in flight while chunk c is stored.
+                uint32_t r[2][32];
+                ptx::tmem_ld_32x32b_x32(taddr, r[0]);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            if (n0 + 8 * i < p.N) {
-                                uint4 o;
-                                o.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * rs, __uint_as_float(r[8 * i + 1]) * rs);
-                                o.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * rs, __uint_as_float(r[8 * i + 3]) * rs);
-                                o.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * rs, __uint_as_float(r[8 * i + 5]) * rs);
-                                o.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * rs, __uint_as_float(r[8 * i + 7]) * rs);
-                                *reinterpret_cast<uint4*>(yrow + n0 + 8 * i) = o;
-                            }
-                        }
-                    } else {
-                        float* yrow = reinterpret_cast<float*>(p.y) + static_cast<int64_t>(m) * p.N;
+                for (int chunk = 0; chunk < BT / 32; ++chunk) {
+                    ptx::tmem_wait_ld();
+                    if (chunk + 1 < BT / 32) ptx::tmem_ld_32x32b_x32(taddr + (chunk + 1) * 32, r[(chunk + 1) & 1]);
+                    const uint32_t* v = r[chunk & 1];
+                    // staging block [32 tokens][32 columns], double-buffered per warp
+                    uint8_t* stage = epi_stage + (nstore & 1) * kStageBytes;
+                    if (lane == 0) ptx::bulk_wait_group_read<1>();   // the store that used this buffer has read it
+                    __syncwarp();
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            if (n0 + 4 * i < p.N) {
-                                *reinterpret_cast<float4*>(yrow + n0 + 4 * i) =
-                                    make_float4(__uint_as_float(r[4 * i + 0]) * rs, __uint_as_float(r[4 * i + 1]) * rs,
-                                                __uint_as_float(r[4 * i + 2]) * rs, __uint_as_float(r[4 * i + 3]) * rs);
-                            }
+                    for (int c = 0; c < 32; ++c) {
+                        const float val = __uint_as_float(v[c]) * __shfl_sync(0xFFFFFFFFu, rs[chunk], c);
+                        if constexpr (kBf16Out) {
+                            reinterpret_cast<__nv_bfloat16*>(stage)[c * 32 + lane] = __float2bfloat16_rn(val);
+                        } else {
+                            reinterpret_cast<float*>(stage)[c * 32 + lane] = val;
                         }
                     }
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        ptx::tma_store_2d(&map_y, stage, n_base, t_blk * BT + chunk * 32);
+                        ptx::bulk_commit_group();
+                    }
+                    ++nstore;
                 }
+                ptx::tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&acc_empty[g]);
             }
-            ptx::tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&aempty[a]);
         }
+        if (lane == 0) ptx::bulk_wait_group_all();   // every store has completed before the CTA exits
     }
 
     ptx::tc_fence_before_sync();
