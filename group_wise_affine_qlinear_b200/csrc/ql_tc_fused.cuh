@@ -24,16 +24,17 @@
 // 512 columns, so each accumulator is single-buffered; the MMA of the next tile
 // waits only for its own group to be drained, which overlaps half the epilogue.
 //
-// Warp roles of one persistent CTA per SM (512 threads):
+// Warp roles of one persistent CTA per SM (640 threads):
 //   warps 0-7   dequantizers: warp w owns TMEM lanes 32*(w%4).. of group w/4,
 //               one weight row per thread, every K-step
 //   warp 8      TMA producer of activation tiles
 //   warp 9      TMEM allocator and single-thread MMA issuer
 //   warp 10     TMA producer of code and parameter tiles
 //   warp 11     idle
-//   warps 12-15 epilogue: TMEM -> registers -> rowscale -> bf16/fp32 -> a 32x32
-//               staging block in shared memory -> TMA tensor store (which also
-//               clips the ragged edges of y)
+//   warps 12-19 epilogue, one set of four per group (warp w drains TMEM lanes
+//               32*(w%4).. of group (w-12)/4): TMEM -> registers -> rowscale ->
+//               bf16/fp32 -> a 32x32 staging block in shared memory -> TMA
+//               tensor store (which also clips the ragged edges of y)
 // Rings: X (activation tiles, freed by MMA completion), C (codes + parameters,
 // freed once read by the dequantizers), A (TMEM weight stages, freed by MMA
 // completion); accumulators are freed per group by the epilogue.
@@ -54,8 +55,9 @@ constexpr int kDequantWarps = 8;
 constexpr int kWarpTmaX = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpTmaC = 10;
-constexpr int kWarpEpi0 = 12;           // 12..15: quarters 0..3
-constexpr int kThreads = 16 * 32;
+constexpr int kWarpEpi0 = 12;           // 12..19: quarters 0..3 of group 0, then of group 1
+constexpr int kEpiWarps = 4 * NG;
+constexpr int kThreads = (kWarpEpi0 + kEpiWarps) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;         // accumulator of group g at columns [g*BT, (g+1)*BT)
 constexpr uint32_t kAStageCol = NG * BT;// A stage s, group g at columns [384 + 64 s + 32 g, +32)
@@ -66,7 +68,7 @@ constexpr uint32_t kXBytes = BT * BK * 2;   // 24 KB
 constexpr uint32_t kCBytes = BW * BK / 2;   // 8 KB of codes
 constexpr uint32_t kPBytes = BW * 4;        // 1 KB of (scale, bias)
 constexpr uint32_t kStageBytes = 32 * 32 * 4;   // one epilogue staging block (fp32 worst case)
-constexpr uint32_t kEpiBytes = 4 * 2 * kStageBytes;   // 4 warps x 2 buffers
+constexpr uint32_t kEpiBytes = kEpiWarps * 2 * kStageBytes;   // 2 buffers per epilogue warp
 
 template <int NX, int NC>
 struct Cfg {
@@ -83,7 +85,7 @@ struct Cfg {
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-using DefaultCfg = Cfg<5, 6>;
+using DefaultCfg = Cfg<4, 6>;
 
 struct Params {
     float* rowscale;      // [M] 2^e_m
@@ -160,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         for (int i = 0; i < NC; ++i) { ptx::mbar_init(&c_full[i], 1); ptx::mbar_init(&c_empty[i], kDequantWarps); }
         for (int i = 0; i < NA; ++i) { ptx::mbar_init(&a_full[i], kDequantWarps); ptx::mbar_init(&a_empty[i], 1); }
         ptx::mbar_init(&acc_full[0], 1);
+        static_assert(kWarpEpi0 % 4 == 0, "epilogue warp w must own TMEM lane quarter w % 4");
         for (int g = 0; g < NG; ++g) ptx::mbar_init(&acc_empty[g], 4);
         ptx::mbar_init(drain, 1);
         *abort_flag = 0;
@@ -194,10 +197,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             uint32_t cph, aph;
             ring_pos<NC>(i, cs, cph);
             ring_pos<NA>(i, as, aph);
+            // Codes arrive far ahead of the tensor core: unpack them into registers first
+            // and wait for the TMEM stage only when the result is ready to be written.
             bool got = ptx::mbar_wait(&c_full[cs], cph, abort_flag);
-            got = got && ptx::mbar_wait(&a_empty[as], aph ^ 1, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
-            ptx::tc_fence_after_sync();
             const uint4* crow = reinterpret_cast<const uint4*>(smem + C::kOffC + cs * kCBytes + r * 32);
             const uint4 first = crow[h];
             const uint4 second = crow[h ^ 1];
@@ -213,6 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             uint32_t a[32];
 #pragma unroll
             for (int c = 0; c < 8; ++c) dequant_word(words[c], s2, b2, &a[4 * c]);
+            got = ptx::mbar_wait(&a_empty[as], aph ^ 1, abort_flag);
+            if (!__all_sync(0xFFFFFFFFu, got)) break;
+            ptx::tc_fence_after_sync();
             ptx::tmem_st_32x32b_x32(tmem_base + lane_addr + kAStageCol + 64u * as + 32u * grp, a);
             ptx::tmem_wait_st();
             ptx::tc_fence_before_sync();
@@ -297,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
     } else if (warp >= kWarpEpi0) {
         // ---------------------------------------------------------------- epilogue
         const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
+        const int g = (warp - kWarpEpi0) >> 2;     // accumulator group this warp drains
         uint8_t* epi_stage = smem + C::kOffEpi + (warp - kWarpEpi0) * 2 * kStageBytes;
         uint32_t nstore = 0;
         int j = 0;
@@ -314,8 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             const bool got = ptx::mbar_wait(&acc_full[0], j & 1, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
             ptx::tc_fence_after_sync();
-#pragma unroll 1
-            for (int g = 0; g < NG; ++g) {
+            {
                 const int n_base = w_blk * BW + g * BWG + quarter * 32;   // this warp's 32 output columns
                 const uint32_t taddr = tmem_base + kAccCol + static_cast<uint32_t>(g * BT) +
                                        (static_cast<uint32_t>(quarter * 32) << 16);
