@@ -40,12 +40,14 @@ FLUSH_BYTES = 512 << 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="qkv", choices=sorted(S.WORKLOADS))
     ap.add_argument("--M", type=int, default=0, help="override the token count (0 = the workload's)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", type=int, default=0, help="force a kernel path (0 = dispatcher's choice)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-small-m", action="store_true", help="skip the small-M weight-streaming measurements")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     return ap.parse_args()
 
@@ -190,6 +192,59 @@ def run_reference(a, rank, world):
 
 # ---------------------------------------------------------------------------- our arm
 
+class Case:
+    """Device-resident inputs of one workload and timed qlinear_forward steps on them."""
+
+    def __init__(self, ql, torch, w, M, path, dev, flush):
+        import numpy as np
+        self.ql, self.torch, self.w, self.M, self.path, self.flush = ql, torch, w, M, path, flush
+        self.K, self.N = w.K, w.N
+        self.x_np = w.x(M)
+        self.codes_np, self.s_np, self.b_np = w.w()
+        self.x = torch.from_numpy(self.x_np.view(np.int16)).view(torch.bfloat16).to(dev)
+        self.codes = torch.from_numpy(self.codes_np.view(np.int32)).to(dev)
+        self.sc = torch.from_numpy(self.s_np).to(dev)
+        self.bi = torch.from_numpy(self.b_np).to(dev)
+        self.y = torch.empty((M, self.N), dtype=torch.bfloat16, device=dev)
+        ws_bytes = ql.workspace_size(M, self.K, self.N, path)
+        self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+
+    def step(self):
+        self.ql.forward(self.x, self.codes, self.sc, self.bi, out=self.y, workspace=self.ws, path=self.path)
+
+    def warm(self, n):
+        for _ in range(n):
+            self.flush.fill_(1)
+            self.step()
+        self.torch.cuda.synchronize()
+        self.dispatch = self.ql.last_dispatch()
+        self.launches = int(self.dispatch.split("launches=")[1].split()[0]) if "launches=" in self.dispatch else 1
+
+    def timed(self, steps):
+        """Per-step device time of the whole call and of its main kernel (L2 flushed before every step)."""
+        torch, ql = self.torch, self.ql
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        evm = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for e0, e1 in evm:            # create the handles so the library can record them
+            e0.record()
+            e1.record()
+        for i in range(steps):
+            self.flush.fill_(i & 0xFF)
+            ql.set_profile_events(*evm[i])
+            ev[i][0].record()
+            self.step()
+            ev[i][1].record()
+        ql.set_profile_events(None, None)
+        torch.cuda.synchronize()
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        main_ms = [a.elapsed_time(b) for a, b in evm]
+        return sum(step_ms) / steps, sum(main_ms) / steps
+
+    def algorithmic_bytes(self):
+        """Bytes a weight-streaming pass must move: packed W + x + y."""
+        return self.w.weight_bytes * self.N // self.w.N + self.M * self.K * 2 + self.M * self.N * 2
+
+
 def main():
     a = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -214,72 +269,53 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
+    dev = torch.device("cuda", local)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     w = S.WORKLOADS[a.workload]
     M = a.M or w.M
     K, N = w.K, w.N
-    x_np = w.x(M)
-    codes_np, s_np, b_np = w.w()
-    dev = torch.device("cuda", local)
-    x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
-    codes = torch.from_numpy(codes_np.view(np.int32)).to(dev)
-    sc = torch.from_numpy(s_np).to(dev)
-    bi = torch.from_numpy(b_np).to(dev)
-    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    ws_bytes = ql.workspace_size(M, K, N)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
-    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-
-    def step():
-        ql.forward(x, codes, sc, bi, out=y, workspace=ws)
-
-    for _ in range(a.warmup):
-        flush.fill_(1)
-        step()
-    torch.cuda.synchronize()
-    dispatch = ql.last_dispatch()
-    launches_per_step = int(dispatch.split("launches=")[1].split()[0]) if "launches=" in dispatch else 1
+    case = Case(ql, torch, w, M, a.path, dev, flush)
+    case.warm(a.warmup)
 
     # ---- device-timed steps (inputs resident; L2 flushed between steps)
-    K_ = a.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_)]
-    evm = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_)]
-    for e0, e1 in evm:            # create the handles so the library can record them
-        e0.record()
-        e1.record()
     clocks = ClockSampler(local)
-    barrier()
     clocks.start()
-    for i in range(K_):
-        flush.fill_(i & 0xFF)
-        ql.set_profile_events(*evm[i])
-        ev[i][0].record()
-        step()
-        ev[i][1].record()
-    ql.set_profile_events(None, None)
+    time.sleep(0.3)                     # let the sampler start before the timed region
+    barrier()
+    mean_step, mean_main = case.timed(a.steps)
     barrier()
     clk = clocks.stop()
-    step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
-    main_ms = [e0.elapsed_time(e1) for e0, e1 in evm]
     assert ql.device_status() == 0, "a kernel reported an error"
 
     # ---- end to end: pinned host x -> device, forward, y -> pinned host, per step
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_)]
+    x_host = torch.from_numpy(case.x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
     barrier()
-    for i in range(K_):
+    for i in range(a.steps):
         flush.fill_(i & 0xFF)
         ev2[i][0].record()
-        x.copy_(x_host, non_blocking=True)
-        step()
-        y_host.copy_(y, non_blocking=True)
+        case.x.copy_(x_host, non_blocking=True)
+        case.step()
+        y_host.copy_(case.y, non_blocking=True)
         ev2[i][1].record()
     barrier()
-    e2e_ms = [e0.elapsed_time(e1) for e0, e1 in ev2]
+    mean_e2e = sum(e0.elapsed_time(e1) for e0, e1 in ev2) / a.steps
 
-    mean_step = sum(step_ms) / K_
-    mean_main = sum(main_ms) / K_
-    mean_e2e = sum(e2e_ms) / K_
+    # ---- the small-M half of the metric: weight streaming on the 53248 -> 4608 text projection
+    small = []
+    if not a.no_small_m:
+        tp = S.WORKLOADS["text_proj"]
+        for Ms in (1, 8, 32):
+            c = Case(ql, torch, tp, Ms, 0, dev, flush)
+            c.warm(3)
+            st, mn = c.timed(max(10, a.steps))
+            small.append({"M": Ms, "dispatch": c.dispatch, "step_us": st * 1e3, "kernel_us": mn * 1e3,
+                          "weight_GBps": tp.weight_bytes / (st * 1e-3) / 1e9,
+                          "algorithmic_GBps": c.algorithmic_bytes() / (st * 1e-3) / 1e9})
+            del c
+        torch.cuda.synchronize()
+
     if pg:
         t = torch.tensor([mean_step, mean_main, mean_e2e], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -289,26 +325,41 @@ def main():
     value = world * flops / (mean_step * 1e-3) / 1e12
     e2e_value = world * flops / (mean_e2e * 1e-3) / 1e12
     peak_tf, peak_gbs, peak_kind = peaks()
-    main_tf = flops / (mean_main * 1e-3) / 1e12
+    dispatch = case.dispatch
+    kernel = dispatch.split()[0].replace("path=", "")
     traffic = recorded_traffic(dispatch.split()[0], f"{w.name}:M={M}")
+    if kernel == "tc_fused":
+        main_rate = flops / (mean_main * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": main_rate, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": main_rate / peak_tf, "traffic": traffic, "kernel": "fused_gemm_kernel",
+                "kernel_ms": mean_main,
+                "peak_kind": f"{peak_kind} bf16 dense burst (f16 has the same tcgen05 rate)",
+                "algorithmic": "2*M*N*K FLOPs per launch"}
+    else:
+        main_rate = case.algorithmic_bytes() / (mean_main * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": main_rate, "peak": peak_gbs, "unit": "GB/s",
+                "frac": main_rate / peak_gbs, "traffic": traffic, "kernel": kernel, "kernel_ms": mean_main,
+                "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                "algorithmic": "packed W (0.5625 B/weight) + x + y bytes per launch"}
+    for sm in small:
+        sm["frac_hbm_weight"] = sm["weight_GBps"] / peak_gbs
 
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K_, "warmup": a.warmup,
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
         "ms_per_step": mean_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16 MMA, fp32 accumulate (bf16 in/out)", "data": "synthetic",
-        "config": {"workload": f"{w.name} M={M} K={K} N={N}", "seed": w.seed, "l2": "flushed between steps (512 MiB write)",
-                   "parallelism": f"replicas x{world}", "dispatch": dispatch,
-                   "weight_GBps": (w.weight_bytes) / (mean_step * 1e-3) / 1e9},
-        "roofline": {"bound": "tensor", "achieved": main_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": main_tf / peak_tf, "traffic": traffic,
-                     "kernel": dispatch.split()[0].replace("path=", ""), "kernel_ms": mean_main,
-                     "peak_kind": f"{peak_kind} bf16 dense burst (f16 has the same tcgen05 rate)"},
+        "config": {"workload": f"{w.name} M={M} K={K} N={N}", "seed": w.seed,
+                   "l2": "flushed between steps (512 MiB write)", "parallelism": f"replicas x{world}",
+                   "dispatch": dispatch, "weight_GBps": w.weight_bytes / (mean_step * 1e-3) / 1e9},
+        "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
-        "gpu_launches": launches_per_step * K_,
+        "gpu_launches": case.launches * a.steps,
         "clocks": clk,
+        "small_m": small,
     }
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        rate, cores, rows, dt = oracle_rate(w, M, a.cpu_seconds, x_np[: min(M, 512)], (codes_np, s_np, b_np))
+        rate, cores, rows, dt = oracle_rate(w, M, a.cpu_seconds, case.x_np[: min(M, 512)],
+                                            (case.codes_np, case.s_np, case.b_np))
         line["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                 "sample": f"{rows} rows x full K x full N of {w.name} in {dt:.1f} s"}
     if rank == 0:

@@ -16,6 +16,7 @@
 #include "ql_pack.cuh"
 #include "ql_prepass.cuh"
 #include "ql_tc_fused.cuh"
+#include "ql_tc_skinny.cuh"
 
 namespace ql {
 namespace {
@@ -45,6 +46,7 @@ void set_dispatch(const char* fmt, ...) {
 struct DeviceInfo {
     int sm_count = 0;
     bool fused_attr_set = false;
+    bool skinny_attr_set = false;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -68,6 +70,15 @@ ql_status device_info(DeviceInfo** out) {
             return QL_ERR_CUDA;
         }
         d.fused_attr_set = true;
+    }
+    if (!d.skinny_attr_set) {
+        if (cudaFuncSetAttribute(skinny::skinny_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 skinny::Layout<16>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(skinny::skinny_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 skinny::Layout<32>::kSmemBytes) != cudaSuccess) {
+            return QL_ERR_CUDA;
+        }
+        d.skinny_attr_set = true;
     }
     *out = &d;
     return QL_OK;
@@ -130,6 +141,9 @@ ql_status check_shape(int64_t M, int64_t K, int64_t N, int32_t group) {
 struct Plan {
     int path = QL_PATH_GEMV;
     int split_k = 1;
+    // skinny path: stream-K runs
+    int ctas = 0, segmax = 0, nt = 0;
+    int64_t units = 0;
     size_t workspace = 0;
     // fused path workspace carve-up
     size_t off_xh = 0, off_rs = 0, off_sb = 0;
@@ -137,13 +151,25 @@ struct Plan {
 
 ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int sm_count, Plan* plan) {
     const int64_t G = K / kGroup;
-    if (path == QL_PATH_AUTO) path = (M <= 64) ? QL_PATH_GEMV : QL_PATH_TC_FUSED;
+    if (path == QL_PATH_AUTO) path = (M <= 32) ? QL_PATH_TC_SKINNY : QL_PATH_TC_FUSED;
     plan->path = path;
     if (path == QL_PATH_GEMV) {
         int s = split_k > 0 ? split_k : gemv_auto_split(K, N, sm_count);
         if (s > G || s > 65535) return QL_ERR_INVALID_ARG;
         plan->split_k = s;
         plan->workspace = s > 1 ? static_cast<size_t>(s) * M * N * sizeof(float) : 0;
+        return QL_OK;
+    }
+    if (path == QL_PATH_TC_SKINNY) {
+        if (M > 32 || split_k > 1) return QL_ERR_UNSUPPORTED;
+        plan->nt = M <= 16 ? 16 : 32;
+        const int64_t cpt = (G + skinny::CG - 1) / skinny::CG;
+        plan->units = ((N + skinny::BW - 1) / skinny::BW) * cpt;
+        plan->ctas = static_cast<int>(std::min<int64_t>(sm_count, plan->units));
+        const int64_t run = (plan->units + plan->ctas - 1) / plan->ctas;
+        plan->segmax = static_cast<int>((run + cpt - 1) / cpt + 1);
+        plan->split_k = 1;
+        plan->workspace = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * M * skinny::BW * sizeof(float), 256);
         return QL_OK;
     }
     if (path == QL_PATH_TC_FUSED) {
@@ -240,6 +266,48 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     return launch_status();
 }
 
+ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const void* scales, const void* biases,
+                     void* y, bool bf16_out, int64_t M, int64_t K, int64_t N, void* ws, cudaStream_t st,
+                     int sm_count) {
+    const int64_t G = K / kGroup;
+    CUtensorMap mc, mx;
+    ql_status s;
+    if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K / 8, N, K / 2,
+                       skinny::kBoxGroups * skinny::BK / 8, skinny::BW, CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
+        return s;
+    if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, skinny::BK, pl.nt,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
+        return s;
+    skinny::Params p;
+    p.partial = static_cast<float*>(ws);
+    p.scales = static_cast<const __half*>(scales);
+    p.biases = static_cast<const __half*>(biases);
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.G = static_cast<int>(G);
+    p.num_w = static_cast<int>((N + skinny::BW - 1) / skinny::BW);
+    p.cpt = static_cast<int>((G + skinny::CG - 1) / skinny::CG);
+    p.units = pl.units;
+    p.segmax = pl.segmax;
+    prof_begin(st);
+    if (pl.nt == 16)
+        skinny::skinny_kernel<16><<<pl.ctas, skinny::kThreads, skinny::Layout<16>::kSmemBytes, st>>>(mc, mx, p);
+    else
+        skinny::skinny_kernel<32><<<pl.ctas, skinny::kThreads, skinny::Layout<32>::kSmemBytes, st>>>(mc, mx, p);
+    prof_end(st);
+    const int64_t total = M * N;
+    const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4 * sm_count));
+    if (bf16_out)
+        skinny::skinny_reduce_kernel<true><<<blocks, 256, 0, st>>>(p.partial, y, p.M, p.N, p.cpt, p.units, pl.ctas,
+                                                                  pl.segmax);
+    else
+        skinny::skinny_reduce_kernel<false><<<blocks, 256, 0, st>>>(p.partial, y, p.M, p.N, p.cpt, p.units, pl.ctas,
+                                                                   pl.segmax);
+    set_dispatch("path=tc_skinny nt=%d ctas=%d segmax=%d units=%lld launches=2", pl.nt, pl.ctas, pl.segmax,
+                 static_cast<long long>(pl.units));
+    return launch_status();
+}
+
 ql_status forward_impl(const void* x, const uint32_t* codes, const void* scales, const void* biases, void* y,
                        ql_dtype out_dtype, int64_t M, int64_t K, int64_t N, int32_t group, int32_t path,
                        int32_t split_k, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
@@ -271,6 +339,8 @@ ql_status forward_impl(const void* x, const uint32_t* codes, const void* scales,
     const bool bf16 = out_dtype == QL_BF16;
     if (pl.path == QL_PATH_GEMV)
         return run_gemv(pl, x, codes, scales, biases, y, bf16, M, K, N, workspace, stream, dev->sm_count);
+    if (pl.path == QL_PATH_TC_SKINNY)
+        return run_skinny(pl, x, codes, scales, biases, y, bf16, M, K, N, workspace, stream, dev->sm_count);
     return run_fused(pl, x, codes, scales, biases, y, bf16, M, K, N, workspace, stream, dev->sm_count);
 }
 

@@ -28,9 +28,9 @@
 //   warps 0-7   dequantizers: warp w owns TMEM lanes 32*(w%4).. of group w/4,
 //               one weight row per thread, every K-step
 //   warp 8      TMA producer of activation tiles
-//   warp 9      TMEM allocator and single-thread MMA issuer
+//   warps 9, 11 single-thread MMA issuers for groups 0 / 1 (warp 9 also allocates TMEM);
+//               issuing from two threads doubles the tcgen05.mma issue rate
 //   warp 10     TMA producer of code and parameter tiles
-//   warp 11     idle
 //   warps 12-19 epilogue, one set of four per group (warp w drains TMEM lanes
 //               32*(w%4).. of group (w-12)/4): TMEM -> registers -> rowscale ->
 //               bf16/fp32 -> a 32x32 staging block in shared memory -> TMA
@@ -55,6 +55,7 @@ constexpr int kDequantWarps = 8;
 constexpr int kWarpTmaX = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpTmaC = 10;
+constexpr int kWarpMma2 = 11;
 constexpr int kWarpEpi0 = 12;           // 12..19: quarters 0..3 of group 0, then of group 1
 constexpr int kEpiWarps = 4 * NG;
 constexpr int kThreads = (kWarpEpi0 + kEpiWarps) * 32;
@@ -78,7 +79,7 @@ struct Cfg {
     static constexpr uint32_t kOffP = kOffC + NC * kCBytes;
     static constexpr uint32_t kOffEpi = kOffP + NC * kPBytes;
     static constexpr uint32_t kOffBar = kOffEpi + kEpiBytes;
-    static constexpr uint32_t kNumBars = 2 * NX + 2 * NC + 2 * NA + 1 + NG + 1;
+    static constexpr uint32_t kNumBars = 2 * NX + 2 * NC + 2 * NA + 1 + NG + NG;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
     static_assert(kXBytes % 1024 == 0, "swizzle atoms need 1 KB alignment");
@@ -158,13 +159,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
     const uint32_t total_steps = my_tiles * static_cast<uint32_t>(p.G);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NX; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], 1); }
+        // x and A stages are released by both MMA warps' commits
+        for (int i = 0; i < NX; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], NG); }
         for (int i = 0; i < NC; ++i) { ptx::mbar_init(&c_full[i], 1); ptx::mbar_init(&c_empty[i], kDequantWarps); }
-        for (int i = 0; i < NA; ++i) { ptx::mbar_init(&a_full[i], kDequantWarps); ptx::mbar_init(&a_empty[i], 1); }
-        ptx::mbar_init(&acc_full[0], 1);
+        for (int i = 0; i < NA; ++i) { ptx::mbar_init(&a_full[i], kDequantWarps); ptx::mbar_init(&a_empty[i], NG); }
+        ptx::mbar_init(&acc_full[0], NG);
         static_assert(kWarpEpi0 % 4 == 0, "epilogue warp w must own TMEM lane quarter w % 4");
         for (int g = 0; g < NG; ++g) ptx::mbar_init(&acc_empty[g], 4);
-        ptx::mbar_init(drain, 1);
+        for (int g = 0; g < NG; ++g) ptx::mbar_init(drain + g, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -258,8 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                 ptx::mbar_wait(&full[j % depth], (j / depth) & 1u, nullptr);
             }
         }
-    } else if (warp == kWarpMma) {
-        // ---------------------------------------------------------------- MMA issuer
+    } else if (warp == kWarpMma || warp == kWarpMma2) {
+        // ---------------------------------------------------------------- MMA issuers, one per group
+        const int gsel = warp == kWarpMma ? 0 : 1;
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_f16(BWG, BT, false);
             uint32_t i = 0;
@@ -276,7 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                     ptx::tc_fence_after_sync();
                     const uint32_t x_addr = ptx::smem_addr(smem + C::kOffX + xs * kXBytes);
 #pragma unroll
-                    for (int g = 0; g < NG; ++g) {
+                    {
+                        const int g = gsel;
                         if (kb == 0) {
                             // the previous tile's group-g results must have been drained
                             if (!ptx::mbar_wait(&acc_empty[g], (j & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -297,8 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                 if (ok) ptx::mma_commit(&acc_full[0]);
             }
             // Wait until every MMA this thread issued has finished before TMEM is released.
-            ptx::mma_commit(drain);
-            ptx::mbar_wait(drain, 0, nullptr);
+            ptx::mma_commit(drain + gsel);
+            ptx::mbar_wait(drain + gsel, 0, nullptr);
         }
     } else if (warp >= kWarpEpi0) {
         // ---------------------------------------------------------------- epilogue

@@ -17,7 +17,8 @@ from ._helpers import bf16_bits, random_layer, sample_rows, to_dev_bf16, to_dev_
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"gemv": ql.PATH_GEMV, "tc_fused": ql.PATH_TC_FUSED}
+PATHS = {"gemv": ql.PATH_GEMV, "tc_fused": ql.PATH_TC_FUSED, "tc_skinny": ql.PATH_TC_SKINNY}
+MAX_M = {"gemv": 129, "tc_fused": 1 << 30, "tc_skinny": 32}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -130,6 +131,24 @@ def test_pack_imatrix_unsupported():
 
 # ------------------------------------------------------------------ forward: small and ragged
 
+def test_skinny_rejects_large_m():
+    rng = np.random.default_rng(12)
+    x, codes, s, b = random_layer(rng, 33, 256, 64)
+    with pytest.raises(ValueError):
+        ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=ql.PATH_TC_SKINNY)
+
+
+@pytest.mark.parametrize("M", [1, 8, 16, 17, 32])
+@pytest.mark.parametrize("K,N", [(64, 8), (128, 4608), (4096, 264), (8192, 1032)])
+def test_skinny_stream_k_shapes(M, K, N):
+    """Runs that start and end inside tiles, tiles shorter than a run, ragged N."""
+    rng = np.random.default_rng(M * 7 + K + N)
+    x, codes, s, b = random_layer(rng, M, K, N)
+    y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=ql.PATH_TC_SKINNY)
+    _check_tol(y, O.forward_ref(x, codes, s, b))
+    assert ql.last_dispatch().startswith("path=tc_skinny")
+
+
 @pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 def test_forward_tiny(path, out):
@@ -145,17 +164,20 @@ def test_forward_tiny(path, out):
 def test_forward_one_hot_bitexact(path):
     """x rows = unit vectors: y selects single weights, so the result is exact.
 
-    CUDA-core path: y = RN_bf16(fp32 dequant).  Tensor-core path (f16 operand): y = RN_bf16(RN_f16(w)).
+    CUDA-core and skinny paths (exact codes, fp32 scale and bias): y = RN_bf16(fp32 dequant).
+    Large-M tensor-core path (f16 operand): y = RN_bf16(RN_f16(w)).
     """
     rng = np.random.default_rng(3)
     K, N = 320, 264
     _, codes, s, b = random_layer(rng, 1, K, N)
     ks = np.array([0, 1, 4, 7, 8, 63, 64, 65, 130, 200, 255, 256, 319] + list(range(9, 320, 23)))
+    if path == "tc_skinny":
+        ks = ks[:32]
     x = np.zeros((ks.size, K), dtype=np.uint16)
     x[np.arange(ks.size), ks] = 0x3F80
     y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=PATHS[path])
     got = bf16_bits(y)
-    if path == "gemv":
+    if path in ("gemv", "tc_skinny"):
         ref = O.dequant_bf16(codes, s, b)[:, ks].T
     else:
         ref = O.round_bf16(O.dequant_f16(codes, s, b).astype(np.float64))[:, ks].T
@@ -170,7 +192,7 @@ RAGGED_M = [1, 2, 3, 7, 8, 31, 32, 33, 127, 129, 255, 257, 513]
 def test_forward_ragged(path, K, N):
     rng = np.random.default_rng(K + N)
     for M in RAGGED_M:
-        if path == "gemv" and M > 129:
+        if M > MAX_M[path]:
             continue
         x, codes, s, b = random_layer(rng, M, K, N)
         y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=PATHS[path])
@@ -196,10 +218,21 @@ def test_forward_deterministic():
     rng = np.random.default_rng(7)
     x, codes, s, b = random_layer(rng, 300, 1024, 512)
     args = (to_dev_bf16(x), *_dev(codes, s, b))
-    for path in PATHS.values():
+    for name, path in PATHS.items():
+        if name == "tc_skinny":
+            continue
         a = bf16_bits(ql.forward(*args, path=path))
         c = bf16_bits(ql.forward(*args, path=path))
         assert np.array_equal(a, c)
+
+
+def test_skinny_deterministic():
+    rng = np.random.default_rng(17)
+    x, codes, s, b = random_layer(rng, 24, 8192, 1024)
+    args = (to_dev_bf16(x), *_dev(codes, s, b))
+    a = bf16_bits(ql.forward(*args, path=ql.PATH_TC_SKINNY))
+    c = bf16_bits(ql.forward(*args, path=ql.PATH_TC_SKINNY))
+    assert np.array_equal(a, c)
 
 
 def test_dispatch_record():
@@ -208,7 +241,7 @@ def test_dispatch_record():
     ql.forward(to_dev_bf16(x), *_dev(codes, s, b))
     assert ql.last_dispatch().startswith("path=tc_fused")
     ql.forward(to_dev_bf16(x[:1]), *_dev(codes, s, b))
-    assert ql.last_dispatch().startswith("path=")
+    assert ql.last_dispatch().startswith("path=tc_skinny")
 
 
 def test_workspace_and_alignment_errors():
