@@ -190,6 +190,24 @@ def run_reference(a, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------- multi-rank reduction
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings over the default process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(work_per_rank: float, slowest_ms: float, world: int) -> float:
+    """Throughput of all ranks together: every rank does work_per_rank (weak scaling); the slowest sets the time."""
+    return world * work_per_rank / (slowest_ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------- our arm
 
 class Case:
@@ -316,14 +334,11 @@ def main():
             del c
         torch.cuda.synchronize()
 
-    if pg:
-        t = torch.tensor([mean_step, mean_main, mean_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        mean_step, mean_main, mean_e2e = t.tolist()
+    mean_step, mean_main, mean_e2e = max_over_ranks([mean_step, mean_main, mean_e2e], dev)
 
     flops = 2.0 * M * K * N
-    value = world * flops / (mean_step * 1e-3) / 1e12
-    e2e_value = world * flops / (mean_e2e * 1e-3) / 1e12
+    value = whole_job_rate(flops, mean_step, world) / 1e12
+    e2e_value = whole_job_rate(flops, mean_e2e, world) / 1e12
     peak_tf, peak_gbs, peak_kind = peaks()
     dispatch = case.dispatch
     kernel = dispatch.split()[0].replace("path=", "")

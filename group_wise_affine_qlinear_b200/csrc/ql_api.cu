@@ -278,7 +278,19 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, skinny::BK, pl.nt,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
+    // scale/bias tiles by TMA need a 16-byte row pitch and chunk-aligned groups
+    const bool param_tma = (G % skinny::CG) == 0;
+    CUtensorMap ms = mc, mb = mc;
+    if (param_tma) {
+        if ((s = encode_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, G, N, G * 2, skinny::CG, skinny::BW,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+            return s;
+        if ((s = encode_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, biases, G, N, G * 2, skinny::CG, skinny::BW,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+            return s;
+    }
     skinny::Params p;
+    p.param_tma = param_tma ? 1 : 0;
     p.partial = static_cast<float*>(ws);
     p.scales = static_cast<const __half*>(scales);
     p.biases = static_cast<const __half*>(biases);
@@ -291,9 +303,9 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     p.segmax = pl.segmax;
     prof_begin(st);
     if (pl.nt == 16)
-        skinny::skinny_kernel<16><<<pl.ctas, skinny::kThreads, skinny::Layout<16>::kSmemBytes, st>>>(mc, mx, p);
+        skinny::skinny_kernel<16><<<pl.ctas, skinny::kThreads, skinny::Layout<16>::kSmemBytes, st>>>(mc, mx, ms, mb, p);
     else
-        skinny::skinny_kernel<32><<<pl.ctas, skinny::kThreads, skinny::Layout<32>::kSmemBytes, st>>>(mc, mx, p);
+        skinny::skinny_kernel<32><<<pl.ctas, skinny::kThreads, skinny::Layout<32>::kSmemBytes, st>>>(mc, mx, ms, mb, p);
     prof_end(st);
     const int64_t total = M * N;
     const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4 * sm_count));

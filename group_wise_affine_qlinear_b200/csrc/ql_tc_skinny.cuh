@@ -23,7 +23,8 @@
 // that covered its tile in CTA order (deterministic) and rounds to bf16.
 //
 // Warp roles (384 threads, one CTA per SM):
-//   warp 0       TMA producer: code chunk (128 rows x CG*32 B) + CG activation tiles (NT x 64), all 128B-swizzled
+//   warp 0       TMA producer: L2 prefetch of the code chunk PD chunks ahead, then the code chunk
+//                (128 rows x CG*32 B) + CG activation tiles (NT x 64), all 128B-swizzled
 //   warps 1, 3   MMA issuers for even / odd groups (warp 1 also allocates TMEM)
 //   warp 2       per-group activation sums xsum_g[t] from the staged activation tile
 //   warps 4-7    A builders: one weight row per thread, codes -> bf16 (128+q) pairs -> TMEM
@@ -42,21 +43,26 @@ constexpr int kThreads = 12 * 32;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpXsum = 2, kWarpMma2 = 3, kWarpBuild0 = 4, kWarpDrain0 = 8;
 constexpr int CG = 8;                    // groups per chunk (one TMA stage), a multiple of 4
 constexpr int kBoxGroups = 4;            // groups per code box: 128 bytes of each row (the 128B-swizzle span)
+constexpr int PD = 12;                   // chunks of codes prefetched into L2 ahead of the shared-memory loads
 constexpr int NA = 4;                    // TMEM A stages (32 columns each)
 constexpr int ND = 8;                    // TMEM accumulator buffers (NT columns each)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBoxBytes = BW * BK / 2 * kBoxGroups;   // 16 KB: one code box
 constexpr uint32_t kCBytes = kBoxBytes * (CG / kBoxGroups);  // codes per chunk
+constexpr int PR = 4;                                         // params ring depth (chunks)
+constexpr uint32_t kParHalf = BW * CG * 2;                    // one chunk's scales (or biases): [128][CG] f16
+constexpr uint32_t kParBytes = 2 * kParHalf;
 
 template <int NT>
 struct Layout {
     static constexpr uint32_t kXBytes = NT * BK * 2;                // one group's activation tile
     static constexpr uint32_t kStageBytes = kCBytes + CG * kXBytes;
-    static constexpr int NS = static_cast<int>(196608 / kStageBytes);   // TMA stages in 192 KB
+    static constexpr int NS = static_cast<int>(212992 / kStageBytes);   // TMA stages (208 KB budget)
     static constexpr uint32_t kOffStage = 0;                       // [NS][codes | x_0 .. x_3], 1 KB aligned
     static constexpr uint32_t kOffXs = NS * kStageBytes;          // xsum ring [ND][NT] fp32
-    static constexpr uint32_t kOffBar = kOffXs + ND * NT * 4;
-    static constexpr uint32_t kNumBars = 2 * NS + 2 * NA + 3 * ND + 2;
+    static constexpr uint32_t kOffPar = kOffXs + ND * NT * 4;      // params ring [PR][scales|biases][128][CG] f16
+    static constexpr uint32_t kOffBar = kOffPar + PR * kParBytes;
+    static constexpr uint32_t kNumBars = 2 * NS + 2 * NA + 3 * ND + 2 * PR + 2;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
     static constexpr uint32_t kAccCol = 0;                          // D buffer j at [j*NT, (j+1)*NT)
@@ -69,6 +75,7 @@ struct Layout {
 
 struct Params {
     float* partial;          // [P][segmax][M][128] fp32
+    int param_tma;           // 1: scales/biases arrive by TMA tiles (needs G % CG == 0); 0: per-group loads
     const __half* scales;    // [N][G]
     const __half* biases;    // [N][G]
     int M, N, G, num_w;
@@ -101,6 +108,8 @@ __device__ __forceinline__ void codes_to_bf16(uint32_t v, uint32_t* o) {
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_constant__ CUtensorMap map_codes,
                                                             const __grid_constant__ CUtensorMap map_x,
+                                                            const __grid_constant__ CUtensorMap map_scales,
+                                                            const __grid_constant__ CUtensorMap map_biases,
                                                             const Params p) {
     using L = Layout<NT>;
     constexpr int NS = L::NS;
@@ -114,7 +123,9 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     uint64_t* d_full = a_empty + NA;
     uint64_t* d_empty = d_full + ND;
     uint64_t* xs_full = d_empty + ND;
-    uint64_t* drain = xs_full + ND;
+    uint64_t* p_full = xs_full + ND;
+    uint64_t* p_empty = p_full + PR;
+    uint64_t* drain = p_empty + PR;
     float* xs = reinterpret_cast<float*>(smem + L::kOffXs);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
@@ -135,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
             ptx::mbar_init(&d_empty[i], 4);
             ptx::mbar_init(&xs_full[i], 1);
         }
+        for (int i = 0; i < PR; ++i) { ptx::mbar_init(&p_full[i], 1); ptx::mbar_init(&p_empty[i], 4); }
         ptx::mbar_init(drain, 1);
         ptx::mbar_init(drain + 1, 1);
         *abort_flag = 0;
@@ -143,6 +155,10 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     if (warp == kWarpTma && lane == 0) {
         ptx::prefetch_tensormap(&map_codes);
         ptx::prefetch_tensormap(&map_x);
+        if (p.param_tma) {
+            ptx::prefetch_tensormap(&map_scales);
+            ptx::prefetch_tensormap(&map_biases);
+        }
     }
     if (warp == kWarpMma) {
         ptx::tmem_alloc(tmem_slot, kTmemCols);
@@ -164,14 +180,35 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     if (warp == kWarpTma) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
-            uint32_t i = 0;
+            // HBM needs far more bytes in flight than the shared-memory stages hold: the code
+            // boxes of chunk i + PD are prefetched into L2 while chunk i is loaded from there.
+            auto prefetch = [&](uint32_t k) {
+                int w, g0, ng;
+                chunk_groups(u0 + k, w, g0, ng);
+#pragma unroll
+                for (int bx = 0; bx < CG / kBoxGroups; ++bx)
+                    ptx::tma_prefetch_2d(&map_codes, (g0 + bx * kBoxGroups) * (BK / 8), w * BW);
+            };
+            for (uint32_t k = 0; k < nchunks && k < static_cast<uint32_t>(PD); ++k) prefetch(k);
+            uint32_t i = 0, pi = 0;     // chunks whose codes / whose params were issued
             for (; i < nchunks; ++i) {
                 const int s = static_cast<int>(i % NS);
                 const uint32_t ph = (i / NS) & 1u;
+                if (i + PD < nchunks) prefetch(i + PD);
                 if (!ptx::mbar_wait(&s_empty[s], ph ^ 1, abort_flag)) break;
                 int w, g0, ng;
                 chunk_groups(u0 + i, w, g0, ng);
                 uint8_t* st = smem + L::kOffStage + s * L::kStageBytes;
+                if (p.param_tma) {
+                    // the drain reads each chunk's scales and biases from a small ring of its own
+                    const int pr = static_cast<int>(i % PR);
+                    if (!ptx::mbar_wait(&p_empty[pr], ((i / PR) & 1u) ^ 1u, abort_flag)) break;
+                    uint8_t* pt = smem + L::kOffPar + pr * kParBytes;
+                    ptx::mbar_arrive_expect_tx(&p_full[pr], kParBytes);
+                    ptx::tma_load_2d(pt, &map_scales, &p_full[pr], g0, w * BW);
+                    ptx::tma_load_2d(pt + kParHalf, &map_biases, &p_full[pr], g0, w * BW);
+                    ++pi;
+                }
                 ptx::mbar_arrive_expect_tx(&s_full[s], L::kStageBytes);
 #pragma unroll
                 for (int bx = 0; bx < CG / kBoxGroups; ++bx)   // consecutive boxes: longer contiguous row segments
@@ -182,6 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
             }
             for (uint32_t j = (i > static_cast<uint32_t>(NS) ? i - NS : 0u); j < i; ++j)
                 ptx::mbar_wait(&s_full[j % NS], (j / NS) & 1u, nullptr);
+            for (uint32_t j = (pi > static_cast<uint32_t>(PR) ? pi - PR : 0u); j < pi; ++j)
+                ptx::mbar_wait(&p_full[j % PR], (j / PR) & 1u, nullptr);
         }
     } else if (warp == kWarpMma || warp == kWarpMma2) {
         // ---------------------------------------------------------------- MMA issuers (even / odd groups)
@@ -308,15 +347,37 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
             int w, g0, ng;
             chunk_groups(u0 + i, w, g0, ng);
             const int n = w * BW + r;
-            for (int q = 0; q < ng; ++q, ++gi) {
+            // this chunk's scales and biases of row r: from the params ring, else from global memory
+            __half sv[CG], bv[CG];
+            if (p.param_tma) {
+                const int pr = static_cast<int>(i % PR);
+                const bool got = ptx::mbar_wait(&p_full[pr], (i / PR) & 1u, abort_flag);
+                if (!__all_sync(0xFFFFFFFFu, got)) break;
+                const uint8_t* pt = smem + L::kOffPar + pr * kParBytes;
+#pragma unroll
+                for (int c = 0; c < CG / 8; ++c) {
+                    *reinterpret_cast<uint4*>(sv + 8 * c) = reinterpret_cast<const uint4*>(pt + r * CG * 2)[c];
+                    *reinterpret_cast<uint4*>(bv + 8 * c) = reinterpret_cast<const uint4*>(pt + kParHalf + r * CG * 2)[c];
+                }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&p_empty[pr]);
+            } else {
+#pragma unroll
+                for (int q = 0; q < CG; ++q) {
+                    const bool in = n < p.N && q < ng;
+                    sv[q] = in ? __ldg(p.scales + static_cast<int64_t>(n) * p.G + g0 + q) : __float2half_rn(0.0f);
+                    bv[q] = in ? __ldg(p.biases + static_cast<int64_t>(n) * p.G + g0 + q) : __float2half_rn(0.0f);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < CG; ++q, ++gi) {
+                if (q >= ng) break;
                 const int j = static_cast<int>(gi % ND);
-                const int g = g0 + q;
                 float sc = 0.0f, cc = 0.0f;
                 if (n < p.N) {
-                    const float s_ = __half2float(__ldg(p.scales + static_cast<int64_t>(n) * p.G + g));
-                    const float b_ = __half2float(__ldg(p.biases + static_cast<int64_t>(n) * p.G + g));
+                    const float s_ = __half2float(sv[q]);
                     sc = s_;
-                    cc = fmaf(-128.0f, s_, b_);
+                    cc = fmaf(-128.0f, s_, __half2float(bv[q]));
                 }
                 bool got = ptx::mbar_wait(&d_full[j], (gi / ND) & 1u, abort_flag);
                 got = got && ptx::mbar_wait(&xs_full[j], (gi / ND) & 1u, abort_flag);
