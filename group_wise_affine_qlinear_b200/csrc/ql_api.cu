@@ -169,7 +169,7 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         const int64_t run = (plan->units + plan->ctas - 1) / plan->ctas;
         plan->segmax = static_cast<int>((run + cpt - 1) / cpt + 1);
         plan->split_k = 1;
-        plan->workspace = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * M * skinny::BW * sizeof(float), 256);
+        plan->workspace = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * 2 * M * skinny::BW * sizeof(float), 256);
         return QL_OK;
     }
     if (path == QL_PATH_TC_FUSED) {
