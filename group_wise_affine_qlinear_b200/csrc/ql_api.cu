@@ -147,6 +147,8 @@ struct Plan {
     size_t workspace = 0;
     // fused path workspace carve-up
     size_t off_xh = 0, off_rs = 0, off_sb = 0;
+    // skinny path workspace carve-up: partials, reordered activations, activation sums
+    size_t off_xp = 0, off_xs = 0;
 };
 
 ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int sm_count, Plan* plan) {
@@ -169,7 +171,9 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         const int64_t run = (plan->units + plan->ctas - 1) / plan->ctas;
         plan->segmax = static_cast<int>((run + cpt - 1) / cpt + 1);
         plan->split_k = 1;
-        plan->workspace = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * 2 * M * skinny::BW * sizeof(float), 256);
+        plan->off_xp = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * 2 * M * skinny::BW * sizeof(float), 256);
+        plan->off_xs = plan->off_xp + round_up(static_cast<size_t>(M) * K * 2, 256);
+        plan->workspace = plan->off_xs + round_up(static_cast<size_t>(G) * plan->nt * sizeof(float), 256);
         return QL_OK;
     }
     if (path == QL_PATH_TC_FUSED) {
@@ -266,17 +270,41 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     return launch_status();
 }
 
+// Launches with programmatic stream serialization: the kernel may start while the previous
+// kernel on the stream is still running and waits for it (griddepcontrol.wait) where it must.
+template <typename... KArgs, typename... Args>
+ql_status launch_dependent(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st,
+                           Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(block));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}
+
 ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const void* scales, const void* biases,
                      void* y, bool bf16_out, int64_t M, int64_t K, int64_t N, void* ws, cudaStream_t st,
                      int sm_count) {
     const int64_t G = K / kGroup;
-    CUtensorMap mc, mx;
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    void* xp = wsb + pl.off_xp;
+    float* xs = reinterpret_cast<float*>(wsb + pl.off_xs);
+    CUtensorMap mc, mx, mxs;
     ql_status s;
     if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K / 8, N, K / 2,
                        skinny::kBoxGroups * skinny::BK / 8, skinny::BW, CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
-    if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, skinny::BK, pl.nt,
+    if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xp, K, M, K * 2, skinny::BK, pl.nt,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
+        return s;
+    if ((s = encode_2d(&mxs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, xs, pl.nt, G, pl.nt * 4, pl.nt, skinny::CG,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
         return s;
     // scale/bias tiles by TMA need a 16-byte row pitch and chunk-aligned groups
     const bool param_tma = (G % skinny::CG) == 0;
@@ -291,7 +319,7 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     }
     skinny::Params p;
     p.param_tma = param_tma ? 1 : 0;
-    p.partial = static_cast<float*>(ws);
+    p.partial = reinterpret_cast<float*>(wsb);
     p.scales = static_cast<const __half*>(scales);
     p.biases = static_cast<const __half*>(biases);
     p.M = static_cast<int>(M);
@@ -301,21 +329,31 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     p.cpt = static_cast<int>((G + skinny::CG - 1) / skinny::CG);
     p.units = pl.units;
     p.segmax = pl.segmax;
+    // reordered activations and per-group activation sums
+    const int64_t pre_threads = static_cast<int64_t>(pl.nt) * (K / 8);
+    skinny::skinny_prepass_kernel<<<static_cast<unsigned>((pre_threads + 255) / 256), 256, 0, st>>>(
+        static_cast<const uint4*>(x), static_cast<uint4*>(xp), xs, p.M, static_cast<int>(K), pl.nt);
+    if ((s = launch_status()) != QL_OK) return s;
     prof_begin(st);
     if (pl.nt == 16)
-        skinny::skinny_kernel<16><<<pl.ctas, skinny::kThreads, skinny::Layout<16>::kSmemBytes, st>>>(mc, mx, ms, mb, p);
+        s = launch_dependent(skinny::skinny_kernel<16>, pl.ctas, skinny::kThreads, skinny::Layout<16>::kSmemBytes, st,
+                             mc, mx, ms, mb, mxs, p);
     else
-        skinny::skinny_kernel<32><<<pl.ctas, skinny::kThreads, skinny::Layout<32>::kSmemBytes, st>>>(mc, mx, ms, mb, p);
+        s = launch_dependent(skinny::skinny_kernel<32>, pl.ctas, skinny::kThreads, skinny::Layout<32>::kSmemBytes, st,
+                             mc, mx, ms, mb, mxs, p);
+    if (s != QL_OK) return s;
     prof_end(st);
     const int64_t total = M * N;
     const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4 * sm_count));
+    const float* part = p.partial;
     if (bf16_out)
-        skinny::skinny_reduce_kernel<true><<<blocks, 256, 0, st>>>(p.partial, y, p.M, p.N, p.cpt, p.units, pl.ctas,
-                                                                  pl.segmax);
+        s = launch_dependent(skinny::skinny_reduce_kernel<true>, blocks, 256, 0, st, part, y, p.M, p.N, p.cpt,
+                             p.units, pl.ctas, pl.segmax);
     else
-        skinny::skinny_reduce_kernel<false><<<blocks, 256, 0, st>>>(p.partial, y, p.M, p.N, p.cpt, p.units, pl.ctas,
-                                                                   pl.segmax);
-    set_dispatch("path=tc_skinny nt=%d ctas=%d segmax=%d units=%lld launches=2", pl.nt, pl.ctas, pl.segmax,
+        s = launch_dependent(skinny::skinny_reduce_kernel<false>, blocks, 256, 0, st, part, y, p.M, p.N, p.cpt,
+                             p.units, pl.ctas, pl.segmax);
+    if (s != QL_OK) return s;
+    set_dispatch("path=tc_skinny nt=%d ctas=%d segmax=%d units=%lld launches=3", pl.nt, pl.ctas, pl.segmax,
                  static_cast<long long>(pl.units));
     return launch_status();
 }

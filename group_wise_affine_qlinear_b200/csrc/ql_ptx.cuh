@@ -64,6 +64,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Lets the next kernel on the stream (launched with programmatic stream
+// serialization) be scheduled before this grid finishes; it must still call
+// grid_dependency_wait before it reads anything this grid writes.
+__device__ __forceinline__ void launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the grids this one depends on have completed and their writes
+// are visible; returns at once for a kernel launched without the dependency.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {

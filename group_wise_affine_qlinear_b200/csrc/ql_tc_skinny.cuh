@@ -9,32 +9,38 @@
 // here": w = scale * q + bias).  128 + q is exact in bf16 (unit 1 at 128), so the
 // tensor core sees the exact codes and the exact bf16 activations; the scale and
 // bias are applied in fp32 per (row, group, token).  The A operand is built from
-// the code nibbles with two byte permutes and an OR per pair of weights and is
+// the code nibbles with one shift and one AND-OR per pair of weights and is
 // written to tensor memory (tcgen05.st); shared memory carries only the streamed
-// code chunks, the small activation tiles and the scale/bias tiles.
+// code chunks, the activation tiles and the per-chunk scale/bias/xsum tiles.
+//
+// A word of codes holds k = 0..7 in nibbles 0..7; the builder pairs nibbles j and
+// j + 4 (16 bits apart, so one AND-OR per pair), which puts k in the order
+// 0,4,1,5,2,6,3,7 along each 8-block of the MMA's reduction dimension.  A small
+// prepass kernel writes the activations in that same order, and the per-group
+// activation sums xsum_g[t], once for all CTAs.  It runs under programmatic
+// dependent launch: the main kernel starts streaming codes at once and waits for
+// the prepass only before its first activation load.
 //
 // Stream-K schedule: the work is cut into chunks of CG consecutive groups of one
 // 128-row weight tile (a tile has ceil(G/CG) chunks; a tile's last chunk may be
 // partial).  The chunks, tile-major, are split into one equal contiguous run per
 // CTA; a run covers at most a few tiles, and each covered tile segment leaves
 // fp32 partials [2][tokens][128] in the workspace (one per group parity).  A
-// second kernel sums, per output, the partials of the CTAs that covered its tile
+// reduce kernel sums, per output, the partials of the CTAs that covered its tile
 // in CTA order (deterministic) and rounds to bf16.  The code boxes of a chunk
 // bring CG * 32 contiguous bytes of each row, so DRAM sees long row segments.
 //
-// Every role works group by group through a serial chain of waits, tensor-memory
-// accesses and arithmetic, so each role runs twice: one copy takes the even
-// groups of the run, the other the odd ones, and the two chains overlap.  The
-// code chunks and the activation tiles have rings of their own, so a code stage
-// is free as soon as the builders have read it into registers.
-// Warp roles (640 threads, one CTA per SM; 5 warps per SM sub-partition leave 96 registers a thread):
-//   warp 0        TMA producer: code chunks (128 rows x CG*32 B, 128B swizzle), scale/bias tiles,
-//                 activation tiles (NT x 64 per group, 128B swizzle)
+// The builders and the drains run as two copies, on the even and the odd groups
+// of the run, and so do the MMA issuers.  Each TMEM slot s (an A stage and an
+// accumulator) serves one parity, with one barrier each way: ready[s] (A built
+// by the 4 builder warps, accumulator read by the 4 drain warps) and done[s]
+// (the slot's MMAs completed).
+// Warp roles (608 threads, one CTA per SM; at most 5 warps per SM sub-partition leave 96 registers a thread):
+//   warp 0        TMA producer: code chunks (128 rows x CG*32 B, 128B swizzle), scale/bias/xsum tiles,
+//                 activation tiles of a chunk (NT x 64 per group, 128B swizzle)
 //   warps 1, 2    MMA issuers for even / odd groups (warp 1 also allocates TMEM)
-//   warp 3        per-group activation sums xsum_g[t]
-//   warps 4-11    A builders, even groups (4-7) / odd groups (8-11): one weight row per thread,
-//                 codes -> bf16 (128+q) pairs -> TMEM
-//   warps 12-19   drain, even (12-15) / odd (16-19): one weight row per thread, fp32
+//   warps 3-10    A builders, even groups (3-6) / odd groups (7-10): one weight row per thread
+//   warps 11-18   drains, even groups (11-14) / odd groups (15-18): one weight row per thread, fp32
 //                 accumulation of s*D + c*xsum over the run
 #pragma once
 
@@ -46,39 +52,38 @@ namespace skinny {
 constexpr int BW = 128;
 constexpr int BK = 64;
 constexpr int UK = 16;
-constexpr int kWarpTma = 0, kWarpMma0 = 1, kWarpXsum = 3, kWarpBuild0 = 4, kWarpDrain0 = 12;
-constexpr int kThreads = 20 * 32;
-constexpr int CG = 8;                    // groups per code chunk, a multiple of 8
+constexpr int kWarpTma = 0, kWarpMma0 = 1, kWarpBuild0 = 3, kWarpDrain0 = 11;
+constexpr int kThreads = 19 * 32;
+constexpr int CG = 8;                    // groups per chunk
 constexpr int kBoxGroups = 4;            // groups per code box: 128 bytes of each row (the 128B-swizzle span)
-constexpr int NC = 4;                    // code chunk stages
-constexpr int PR = 4;                    // scale/bias chunk stages
-constexpr int NA = 4;                    // TMEM A stages (32 columns each), even
-constexpr int ND = 8;                    // TMEM accumulator buffers (NT columns each), even
+constexpr int NS = 8;                    // TMEM slots (A stage + accumulator), even
+constexpr int PR = 4;                    // scale/bias/xsum chunk stages
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBoxBytes = BW * BK / 2 * kBoxGroups;     // 16 KB: one code box
 constexpr uint32_t kCBytes = kBoxBytes * (CG / kBoxGroups);  // codes per chunk
 constexpr uint32_t kParHalf = BW * CG * 2;                   // one chunk's scales (or biases): [128][CG] f16
-constexpr uint32_t kParBytes = 2 * kParHalf;
 static_assert(CG % kBoxGroups == 0 && CG % 8 == 0, "whole code boxes and 16-byte scale rows per chunk");
-static_assert(NA % 2 == 0 && ND % 2 == 0, "ring slots of one group parity only");
 
 template <int NT>
 struct Layout {
-    static constexpr uint32_t kXBytes = NT * BK * 2;                    // one group's activation tile
-    static constexpr int NX = NT == 16 ? 24 : 20;                       // activation stages (one group each), even
-    static constexpr uint32_t kOffC = 0;                                 // [NC][codes], 1 KB aligned
-    static constexpr uint32_t kOffX = kOffC + NC * kCBytes;             // [NX][x tile], 1 KB aligned
-    static constexpr uint32_t kOffPar = kOffX + NX * kXBytes;           // [PR][scales|biases][128][CG]
-    static constexpr uint32_t kOffXs = kOffPar + PR * kParBytes;        // xsum ring [ND][NT] fp32
-    static constexpr uint32_t kOffBar = kOffXs + ND * NT * 4;
-    static constexpr uint32_t kNumBars = 2 * NC + 2 * PR + 2 * NX + 2 * NA + 3 * ND + 2;
+    static constexpr int NC = NT == 16 ? 4 : 3;                          // code chunk stages
+    static constexpr int NXC = NT == 16 ? 4 : 3;                         // activation chunk stages
+    static constexpr uint32_t kXTile = NT * BK * 2;                      // one group's activation tile
+    static constexpr uint32_t kXBytes = CG * kXTile;                     // one chunk's activation tiles
+    static constexpr uint32_t kXsBytes = CG * NT * 4;                    // one chunk's xsum rows [CG][NT] fp32
+    static constexpr uint32_t kParBytes = 2 * kParHalf + kXsBytes;       // [scales | biases | xsum]
+    static constexpr uint32_t kOffC = 0;                                  // [NC][codes], 1 KB aligned
+    static constexpr uint32_t kOffX = kOffC + NC * kCBytes;              // [NXC][CG][x tile], 1 KB aligned
+    static constexpr uint32_t kOffPar = kOffX + NXC * kXBytes;           // [PR][par]
+    static constexpr uint32_t kOffBar = kOffPar + PR * kParBytes;
+    static constexpr uint32_t kNumBars = 2 * NC + 2 * PR + 2 * NXC + 2 * NS + 2;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
-    static constexpr uint32_t kAccCol = 0;                               // D buffer j at [j*NT, (j+1)*NT)
-    static constexpr uint32_t kACol = ND * NT;                           // A stage a at [kACol + 32a, +32)
-    static_assert(kCBytes % 1024 == 0 && kXBytes % 1024 == 0, "stage pieces need 1 KB alignment");
-    static_assert(NX % 2 == 0, "ring slots of one group parity only");
-    static_assert(kACol + NA * 32 <= kTmemCols, "tensor memory budget");
+    static constexpr uint32_t kAccCol = 0;                                // accumulator of slot s at [s*NT, (s+1)*NT)
+    static constexpr uint32_t kACol = NS * NT;                            // A stage of slot s at [kACol + 32s, +32)
+    static_assert(kCBytes % 1024 == 0 && kXTile % 1024 == 0, "swizzled stage pieces need 1 KB alignment");
+    static_assert(kParBytes % 128 == 0, "TMA destinations 128-byte aligned");
+    static_assert(kACol + NS * 32 <= kTmemCols, "tensor memory budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -98,20 +103,42 @@ __host__ __device__ __forceinline__ int64_t run_first(int64_t units, int P, int 
     return units * c / P;
 }
 
-// Codes word (8 codes, k order 0..7) -> 4 words of bf16 pairs (128+q_2t, 128+q_2t+1), k order kept.
-// prmt selector nibble = byte index (0-3 from a, 4-7 from b); bit 3 set replicates the
-// selected byte's sign bit, which is 0 for a code byte, giving 0x00.
+// Codes word (code j in nibble j) -> 4 words of bf16 pairs (128 + code j, 128 + code j+4), j = 0..3.
 __device__ __forceinline__ void codes_to_bf16(uint32_t v, uint32_t* o) {
-    const uint32_t lo = v & 0x0F0F0F0Fu;            // q0 q2 q4 q6
-    const uint32_t hi = (v >> 4) & 0x0F0F0F0Fu;     // q1 q3 q5 q7
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const uint32_t sel = static_cast<uint32_t>(t) | (static_cast<uint32_t>(8 | t) << 4) |
-                             (static_cast<uint32_t>(4 + t) << 8) | (static_cast<uint32_t>(12 + t) << 12);
-        uint32_t w;
-        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(w) : "r"(lo), "r"(hi), "r"(sel));
-        o[t] = w | 0x43004300u;
+    o[0] = (v & 0x000F000Fu) | 0x43004300u;
+    o[1] = ((v >> 4) & 0x000F000Fu) | 0x43004300u;
+    o[2] = ((v >> 8) & 0x000F000Fu) | 0x43004300u;
+    o[3] = ((v >> 12) & 0x000F000Fu) | 0x43004300u;
+}
+
+// x [M][K] bf16 -> xp [M][K] with each 8-block of k in the order 0,4,1,5,2,6,3,7, and
+// xsum[g][t] = sum over group g of x[t][k] in fp32 for t < NT (zero for t >= M).
+// One thread per (row, 8-block); the 8 threads of a group are 8 aligned lanes.
+__global__ void __launch_bounds__(256) skinny_prepass_kernel(const uint4* __restrict__ x, uint4* __restrict__ xp,
+                                                             float* __restrict__ xsum, int M, int K, int NT) {
+    ptx::launch_dependents();
+    const int kb = K / 8;
+    const int64_t total = static_cast<int64_t>(NT) * kb;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const bool in = idx < total;
+    const int t = in ? static_cast<int>(idx / kb) : 0;
+    const int c = in ? static_cast<int>(idx % kb) : 0;
+    float sum = 0.0f;
+    if (in && t < M) {
+        const uint4 v = x[static_cast<int64_t>(t) * kb + c];     // (k0,k1) (k2,k3) (k4,k5) (k6,k7), low half first
+        uint4 o;
+        asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(o.x) : "r"(v.x), "r"(v.z));   // (k0, k4)
+        asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(o.y) : "r"(v.x), "r"(v.z));   // (k1, k5)
+        asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(o.z) : "r"(v.y), "r"(v.w));   // (k2, k6)
+        asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(o.w) : "r"(v.y), "r"(v.w));   // (k3, k7)
+        xp[static_cast<int64_t>(t) * kb + c] = o;
+        sum = ((bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y))) +
+              ((bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w)));
     }
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
+    if (in && (c & 7) == 0) xsum[static_cast<int64_t>(c >> 3) * NT + t] = sum;
 }
 
 template <int NT>
@@ -119,9 +146,11 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
                                                             const __grid_constant__ CUtensorMap map_x,
                                                             const __grid_constant__ CUtensorMap map_scales,
                                                             const __grid_constant__ CUtensorMap map_biases,
+                                                            const __grid_constant__ CUtensorMap map_xsum,
                                                             const Params p) {
     using L = Layout<NT>;
-    constexpr int NX = L::NX;
+    constexpr int NC = L::NC;
+    constexpr int NXC = L::NXC;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
@@ -130,14 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     uint64_t* p_full = c_empty + NC;
     uint64_t* p_empty = p_full + PR;
     uint64_t* x_full = p_empty + PR;
-    uint64_t* x_empty = x_full + NX;
-    uint64_t* a_full = x_empty + NX;
-    uint64_t* a_empty = a_full + NA;
-    uint64_t* d_full = a_empty + NA;
-    uint64_t* d_empty = d_full + ND;
-    uint64_t* xs_full = d_empty + ND;
-    uint64_t* drain = xs_full + ND;             // two: one per MMA issuer
-    float* xs = reinterpret_cast<float*>(smem + L::kOffXs);
+    uint64_t* x_empty = x_full + NXC;
+    uint64_t* ready = x_empty + NXC;
+    uint64_t* done = ready + NS;
+    uint64_t* drain = done + NS;                // two: one per MMA issuer
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
 
@@ -149,17 +174,10 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     const uint32_t nchunks = static_cast<uint32_t>(u1 - u0);
 
     if (threadIdx.x == 0) {
-        // a code stage is free once all 8 builder warps hold it in registers
         for (int i = 0; i < NC; ++i) { ptx::mbar_init(&c_full[i], 1); ptx::mbar_init(&c_empty[i], 8); }
         for (int i = 0; i < PR; ++i) { ptx::mbar_init(&p_full[i], 1); ptx::mbar_init(&p_empty[i], 8); }
-        // an activation stage is free once its MMAs (one commit) and the xsum warp are done with it
-        for (int i = 0; i < NX; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], 2); }
-        for (int i = 0; i < NA; ++i) { ptx::mbar_init(&a_full[i], 4); ptx::mbar_init(&a_empty[i], 1); }
-        for (int i = 0; i < ND; ++i) {
-            ptx::mbar_init(&d_full[i], 1);
-            ptx::mbar_init(&d_empty[i], 4);
-            ptx::mbar_init(&xs_full[i], 1);
-        }
+        for (int i = 0; i < NXC; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], 2); }
+        for (int i = 0; i < NS; ++i) { ptx::mbar_init(&ready[i], 8); ptx::mbar_init(&done[i], 1); }
         ptx::mbar_init(drain, 1);
         ptx::mbar_init(drain + 1, 1);
         *abort_flag = 0;
@@ -168,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     if (warp == kWarpTma && lane == 0) {
         ptx::prefetch_tensormap(&map_codes);
         ptx::prefetch_tensormap(&map_x);
+        ptx::prefetch_tensormap(&map_xsum);
         if (p.param_tma) {
             ptx::prefetch_tensormap(&map_scales);
             ptx::prefetch_tensormap(&map_biases);
@@ -181,11 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     __syncthreads();
     ptx::tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
+    ptx::launch_dependents();
 
-    // chunk u -> tile w = u / cpt, groups g = (u % cpt) * CG + q, q < ng.
-    // Groups are numbered gi along the run; group gi belongs to the role copies of parity gi & 1
-    // and uses activation stage gi % NX, TMEM A stage gi % NA and accumulator gi % ND (all even
-    // ring sizes, so every slot serves one parity only).
+    // chunk u -> tile w = u / cpt, groups g = (u % cpt) * CG + q, q < ng.  Groups are numbered
+    // gi along the run; group gi belongs to the copies of parity gi & 1 and uses TMEM slot gi % NS.
     auto chunk_groups = [&](int64_t u, int& w, int& g0, int& ng) {
         w = static_cast<int>(u / p.cpt);
         g0 = static_cast<int>(u % p.cpt) * CG;
@@ -195,34 +213,51 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     if (warp == kWarpTma) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
-            uint32_t i = 0, pi = 0, ci = 0, gi = 0;   // chunks started / with scales+biases / with codes; x tiles
-            bool ok = true;
-            for (; i < nchunks && ok; ++i) {
+            uint32_t ci = 0, pi = 0, xi = 0;     // chunks whose codes / parameters / activations were issued
+            auto issue_codes = [&](uint32_t i) -> bool {
                 int w, g0, ng;
                 chunk_groups(u0 + i, w, g0, ng);
-                if (p.param_tma) {
-                    const int pr = static_cast<int>(i % PR);
-                    if (!ptx::mbar_wait(&p_empty[pr], ((i / PR) & 1u) ^ 1u, abort_flag)) break;
-                    uint8_t* pt = smem + L::kOffPar + pr * kParBytes;
-                    ptx::mbar_arrive_expect_tx(&p_full[pr], kParBytes);
-                    ptx::tma_load_2d(pt, &map_scales, &p_full[pr], g0, w * BW);
-                    ptx::tma_load_2d(pt + kParHalf, &map_biases, &p_full[pr], g0, w * BW);
-                    ++pi;
-                }
                 const int s = static_cast<int>(i % NC);
-                if (!ptx::mbar_wait(&c_empty[s], ((i / NC) & 1u) ^ 1u, abort_flag)) break;
+                if (!ptx::mbar_wait(&c_empty[s], ((i / NC) & 1u) ^ 1u, abort_flag)) return false;
                 uint8_t* st = smem + L::kOffC + s * kCBytes;
                 ptx::mbar_arrive_expect_tx(&c_full[s], kCBytes);
 #pragma unroll
                 for (int bx = 0; bx < CG / kBoxGroups; ++bx)   // consecutive boxes: long contiguous row segments
                     ptx::tma_load_2d(st + bx * kBoxBytes, &map_codes, &c_full[s], (g0 + bx * kBoxGroups) * (BK / 8), w * BW);
-                ++ci;
-                for (int q = 0; q < ng; ++q) {
-                    const int xst = static_cast<int>(gi % NX);
-                    if (!ptx::mbar_wait(&x_empty[xst], ((gi / NX) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-                    ptx::mbar_arrive_expect_tx(&x_full[xst], L::kXBytes);
-                    ptx::tma_load_2d(smem + L::kOffX + xst * L::kXBytes, &map_x, &x_full[xst], (g0 + q) * BK, 0);
-                    ++gi;
+                return true;
+            };
+            // the codes do not depend on the prepass: start streaming them at once
+            bool ok = true;
+            while (ok && ci < nchunks && ci < static_cast<uint32_t>(NC)) {
+                ok = issue_codes(ci);
+                if (ok) ++ci;
+            }
+            ptx::grid_dependency_wait();
+            for (uint32_t i = 0; i < nchunks && ok; ++i) {
+                int w, g0, ng;
+                chunk_groups(u0 + i, w, g0, ng);
+                // scales, biases and activation sums of the chunk
+                const int pr = static_cast<int>(i % PR);
+                if (!ptx::mbar_wait(&p_empty[pr], ((i / PR) & 1u) ^ 1u, abort_flag)) break;
+                uint8_t* pt = smem + L::kOffPar + pr * L::kParBytes;
+                ptx::mbar_arrive_expect_tx(&p_full[pr], (p.param_tma ? 2 * kParHalf : 0u) + L::kXsBytes);
+                if (p.param_tma) {
+                    ptx::tma_load_2d(pt, &map_scales, &p_full[pr], g0, w * BW);
+                    ptx::tma_load_2d(pt + kParHalf, &map_biases, &p_full[pr], g0, w * BW);
+                }
+                ptx::tma_load_2d(pt + 2 * kParHalf, &map_xsum, &p_full[pr], 0, g0);   // rows past G read zeros
+                ++pi;
+                // activation tiles of the chunk
+                const int xc = static_cast<int>(i % NXC);
+                if (!ptx::mbar_wait(&x_empty[xc], ((i / NXC) & 1u) ^ 1u, abort_flag)) break;
+                ptx::mbar_arrive_expect_tx(&x_full[xc], static_cast<uint32_t>(ng) * L::kXTile);
+                for (int q = 0; q < ng; ++q)
+                    ptx::tma_load_2d(smem + L::kOffX + xc * L::kXBytes + q * L::kXTile, &map_x, &x_full[xc], (g0 + q) * BK, 0);
+                ++xi;
+                // codes run NC chunks ahead
+                if (ci < nchunks) {
+                    if (!issue_codes(ci)) break;
+                    ++ci;
                 }
             }
             // never leave the CTA with bulk copies still landing in its shared memory
@@ -230,76 +265,51 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
                 ptx::mbar_wait(&c_full[j % NC], (j / NC) & 1u, nullptr);
             for (uint32_t j = (pi > static_cast<uint32_t>(PR) ? pi - PR : 0u); j < pi; ++j)
                 ptx::mbar_wait(&p_full[j % PR], (j / PR) & 1u, nullptr);
-            for (uint32_t j = (gi > static_cast<uint32_t>(NX) ? gi - NX : 0u); j < gi; ++j)
-                ptx::mbar_wait(&x_full[j % NX], (j / NX) & 1u, nullptr);
+            for (uint32_t j = (xi > static_cast<uint32_t>(NXC) ? xi - NXC : 0u); j < xi; ++j)
+                ptx::mbar_wait(&x_full[j % NXC], (j / NXC) & 1u, nullptr);
         }
     } else if (warp == kWarpMma0 || warp == kWarpMma0 + 1) {
         // ---------------------------------------------------------------- MMA issuers (even / odd groups)
+        // The whole warp runs the loop, so the addresses stay warp-uniform; lane 0 issues.
         const uint32_t par = static_cast<uint32_t>(warp - kWarpMma0);
-        if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_f16(BW, NT, true);
-            uint32_t gi = 0;
-            bool ok = true;
-            for (uint32_t i = 0; i < nchunks && ok; ++i) {
-                int w, g0, ng;
-                chunk_groups(u0 + i, w, g0, ng);
-                for (int q = 0; q < ng; ++q, ++gi) {
-                    if ((gi & 1u) != par) continue;
-                    const int xst = static_cast<int>(gi % NX), a = static_cast<int>(gi % NA);
-                    const int j = static_cast<int>(gi % ND);
-                    if (!ptx::mbar_wait(&x_full[xst], (gi / NX) & 1u, abort_flag)) { ok = false; break; }
-                    if (!ptx::mbar_wait(&a_full[a], (gi / NA) & 1u, abort_flag)) { ok = false; break; }
-                    if (!ptx::mbar_wait(&d_empty[j], ((gi / ND) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after_sync();
-                    const uint32_t x_addr = ptx::smem_addr(smem + L::kOffX + xst * L::kXBytes);
-                    const uint32_t d = tmem_base + L::kAccCol + static_cast<uint32_t>(j * NT);
-                    const uint32_t a_tm = tmem_base + L::kACol + 32u * a;
-#pragma unroll
-                    for (int u = 0; u < BK / UK; ++u)
-                        ptx::mma_f16_ts(d, a_tm + u * (UK / 2), ptx::sdesc_sw128(x_addr + u * UK * 2), idesc, u != 0);
-                    ptx::mma_commit(&x_empty[xst]);
-                    ptx::mma_commit(&a_empty[a]);
-                    ptx::mma_commit(&d_full[j]);
-                }
-            }
-            ptx::mma_commit(drain + par);
-            ptx::mbar_wait(drain + par, 0, nullptr);
-        }
-    } else if (warp == kWarpXsum) {
-        // ---------------------------------------------------------------- activation sums per group
-        // NT = 32: lane t sums all of token row t; NT = 16: lanes t and t+16 each sum half of row t
+        constexpr uint32_t idesc = ptx::idesc_f16(BW, NT, true);
+        const uint32_t x_base = ptx::smem_addr(smem + L::kOffX);
         uint32_t gi = 0;
         bool ok = true;
         for (uint32_t i = 0; i < nchunks && ok; ++i) {
             int w, g0, ng;
             chunk_groups(u0 + i, w, g0, ng);
-            for (int q = 0; q < ng; ++q, ++gi) {
-                const int xst = static_cast<int>(gi % NX), j = static_cast<int>(gi % ND);
-                bool got = ptx::mbar_wait(&x_full[xst], (gi / NX) & 1u, abort_flag);
-                got = got && ptx::mbar_wait(&d_empty[j], ((gi / ND) & 1u) ^ 1u, abort_flag);
+            const int xc = static_cast<int>(i % NXC);
+            bool got = ptx::mbar_wait(&x_full[xc], (i / NXC) & 1u, abort_flag);
+            if (!__all_sync(0xFFFFFFFFu, got)) break;
+            for (int q = static_cast<int>((par - gi) & 1u); q < ng; q += 2) {
+                const uint32_t gq = gi + static_cast<uint32_t>(q);
+                const int sl = static_cast<int>(gq % NS);
+                got = ptx::mbar_wait(&ready[sl], (gq / NS) & 1u, abort_flag);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
-                const uint8_t* xt = smem + L::kOffX + xst * L::kXBytes;
-                const int row = (NT == 32) ? lane : (lane & 15);
-                const int c0 = (NT == 32) ? 0 : ((lane >> 4) * 4), nc = (NT == 32) ? 8 : 4;
-                float acc = 0.0f;
-                for (int c = c0; c < c0 + nc; ++c) {          // 16-byte piece c of the row (swizzled position)
-                    const uint4 v = *reinterpret_cast<const uint4*>(xt + row * 128 + ((c ^ (row & 7)) << 4));
-                    acc += (bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y)) +
-                           (bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w));
-                }
-                if (NT == 16) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 16);
-                if (lane < NT) xs[j * NT + lane] = acc;
-                __syncwarp();
+                ptx::tc_fence_after_sync();
+                const uint32_t xa = x_base + static_cast<uint32_t>(xc) * L::kXBytes + static_cast<uint32_t>(q) * L::kXTile;
+                const uint32_t d = tmem_base + L::kAccCol + static_cast<uint32_t>(sl * NT);
+                const uint32_t a_tm = tmem_base + L::kACol + 32u * static_cast<uint32_t>(sl);
                 if (lane == 0) {
-                    ptx::mbar_arrive(&xs_full[j]);
-                    ptx::mbar_arrive(&x_empty[xst]);
+#pragma unroll
+                    for (int u = 0; u < BK / UK; ++u)
+                        ptx::mma_f16_ts(d, a_tm + u * (UK / 2), ptx::sdesc_sw128(xa + u * UK * 2), idesc, u != 0);
+                    ptx::mma_commit(&done[sl]);
                 }
+                __syncwarp();
             }
+            if (ok && lane == 0) ptx::mma_commit(&x_empty[xc]);
+            __syncwarp();
+            gi += static_cast<uint32_t>(ng);
         }
+        if (lane == 0) ptx::mma_commit(drain + par);
+        __syncwarp();
+        ptx::mbar_wait(drain + par, 0, nullptr);
     } else if (warp >= kWarpBuild0 && warp < kWarpDrain0) {
         // ---------------------------------------------------------------- A builders (even / odd groups)
         const uint32_t par = static_cast<uint32_t>((warp - kWarpBuild0) >> 2);
-        const int quarter = warp & 3;
+        const int quarter = warp & 3;                      // TMEM lanes 32*quarter.. belong to this warp
         const int r = quarter * 32 + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         uint32_t gi = 0;
@@ -333,29 +343,33 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
                 const int q = q0 + 2 * k;
                 if (q >= ng) break;
                 const uint32_t gq = gi + static_cast<uint32_t>(q);
-                const int a = static_cast<int>(gq % NA);
+                const int sl = static_cast<int>(gq % NS);
                 const uint4 c0 = cw[2 * k], c1 = cw[2 * k + 1];
                 const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
                 uint32_t av[32];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) codes_to_bf16(words[c], &av[4 * c]);
-                got = ptx::mbar_wait(&a_empty[a], ((gq / NA) & 1u) ^ 1u, abort_flag);
+                // the slot's previous MMAs must have finished reading its A stage
+                got = ptx::mbar_wait(&done[sl], ((gq / NS) & 1u) ^ 1u, abort_flag);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
                 ptx::tc_fence_after_sync();
-                ptx::tmem_st_32x32b_x32(tmem_base + lane_addr + L::kACol + 32u * a, av);
+                ptx::tmem_st_32x32b_x32(tmem_base + lane_addr + L::kACol + 32u * sl, av);
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before_sync();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&a_full[a]);
+                if (lane == 0) ptx::mbar_arrive(&ready[sl]);
             }
             gi += static_cast<uint32_t>(ng);
         }
     } else if (warp >= kWarpDrain0) {
-        // ---------------------------------------------------------------- drain (even / odd groups)
+        // ---------------------------------------------------------------- drains (even / odd groups)
         const uint32_t par = static_cast<uint32_t>((warp - kWarpDrain0) >> 2);
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        // a slot's first use has no accumulator to read back: arrive for it in advance
+        if (lane == 0)
+            for (int sl = static_cast<int>(par); sl < NS; sl += 2) ptx::mbar_arrive(&ready[sl]);
         float yacc[NT];
 #pragma unroll
         for (int t = 0; t < NT; ++t) yacc[t] = 0.0f;
@@ -367,22 +381,19 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
             chunk_groups(u0 + i, w, g0, ng);
             const int n = w * BW + r;
             const int q0 = static_cast<int>((par - gi) & 1u);
-            // this copy's scales and biases of row r in this chunk (groups q0, q0 + 2, ...): from the
-            // scale/bias ring, else from global memory
+            const int pr = static_cast<int>(i % PR);
+            bool got = ptx::mbar_wait(&p_full[pr], (i / PR) & 1u, abort_flag);
+            if (!__all_sync(0xFFFFFFFFu, got)) break;
+            const uint8_t* pt = smem + L::kOffPar + pr * L::kParBytes;
+            // this copy's scales and biases of row r (groups q0, q0 + 2, ...)
             __half sv[CG / 2], bv[CG / 2];
             if (p.param_tma) {
-                const int pr = static_cast<int>(i % PR);
-                const bool got = ptx::mbar_wait(&p_full[pr], (i / PR) & 1u, abort_flag);
-                if (!__all_sync(0xFFFFFFFFu, got)) break;
-                const uint8_t* pt = smem + L::kOffPar + pr * kParBytes;
                 __align__(16) __half sa[CG], ba[CG];
 #pragma unroll
                 for (int c = 0; c < CG / 8; ++c) {
                     *reinterpret_cast<uint4*>(sa + 8 * c) = reinterpret_cast<const uint4*>(pt + r * CG * 2)[c];
                     *reinterpret_cast<uint4*>(ba + 8 * c) = reinterpret_cast<const uint4*>(pt + kParHalf + r * CG * 2)[c];
                 }
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&p_empty[pr]);
 #pragma unroll
                 for (int k = 0; k < CG / 2; ++k) {
                     sv[k] = q0 ? sa[2 * k + 1] : sa[2 * k];
@@ -397,38 +408,37 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
                     bv[k] = in ? __ldg(p.biases + static_cast<int64_t>(n) * p.G + g0 + q) : __float2half_rn(0.0f);
                 }
             }
+            const float* xsp = reinterpret_cast<const float*>(pt + 2 * kParHalf);     // [CG][NT]
 #pragma unroll
             for (int k = 0; k < CG / 2; ++k) {
                 const int q = q0 + 2 * k;
                 if (q >= ng) break;
                 const uint32_t gq = gi + static_cast<uint32_t>(q);
-                const int j = static_cast<int>(gq % ND);
+                const int sl = static_cast<int>(gq % NS);
                 float sc = 0.0f, cc = 0.0f;
                 if (n < p.N) {
                     sc = __half2float(sv[k]);
                     cc = fmaf(-128.0f, sc, __half2float(bv[k]));
                 }
                 // the activation-sum term first (few live registers), then the tensor-core sums
-                bool got = ptx::mbar_wait(&xs_full[j], (gq / ND) & 1u, abort_flag);
-                if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
-                const float4* xsj = reinterpret_cast<const float4*>(xs + j * NT);
+                const float4* xsq = reinterpret_cast<const float4*>(xsp + q * NT);
 #pragma unroll
                 for (int t4 = 0; t4 < NT / 4; ++t4) {
-                    const float4 v = xsj[t4];
+                    const float4 v = xsq[t4];
                     yacc[4 * t4 + 0] = fmaf(cc, v.x, yacc[4 * t4 + 0]);
                     yacc[4 * t4 + 1] = fmaf(cc, v.y, yacc[4 * t4 + 1]);
                     yacc[4 * t4 + 2] = fmaf(cc, v.z, yacc[4 * t4 + 2]);
                     yacc[4 * t4 + 3] = fmaf(cc, v.w, yacc[4 * t4 + 3]);
                 }
-                got = ptx::mbar_wait(&d_full[j], (gq / ND) & 1u, abort_flag);
+                got = ptx::mbar_wait(&done[sl], (gq / NS) & 1u, abort_flag);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
                 ptx::tc_fence_after_sync();
                 uint32_t dv[NT];
                 if constexpr (NT == 32) {
-                    ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + L::kAccCol + static_cast<uint32_t>(j * NT),
+                    ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + L::kAccCol + static_cast<uint32_t>(sl * NT),
                                             *reinterpret_cast<uint32_t(*)[32]>(dv));
                 } else {
-                    ptx::tmem_ld_32x32b_x16(tmem_base + lane_addr + L::kAccCol + static_cast<uint32_t>(j * NT),
+                    ptx::tmem_ld_32x32b_x16(tmem_base + lane_addr + L::kAccCol + static_cast<uint32_t>(sl * NT),
                                             *reinterpret_cast<uint32_t(*)[16]>(dv));
                 }
                 ptx::tmem_wait_ld();
@@ -436,12 +446,15 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
                 for (int t = 0; t < NT; ++t) yacc[t] = fmaf(sc, __uint_as_float(dv[t]), yacc[t]);
                 ptx::tc_fence_before_sync();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&d_empty[j]);
+                if (lane == 0) ptx::mbar_arrive(&ready[sl]);
             }
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&p_empty[pr]);
             gi += static_cast<uint32_t>(ng);
             // end of this tile's segment: write this copy's partial and start over
             const bool seg_end = (i + 1 == nchunks) || ((u0 + i + 1) % p.cpt == 0);
-            if (ok && seg_end) {
+            if (seg_end) {
                 float* dst = p.partial +
                              (((static_cast<int64_t>(blockIdx.x) * p.segmax + (w - w_first)) * 2 + par) * p.M) * BW;
 #pragma unroll
@@ -466,6 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
 template <bool kBf16Out>
 __global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restrict__ partial, void* __restrict__ y,
                                                             int M, int N, int cpt, int64_t units, int P, int segmax) {
+    ptx::grid_dependency_wait();
     const int64_t total = static_cast<int64_t>(M) * N;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
