@@ -147,8 +147,8 @@ struct Plan {
     size_t workspace = 0;
     // fused path workspace carve-up
     size_t off_xh = 0, off_rs = 0, off_sb = 0;
-    // skinny path workspace carve-up: partials, reordered activations, activation sums
-    size_t off_xp = 0, off_xs = 0;
+    // skinny path workspace carve-up: partials, scaled f16 activations, activation sums, row exponents
+    size_t off_xp = 0, off_xs = 0, off_re = 0;
 };
 
 ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int sm_count, Plan* plan) {
@@ -173,7 +173,8 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         plan->split_k = 1;
         plan->off_xp = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * 2 * M * skinny::BW * sizeof(float), 256);
         plan->off_xs = plan->off_xp + round_up(static_cast<size_t>(M) * K * 2, 256);
-        plan->workspace = plan->off_xs + round_up(static_cast<size_t>(G) * plan->nt * sizeof(float), 256);
+        plan->off_re = plan->off_xs + round_up(static_cast<size_t>(G) * plan->nt * sizeof(float), 256);
+        plan->workspace = plan->off_re + round_up(static_cast<size_t>(plan->nt) * sizeof(int), 256);
         return QL_OK;
     }
     if (path == QL_PATH_TC_FUSED) {
@@ -295,12 +296,13 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     void* xp = wsb + pl.off_xp;
     float* xs = reinterpret_cast<float*>(wsb + pl.off_xs);
+    int* rowexp = reinterpret_cast<int*>(wsb + pl.off_re);
     CUtensorMap mc, mx, mxs;
     ql_status s;
     if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K / 8, N, K / 2,
                        skinny::kBoxGroups * skinny::BK / 8, skinny::BW, CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
-    if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xp, K, M, K * 2, skinny::BK, pl.nt,
+    if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xp, K, M, K * 2, skinny::BK, pl.nt,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
     if ((s = encode_2d(&mxs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, xs, pl.nt, G, pl.nt * 4, pl.nt, skinny::CG,
@@ -329,10 +331,9 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     p.cpt = static_cast<int>((G + skinny::CG - 1) / skinny::CG);
     p.units = pl.units;
     p.segmax = pl.segmax;
-    // reordered activations and per-group activation sums
-    const int64_t pre_threads = static_cast<int64_t>(pl.nt) * (K / 8);
-    skinny::skinny_prepass_kernel<<<static_cast<unsigned>((pre_threads + 255) / 256), 256, 0, st>>>(
-        static_cast<const uint4*>(x), static_cast<uint4*>(xp), xs, p.M, static_cast<int>(K), pl.nt);
+    // scaled and reordered f16 activations, per-group activation sums, row exponents: one CTA per row
+    skinny::skinny_prepass_kernel<<<static_cast<unsigned>(pl.nt), 256, 0, st>>>(
+        static_cast<const uint4*>(x), static_cast<uint4*>(xp), xs, rowexp, p.M, static_cast<int>(K), pl.nt);
     if ((s = launch_status()) != QL_OK) return s;
     prof_begin(st);
     if (pl.nt == 16)
@@ -346,11 +347,12 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     const int64_t total = M * N;
     const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4 * sm_count));
     const float* part = p.partial;
+    const int* rexp = rowexp;
     if (bf16_out)
-        s = launch_dependent(skinny::skinny_reduce_kernel<true>, blocks, 256, 0, st, part, y, p.M, p.N, p.cpt,
+        s = launch_dependent(skinny::skinny_reduce_kernel<true>, blocks, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
                              p.units, pl.ctas, pl.segmax);
     else
-        s = launch_dependent(skinny::skinny_reduce_kernel<false>, blocks, 256, 0, st, part, y, p.M, p.N, p.cpt,
+        s = launch_dependent(skinny::skinny_reduce_kernel<false>, blocks, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
                              p.units, pl.ctas, pl.segmax);
     if (s != QL_OK) return s;
     set_dispatch("path=tc_skinny nt=%d ctas=%d segmax=%d units=%lld launches=3", pl.nt, pl.ctas, pl.segmax,

@@ -64,6 +64,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Elects one lane of the fully active warp.  Callers elect once and keep the
+// result, so the thread that issues MMAs also issues the commits that track them.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xFFFFFFFF;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
 
 // Lets the next kernel on the stream (launched with programmatic stream

@@ -2,46 +2,56 @@
 // is to read the 4.5-bit weights once at full bandwidth and spend as few
 // instructions per weight as possible.
 //
-// Per 64-group g of a 128-row weight tile, with q the exact codes:
-//   D_g[n][t] = sum_{k in g} (128 + q(n,k)) * x[t][k]          (tcgen05.mma, kind::f16, bf16 in, fp32 acc)
-//   y[t][n]  += s(n,g) * D_g[n][t] + (b(n,g) - 128 s(n,g)) * xsum_g[t]
-// which equals sum_k (s q + b) x (aimarketly "Ideogram-4-IQ4_M", "What IQ4 means
-// here": w = scale * q + bias).  128 + q is exact in bf16 (unit 1 at 128), so the
-// tensor core sees the exact codes and the exact bf16 activations; the scale and
-// bias are applied in fp32 per (row, group, token).  The A operand is built from
-// the code nibbles with one shift and one AND-OR per pair of weights and is
-// written to tensor memory (tcgen05.st); shared memory carries only the streamed
-// code chunks, the activation tiles and the per-chunk scale/bias/xsum tiles.
+// The weight of row n, column k is w = s(n,g) q(n,k) + b(n,g) for the 64-group g
+// holding k (aimarketly "Ideogram-4-IQ4_M", "What IQ4 means here": w = scale * q +
+// bias), so per group
+//   y[t][n] += s(n,g) * sum_{k in g} q(n,k) x[t][k] + b(n,g) * sum_{k in g} x[t][k].
+// The tensor core (tcgen05.mma, kind::f16, f16 operands, fp32 accumulation) forms
+// the first sum from the exact codes; the drain applies s and b in fp32.
 //
-// A word of codes holds k = 0..7 in nibbles 0..7; the builder pairs nibbles j and
-// j + 4 (16 bits apart, so one AND-OR per pair), which puts k in the order
-// 0,4,1,5,2,6,3,7 along each 8-block of the MMA's reduction dimension.  A small
-// prepass kernel writes the activations in that same order, and the per-group
-// activation sums xsum_g[t], once for all CTAs.  It runs under programmatic
-// dependent launch: the main kernel starts streaming codes at once and waits for
-// the prepass only before its first activation load.
+// Codes as f16 operands.  A word of codes holds k = 0..7 of an 8-block in nibbles
+// 0..7.  Read as a pair of f16 values, (v & 0x000F000F) is (q0, q4) * 2^-24 and
+// (v & 0x00F000F0) is (q1, q5) * 16 * 2^-24 exactly (f16 subnormals), and the same
+// masks on v >> 8 give (q2, q6) * 2^-24 and (q3, q7) * 16 * 2^-24: one shift and
+// four ANDs per 8 weights, with k in the order 0,4,1,5,2,6,3,7 along each 8-block
+// of the reduction dimension.  A prepass kernel writes the activations in that
+// order as f16, x'[t][k] = x[t][k] * 2^e_t (a per-row power of two that puts the
+// row maximum in [2^14, 2^15)) and a further 2^-4 at odd k to cancel the factor
+// 16 on those codes, so that
+//   D_g[n][t] = sum_{k in g} A[n][k] x'[t][k] = 2^(e_t - 24) sum_{k in g} q(n,k) x[t][k].
+// The prepass also writes xs_g[t] = 2^(e_t - 24) sum_{k in g} x[t][k], so the drain
+// accumulates s * D + b * xs, all scaled by 2^(e_t - 24), and the reduce kernel
+// scales back by 2^(24 - e_t) (ldexpf, exact).  Activation entries below 2^-25 of
+// the row maximum lose bits as f16 subnormals; nothing else is rounded before the
+// fp32 accumulation.  The prepass runs under programmatic dependent launch: the
+// main kernel starts streaming codes at once and waits for the prepass only
+// before its first activation load.
 //
-// Stream-K schedule: the work is cut into chunks of CG consecutive groups of one
-// 128-row weight tile (a tile has ceil(G/CG) chunks; a tile's last chunk may be
-// partial).  The chunks, tile-major, are split into one equal contiguous run per
-// CTA; a run covers at most a few tiles, and each covered tile segment leaves
-// fp32 partials [2][tokens][128] in the workspace (one per group parity).  A
-// reduce kernel sums, per output, the partials of the CTAs that covered its tile
-// in CTA order (deterministic) and rounds to bf16.  The code boxes of a chunk
-// bring CG * 32 contiguous bytes of each row, so DRAM sees long row segments.
+// Stream-K schedule: the work is cut into chunks of CG = 8 consecutive groups of
+// one 128-row weight tile (a tile has ceil(G/CG) chunks; a tile's last chunk may
+// be partial).  The chunks, tile-major, are split into one equal contiguous run
+// per CTA; a run covers at most a few tiles, and each covered tile segment leaves
+// fp32 partials [2][tokens][128] in the workspace (one per drain copy).  The reduce
+// kernel sums, per output, the partials of the CTAs that covered its tile in CTA
+// order (deterministic).  The code boxes of a chunk bring CG * 32 contiguous bytes
+// of each row, so DRAM sees long row segments.
 //
-// The builders and the drains run as two copies, on the even and the odd groups
-// of the run, and so do the MMA issuers.  Each TMEM slot s (an A stage and an
-// accumulator) serves one parity, with one barrier each way: ready[s] (A built
-// by the 4 builder warps, accumulator read by the 4 drain warps) and done[s]
-// (the slot's MMAs completed).
-// Warp roles (608 threads, one CTA per SM; at most 5 warps per SM sub-partition leave 96 registers a thread):
-//   warp 0        TMA producer: code chunks (128 rows x CG*32 B, 128B swizzle), scale/bias/xsum tiles,
-//                 activation tiles of a chunk (NT x 64 per group, 128B swizzle)
-//   warps 1, 2    MMA issuers for even / odd groups (warp 1 also allocates TMEM)
-//   warps 3-10    A builders, even groups (3-6) / odd groups (7-10): one weight row per thread
-//   warps 11-18   drains, even groups (11-14) / odd groups (15-18): one weight row per thread, fp32
-//                 accumulation of s*D + c*xsum over the run
+// Each barrier wait, arrive or commit costs a role on the order of a hundred
+// cycles, so the roles step over pairs of consecutive groups of a chunk (pair j =
+// groups 2j, 2j+1): one wait and one signal per pair.  Pairs are numbered pc along
+// the run.  The A builders, the slowest role, run as four copies (pair pc goes to
+// copy pc % 4, one pair of every chunk each); the drains and the MMA issuers run
+// as two (pc % 2).  TMEM slot pc % NS holds the pair's two A stages and two
+// accumulators, with one barrier each way: ready[s] (A built by the 4 builder warps
+// of the slot's copy, accumulators read back by the 4 drain warps of its copy) and
+// done[s] (the slot's MMAs completed).
+// Warp roles (864 threads, one CTA per SM; 7 warps per SM sub-partition leave 72 registers a thread):
+//   warp 0        TMA producer: code chunks (128 rows x CG*32 B, 128B swizzle), scale/bias/xs tiles,
+//                 activation tiles of a chunk (NT x 64 f16 per group, 128B swizzle)
+//   warps 1, 2    MMA issuers for even / odd pairs (warp 1 also allocates TMEM)
+//   warps 3-18    A builders, copies 0-3 of 4 warps: one weight row per thread
+//   warps 19-26   drains, even pairs (19-22) / odd pairs (23-26): one weight row per thread, fp32
+//                 accumulation of s*D + b*xs over the run
 #pragma once
 
 #include "ql_ptx.cuh"
@@ -52,43 +62,46 @@ namespace skinny {
 constexpr int BW = 128;
 constexpr int BK = 64;
 constexpr int UK = 16;
-constexpr int kWarpTma = 0, kWarpMma0 = 1, kWarpBuild0 = 3, kWarpDrain0 = 11;
-constexpr int kThreads = 19 * 32;
-constexpr int CG = 8;                    // groups per chunk
+constexpr int kBuildCopies = 4, kDrainCopies = 2, kMmaCopies = 2;
+constexpr int kWarpTma = 0, kWarpMma0 = 1, kWarpBuild0 = 3, kWarpDrain0 = kWarpBuild0 + 4 * kBuildCopies;
+constexpr int kThreads = (kWarpDrain0 + 4 * kDrainCopies) * 32;
+constexpr int CG = 8;                    // groups per chunk: four pairs, one per builder copy
 constexpr int kBoxGroups = 4;            // groups per code box: 128 bytes of each row (the 128B-swizzle span)
-constexpr int NS = 8;                    // TMEM slots (A stage + accumulator), even
-constexpr int PR = 4;                    // scale/bias/xsum chunk stages
+constexpr int NS = 4;                    // TMEM slots (two A stages + two accumulators each)
+constexpr int PR = 4;                    // scale/bias/xs chunk stages
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBoxBytes = BW * BK / 2 * kBoxGroups;     // 16 KB: one code box
 constexpr uint32_t kCBytes = kBoxBytes * (CG / kBoxGroups);  // codes per chunk
 constexpr uint32_t kParHalf = BW * CG * 2;                   // one chunk's scales (or biases): [128][CG] f16
-static_assert(CG % kBoxGroups == 0 && CG % 8 == 0, "whole code boxes and 16-byte scale rows per chunk");
+static_assert(CG == 2 * kBuildCopies && kBoxGroups == 4, "one pair of every chunk per builder copy");
+static_assert(NS % kBuildCopies == 0 && NS % kDrainCopies == 0 && NS % kMmaCopies == 0,
+              "every TMEM slot serves one copy of each role");
 
 template <int NT>
 struct Layout {
     static constexpr int NC = NT == 16 ? 4 : 3;                          // code chunk stages
     static constexpr int NXC = NT == 16 ? 4 : 3;                         // activation chunk stages
-    static constexpr uint32_t kXTile = NT * BK * 2;                      // one group's activation tile
+    static constexpr uint32_t kXTile = NT * BK * 2;                      // one group's activation tile (f16)
     static constexpr uint32_t kXBytes = CG * kXTile;                     // one chunk's activation tiles
-    static constexpr uint32_t kXsBytes = CG * NT * 4;                    // one chunk's xsum rows [CG][NT] fp32
-    static constexpr uint32_t kParBytes = 2 * kParHalf + kXsBytes;       // [scales | biases | xsum]
+    static constexpr uint32_t kXsBytes = CG * NT * 4;                    // one chunk's xs rows [CG][NT] fp32
+    static constexpr uint32_t kParBytes = 2 * kParHalf + kXsBytes;       // [scales | biases | xs]
     static constexpr uint32_t kOffC = 0;                                  // [NC][codes], 1 KB aligned
     static constexpr uint32_t kOffX = kOffC + NC * kCBytes;              // [NXC][CG][x tile], 1 KB aligned
     static constexpr uint32_t kOffPar = kOffX + NXC * kXBytes;           // [PR][par]
     static constexpr uint32_t kOffBar = kOffPar + PR * kParBytes;
-    static constexpr uint32_t kNumBars = 2 * NC + 2 * PR + 2 * NXC + 2 * NS + 2;
+    static constexpr uint32_t kNumBars = 2 * NC + 2 * PR + 2 * NXC + 2 * NS + kMmaCopies;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
-    static constexpr uint32_t kAccCol = 0;                                // accumulator of slot s at [s*NT, (s+1)*NT)
-    static constexpr uint32_t kACol = NS * NT;                            // A stage of slot s at [kACol + 32s, +32)
+    static constexpr uint32_t kAccCol = 0;                                // accumulator h of slot s at (2s+h)*NT
+    static constexpr uint32_t kACol = 2 * NS * NT;                        // A stage h of slot s at kACol + 32(2s+h)
     static_assert(kCBytes % 1024 == 0 && kXTile % 1024 == 0, "swizzled stage pieces need 1 KB alignment");
     static_assert(kParBytes % 128 == 0, "TMA destinations 128-byte aligned");
-    static_assert(kACol + NS * 32 <= kTmemCols, "tensor memory budget");
+    static_assert(kACol + 2 * NS * 32 <= kTmemCols, "tensor memory budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 struct Params {
-    float* partial;          // [P][segmax][2][M][128] fp32
+    float* partial;          // [P][segmax][2][M][128] fp32, scaled by 2^(e_t - 24)
     const __half* scales;    // [N][G]
     const __half* biases;    // [N][G]
     int param_tma;           // 1: scales/biases arrive as TMA tiles (needs G % CG == 0); 0: direct loads
@@ -103,42 +116,85 @@ __host__ __device__ __forceinline__ int64_t run_first(int64_t units, int P, int 
     return units * c / P;
 }
 
-// Codes word (code j in nibble j) -> 4 words of bf16 pairs (128 + code j, 128 + code j+4), j = 0..3.
-__device__ __forceinline__ void codes_to_bf16(uint32_t v, uint32_t* o) {
-    o[0] = (v & 0x000F000Fu) | 0x43004300u;
-    o[1] = ((v >> 4) & 0x000F000Fu) | 0x43004300u;
-    o[2] = ((v >> 8) & 0x000F000Fu) | 0x43004300u;
-    o[3] = ((v >> 12) & 0x000F000Fu) | 0x43004300u;
+// Codes word (code j in nibble j) -> 4 words of f16 pairs (subnormals, exact):
+// (q0, q4) 2^-24, (q1, q5) 16 2^-24, (q2, q6) 2^-24, (q3, q7) 16 2^-24.
+__device__ __forceinline__ void codes_to_f16(uint32_t v, uint32_t* o) {
+    const uint32_t u = v >> 8;
+    o[0] = v & 0x000F000Fu;
+    o[1] = v & 0x00F000F0u;
+    o[2] = u & 0x000F000Fu;
+    o[3] = u & 0x00F000F0u;
 }
 
-// x [M][K] bf16 -> xp [M][K] with each 8-block of k in the order 0,4,1,5,2,6,3,7, and
-// xsum[g][t] = sum over group g of x[t][k] in fp32 for t < NT (zero for t >= M).
-// One thread per (row, 8-block); the 8 threads of a group are 8 aligned lanes.
+// Packed fp32 FMA on two lanes: d = a * b + c, each lane rounded as fmaf.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
+          "l"(*reinterpret_cast<const uint64_t*>(&c)));
+    return *reinterpret_cast<float2*>(&d);
+}
+
+// Per activation row t (one CTA each, t < NT): e_t puts max_k |x[t][k]| in [2^14, 2^15) (0 for a
+// zero or non-finite row); xp[t][k] = f16(x * 2^e_t), times 2^-4 at odd k, in the order
+// 0,4,1,5,2,6,3,7 of each 8-block; xs[g][t] = 2^(e_t - 24) * sum over group g of x[t][k] in fp32
+// (zero for t >= M); rowexp[t] = 24 - e_t.
 __global__ void __launch_bounds__(256) skinny_prepass_kernel(const uint4* __restrict__ x, uint4* __restrict__ xp,
-                                                             float* __restrict__ xsum, int M, int K, int NT) {
+                                                             float* __restrict__ xs, int* __restrict__ rowexp,
+                                                             int M, int K, int NT) {
     ptx::launch_dependents();
-    const int kb = K / 8;
-    const int64_t total = static_cast<int64_t>(NT) * kb;
-    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const bool in = idx < total;
-    const int t = in ? static_cast<int>(idx / kb) : 0;
-    const int c = in ? static_cast<int>(idx % kb) : 0;
-    float sum = 0.0f;
-    if (in && t < M) {
-        const uint4 v = x[static_cast<int64_t>(t) * kb + c];     // (k0,k1) (k2,k3) (k4,k5) (k6,k7), low half first
-        uint4 o;
-        asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(o.x) : "r"(v.x), "r"(v.z));   // (k0, k4)
-        asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(o.y) : "r"(v.x), "r"(v.z));   // (k1, k5)
-        asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(o.z) : "r"(v.y), "r"(v.w));   // (k2, k6)
-        asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(o.w) : "r"(v.y), "r"(v.w));   // (k3, k7)
-        xp[static_cast<int64_t>(t) * kb + c] = o;
-        sum = ((bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y))) +
-              ((bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w)));
+    __shared__ float red[8];
+    const int t = blockIdx.x;
+    const int kb = K / 8;                                      // 8-blocks per row, a multiple of 8
+    const bool row = t < M;
+    const uint4* xr = x + static_cast<int64_t>(t) * kb;
+    float m = 0.0f;
+    if (row)
+        for (int c = threadIdx.x; c < kb; c += blockDim.x) {
+            const uint4 v = xr[c];
+            m = fmaxf(m, fmaxf(fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))),
+                               fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w))))));
+        }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = red[0];
+    for (int i = 1; i < static_cast<int>(blockDim.x >> 5); ++i) m = fmaxf(m, red[i]);
+    int ex = 0;
+    if (m > 0.0f && m <= 3.4028235e38f) {
+        int E;
+        frexpf(m, &E);                                         // m = f 2^E, f in [0.5, 1)
+        ex = 15 - E;
     }
-    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
-    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
-    if (in && (c & 7) == 0) xsum[static_cast<int64_t>(c >> 3) * NT + t] = sum;
+    if (threadIdx.x == 0) rowexp[t] = 24 - ex;
+    // the 8 blocks of a group are 8 consecutive threads (blockDim.x is a multiple of 8)
+    const int iters = (kb + static_cast<int>(blockDim.x) - 1) / static_cast<int>(blockDim.x);
+    for (int it = 0; it < iters; ++it) {
+        const int c = it * static_cast<int>(blockDim.x) + static_cast<int>(threadIdx.x);
+        const bool in = c < kb;
+        float sum = 0.0f;
+        if (in && row) {
+            const uint4 v = xr[c];
+            const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                                bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+            sum = ((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]));
+            // slot pairs (k0, k4) (k1, k5) (k2, k6) (k3, k7); odd k carry the extra 2^-4
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int sh = ex - ((j & 1) ? 4 : 0);
+                const __half2 h = __halves2half2(__float2half_rn(ldexpf(f[j], sh)), __float2half_rn(ldexpf(f[j + 4], sh)));
+                o[j] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            xp[static_cast<int64_t>(t) * kb + c] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
+        if (in && (c & 7) == 0) xs[static_cast<int64_t>(c >> 3) * NT + t] = row ? ldexpf(sum, ex - 24) : 0.0f;
+    }
 }
 
 template <int NT>
@@ -146,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
                                                             const __grid_constant__ CUtensorMap map_x,
                                                             const __grid_constant__ CUtensorMap map_scales,
                                                             const __grid_constant__ CUtensorMap map_biases,
-                                                            const __grid_constant__ CUtensorMap map_xsum,
+                                                            const __grid_constant__ CUtensorMap map_xs,
                                                             const Params p) {
     using L = Layout<NT>;
     constexpr int NC = L::NC;
@@ -162,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     uint64_t* x_empty = x_full + NXC;
     uint64_t* ready = x_empty + NXC;
     uint64_t* done = ready + NS;
-    uint64_t* drain = done + NS;                // two: one per MMA issuer
+    uint64_t* drain = done + NS;                // one per MMA issuer
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
 
@@ -174,19 +230,18 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     const uint32_t nchunks = static_cast<uint32_t>(u1 - u0);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NC; ++i) { ptx::mbar_init(&c_full[i], 1); ptx::mbar_init(&c_empty[i], 8); }
-        for (int i = 0; i < PR; ++i) { ptx::mbar_init(&p_full[i], 1); ptx::mbar_init(&p_empty[i], 8); }
-        for (int i = 0; i < NXC; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], 2); }
+        for (int i = 0; i < NC; ++i) { ptx::mbar_init(&c_full[i], 1); ptx::mbar_init(&c_empty[i], 4 * kBuildCopies); }
+        for (int i = 0; i < PR; ++i) { ptx::mbar_init(&p_full[i], 1); ptx::mbar_init(&p_empty[i], 4 * kDrainCopies); }
+        for (int i = 0; i < NXC; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], kMmaCopies); }
         for (int i = 0; i < NS; ++i) { ptx::mbar_init(&ready[i], 8); ptx::mbar_init(&done[i], 1); }
-        ptx::mbar_init(drain, 1);
-        ptx::mbar_init(drain + 1, 1);
+        for (int i = 0; i < kMmaCopies; ++i) ptx::mbar_init(&drain[i], 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
     if (warp == kWarpTma && lane == 0) {
         ptx::prefetch_tensormap(&map_codes);
         ptx::prefetch_tensormap(&map_x);
-        ptx::prefetch_tensormap(&map_xsum);
+        ptx::prefetch_tensormap(&map_xs);
         if (p.param_tma) {
             ptx::prefetch_tensormap(&map_scales);
             ptx::prefetch_tensormap(&map_biases);
@@ -202,21 +257,38 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     const uint32_t tmem_base = *tmem_slot;
     ptx::launch_dependents();
 
-    // chunk u -> tile w = u / cpt, groups g = (u % cpt) * CG + q, q < ng.  Groups are numbered
-    // gi along the run; group gi belongs to the copies of parity gi & 1 and uses TMEM slot gi % NS.
-    auto chunk_groups = [&](int64_t u, int& w, int& g0, int& ng) {
-        w = static_cast<int>(u / p.cpt);
-        g0 = static_cast<int>(u % p.cpt) * CG;
+    // chunk u is chunk cq = u % cpt of tile w = u / cpt, groups g = cq * CG + q, q < ng; pair j of the
+    // chunk is groups 2j and 2j + 1 (the second may be missing in a tile's last chunk).  Each role
+    // walks its chunks with a (w, cq) position advanced by one per chunk, without dividing.
+    struct ChunkPos {
+        int w, cq;
+    };
+    const ChunkPos start{static_cast<int>(u0 / p.cpt), static_cast<int>(u0 % p.cpt)};
+    auto advance = [&](ChunkPos& c) {
+        if (++c.cq == p.cpt) {
+            c.cq = 0;
+            ++c.w;
+        }
+    };
+    auto chunk_groups = [&](const ChunkPos& c, int& w, int& g0, int& ng) {
+        w = c.w;
+        g0 = c.cq * CG;
         ng = min(CG, p.G - g0);
+    };
+    // first pair j of a chunk whose run-wide number pb + j is copy (mod ncopies)
+    auto first_pair = [](uint32_t pb, int copy, int ncopies) {
+        const uint32_t nc = static_cast<uint32_t>(ncopies);
+        return static_cast<int>((static_cast<uint32_t>(copy) + nc - pb % nc) % nc);
     };
 
     if (warp == kWarpTma) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
             uint32_t ci = 0, pi = 0, xi = 0;     // chunks whose codes / parameters / activations were issued
+            ChunkPos cpc = start, cpi = start;    // positions of chunk ci and of chunk i
             auto issue_codes = [&](uint32_t i) -> bool {
                 int w, g0, ng;
-                chunk_groups(u0 + i, w, g0, ng);
+                chunk_groups(cpc, w, g0, ng);
                 const int s = static_cast<int>(i % NC);
                 if (!ptx::mbar_wait(&c_empty[s], ((i / NC) & 1u) ^ 1u, abort_flag)) return false;
                 uint8_t* st = smem + L::kOffC + s * kCBytes;
@@ -224,6 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
 #pragma unroll
                 for (int bx = 0; bx < CG / kBoxGroups; ++bx)   // consecutive boxes: long contiguous row segments
                     ptx::tma_load_2d(st + bx * kBoxBytes, &map_codes, &c_full[s], (g0 + bx * kBoxGroups) * (BK / 8), w * BW);
+                advance(cpc);
                 return true;
             };
             // the codes do not depend on the prepass: start streaming them at once
@@ -233,9 +306,9 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
                 if (ok) ++ci;
             }
             ptx::grid_dependency_wait();
-            for (uint32_t i = 0; i < nchunks && ok; ++i) {
+            for (uint32_t i = 0; i < nchunks && ok; ++i, advance(cpi)) {
                 int w, g0, ng;
-                chunk_groups(u0 + i, w, g0, ng);
+                chunk_groups(cpi, w, g0, ng);
                 // scales, biases and activation sums of the chunk
                 const int pr = static_cast<int>(i % PR);
                 if (!ptx::mbar_wait(&p_empty[pr], ((i / PR) & 1u) ^ 1u, abort_flag)) break;
@@ -245,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
                     ptx::tma_load_2d(pt, &map_scales, &p_full[pr], g0, w * BW);
                     ptx::tma_load_2d(pt + kParHalf, &map_biases, &p_full[pr], g0, w * BW);
                 }
-                ptx::tma_load_2d(pt + 2 * kParHalf, &map_xsum, &p_full[pr], 0, g0);   // rows past G read zeros
+                ptx::tma_load_2d(pt + 2 * kParHalf, &map_xs, &p_full[pr], 0, g0);   // rows past G read zeros
                 ++pi;
                 // activation tiles of the chunk
                 const int xc = static_cast<int>(i % NXC);
@@ -268,182 +341,216 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
             for (uint32_t j = (xi > static_cast<uint32_t>(NXC) ? xi - NXC : 0u); j < xi; ++j)
                 ptx::mbar_wait(&x_full[j % NXC], (j / NXC) & 1u, nullptr);
         }
-    } else if (warp == kWarpMma0 || warp == kWarpMma0 + 1) {
-        // ---------------------------------------------------------------- MMA issuers (even / odd groups)
-        // The whole warp runs the loop, so the addresses stay warp-uniform; lane 0 issues.
-        const uint32_t par = static_cast<uint32_t>(warp - kWarpMma0);
-        constexpr uint32_t idesc = ptx::idesc_f16(BW, NT, true);
-        const uint32_t x_base = ptx::smem_addr(smem + L::kOffX);
-        uint32_t gi = 0;
+    } else if (warp < kWarpMma0 + kMmaCopies) {
+        // ---------------------------------------------------------------- MMA issuers (even / odd pairs)
+        // The whole warp runs the loop; one elected lane issues the MMAs and the commits.
+        const int copy = warp - kWarpMma0;
+        const bool leader = ptx::elect_one();
+        constexpr uint32_t idesc = ptx::idesc_f16(BW, NT, false);
+        const uint64_t xdesc0 = ptx::sdesc_sw128(ptx::smem_addr(smem + L::kOffX));
+        uint32_t pb = 0;     // pairs of the run before this chunk
         bool ok = true;
-        for (uint32_t i = 0; i < nchunks && ok; ++i) {
+        ChunkPos cp = start;
+        for (uint32_t i = 0; i < nchunks && ok; ++i, advance(cp)) {
             int w, g0, ng;
-            chunk_groups(u0 + i, w, g0, ng);
+            chunk_groups(cp, w, g0, ng);
+            const int np = (ng + 1) >> 1;
             const int xc = static_cast<int>(i % NXC);
             bool got = ptx::mbar_wait(&x_full[xc], (i / NXC) & 1u, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
-            for (int q = static_cast<int>((par - gi) & 1u); q < ng; q += 2) {
-                const uint32_t gq = gi + static_cast<uint32_t>(q);
-                const int sl = static_cast<int>(gq % NS);
-                got = ptx::mbar_wait(&ready[sl], (gq / NS) & 1u, abort_flag);
+            // descriptor of the chunk's first activation tile (the address field counts 16-byte units)
+            const uint64_t xdesc = xdesc0 + ((static_cast<uint32_t>(xc) * L::kXBytes) >> 4);
+            for (int j = first_pair(pb, copy, kMmaCopies); j < np; j += kMmaCopies) {
+                const uint32_t pc = pb + static_cast<uint32_t>(j);
+                const int sl = static_cast<int>(pc % NS);
+                got = ptx::mbar_wait(&ready[sl], (pc / NS) & 1u, abort_flag);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
                 ptx::tc_fence_after_sync();
-                const uint32_t xa = x_base + static_cast<uint32_t>(xc) * L::kXBytes + static_cast<uint32_t>(q) * L::kXTile;
-                const uint32_t d = tmem_base + L::kAccCol + static_cast<uint32_t>(sl * NT);
-                const uint32_t a_tm = tmem_base + L::kACol + 32u * static_cast<uint32_t>(sl);
-                if (lane == 0) {
+                if (leader) {
 #pragma unroll
-                    for (int u = 0; u < BK / UK; ++u)
-                        ptx::mma_f16_ts(d, a_tm + u * (UK / 2), ptx::sdesc_sw128(xa + u * UK * 2), idesc, u != 0);
+                    for (int h = 0; h < 2; ++h) {
+                        if (2 * j + h < ng) {
+                            const uint32_t d = tmem_base + L::kAccCol + static_cast<uint32_t>((2 * sl + h) * NT);
+                            const uint32_t a_tm = tmem_base + L::kACol + 32u * static_cast<uint32_t>(2 * sl + h);
+                            const uint64_t bd = xdesc + ((static_cast<uint32_t>(2 * j + h) * L::kXTile) >> 4);
+#pragma unroll
+                            for (int u = 0; u < BK / UK; ++u)
+                                ptx::mma_f16_ts(d, a_tm + u * (UK / 2), bd + ((u * UK * 2) >> 4), idesc, u != 0);
+                        }
+                    }
                     ptx::mma_commit(&done[sl]);
                 }
                 __syncwarp();
             }
-            if (ok && lane == 0) ptx::mma_commit(&x_empty[xc]);
+            if (ok && leader) ptx::mma_commit(&x_empty[xc]);
             __syncwarp();
-            gi += static_cast<uint32_t>(ng);
+            pb += static_cast<uint32_t>(np);
         }
-        if (lane == 0) ptx::mma_commit(drain + par);
+        if (leader) ptx::mma_commit(&drain[copy]);
         __syncwarp();
-        ptx::mbar_wait(drain + par, 0, nullptr);
+        ptx::mbar_wait(&drain[copy], 0, nullptr);
     } else if (warp >= kWarpBuild0 && warp < kWarpDrain0) {
-        // ---------------------------------------------------------------- A builders (even / odd groups)
-        const uint32_t par = static_cast<uint32_t>((warp - kWarpBuild0) >> 2);
+        // ---------------------------------------------------------------- A builders (four copies)
+        const int copy = (warp - kWarpBuild0) >> 2;
         const int quarter = warp & 3;                      // TMEM lanes 32*quarter.. belong to this warp
         const int r = quarter * 32 + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        uint32_t gi = 0;
+        uint32_t pb = 0;
         bool ok = true;
-        for (uint32_t i = 0; i < nchunks && ok; ++i) {
+        ChunkPos cp = start;
+        for (uint32_t i = 0; i < nchunks && ok; ++i, advance(cp)) {
             int w, g0, ng;
-            chunk_groups(u0 + i, w, g0, ng);
+            chunk_groups(cp, w, g0, ng);
+            const int np = (ng + 1) >> 1;
+            const int j = first_pair(pb, copy, kBuildCopies);     // this copy's pair of the chunk, if j < np
+            const bool mine = j < np;
             const int s = static_cast<int>(i % NC);
             bool got = ptx::mbar_wait(&c_full[s], (i / NC) & 1u, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
-            // this copy's groups of the chunk are q = q0, q0 + 2, ...  Row r's 32 code bytes of group q
-            // sit in box q / 4 at the 16-byte pieces 2 (q % 4) and 2 (q % 4) + 1, stored with the
-            // 128-byte swizzle (piece c at c ^ (r % 8)), so every 8 lanes of a load touch 8 bank groups.
-            const int q0 = static_cast<int>((par - gi) & 1u);
-            const uint8_t* crow = smem + L::kOffC + s * kCBytes + r * 128;
-            uint4 cw[CG];
+            // row r's 32 code bytes of group q sit in code box q / 4 at the 16-byte pieces 2 (q % 4) and
+            // 2 (q % 4) + 1 of its box row, stored with the 128-byte swizzle (piece c at c ^ (r % 8)), so
+            // every 8 lanes of a load touch 8 bank groups
+            uint4 cw[4];
+            if (mine) {
+                const uint8_t* crow = smem + L::kOffC + s * kCBytes + (j >> 1) * kBoxBytes + r * 128;
 #pragma unroll
-            for (int k = 0; k < CG / 2; ++k) {
-                const int q = q0 + 2 * k;
-                if (q < ng) {
-                    const uint8_t* bxp = crow + (q / kBoxGroups) * kBoxBytes;
-                    const int c = 2 * (q % kBoxGroups);
-                    cw[2 * k] = *reinterpret_cast<const uint4*>(bxp + ((c ^ (r & 7)) << 4));
-                    cw[2 * k + 1] = *reinterpret_cast<const uint4*>(bxp + (((c + 1) ^ (r & 7)) << 4));
+                for (int h = 0; h < 2; ++h) {
+                    const int c = 2 * ((2 * j + h) & 3);
+                    if (2 * j + h < ng) {
+                        cw[2 * h] = *reinterpret_cast<const uint4*>(crow + ((c ^ (r & 7)) << 4));
+                        cw[2 * h + 1] = *reinterpret_cast<const uint4*>(crow + (((c + 1) ^ (r & 7)) << 4));
+                    }
                 }
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&c_empty[s]);
-#pragma unroll
-            for (int k = 0; k < CG / 2; ++k) {
-                const int q = q0 + 2 * k;
-                if (q >= ng) break;
-                const uint32_t gq = gi + static_cast<uint32_t>(q);
-                const int sl = static_cast<int>(gq % NS);
-                const uint4 c0 = cw[2 * k], c1 = cw[2 * k + 1];
-                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint32_t av[32];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) codes_to_bf16(words[c], &av[4 * c]);
-                // the slot's previous MMAs must have finished reading its A stage
-                got = ptx::mbar_wait(&done[sl], ((gq / NS) & 1u) ^ 1u, abort_flag);
+            if (mine) {
+                const uint32_t pc = pb + static_cast<uint32_t>(j);
+                const int sl = static_cast<int>(pc % NS);
+                // the slot's previous MMAs must have finished reading its A stages
+                got = ptx::mbar_wait(&done[sl], ((pc / NS) & 1u) ^ 1u, abort_flag);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
                 ptx::tc_fence_after_sync();
-                ptx::tmem_st_32x32b_x32(tmem_base + lane_addr + L::kACol + 32u * sl, av);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (2 * j + h < ng) {
+                        const uint4 c0 = cw[2 * h], c1 = cw[2 * h + 1];
+                        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                        uint32_t av[32];
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) codes_to_f16(words[c], &av[4 * c]);
+                        ptx::tmem_st_32x32b_x32(tmem_base + lane_addr + L::kACol + 32u * static_cast<uint32_t>(2 * sl + h), av);
+                    }
+                }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&ready[sl]);
             }
-            gi += static_cast<uint32_t>(ng);
+            pb += static_cast<uint32_t>(np);
         }
-    } else if (warp >= kWarpDrain0) {
-        // ---------------------------------------------------------------- drains (even / odd groups)
-        const uint32_t par = static_cast<uint32_t>((warp - kWarpDrain0) >> 2);
+    } else {
+        // ---------------------------------------------------------------- drains (even / odd pairs)
+        const int copy = (warp - kWarpDrain0) >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        // a slot's first use has no accumulator to read back: arrive for it in advance
+        // a slot's first use has no accumulators to read back: arrive for it in advance
         if (lane == 0)
-            for (int sl = static_cast<int>(par); sl < NS; sl += 2) ptx::mbar_arrive(&ready[sl]);
-        float yacc[NT];
+            for (int sl = copy; sl < NS; sl += kDrainCopies) ptx::mbar_arrive(&ready[sl]);
+        float2 yacc[NT / 2];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) yacc[t] = 0.0f;
-        const int w_first = static_cast<int>(u0 / p.cpt);
-        uint32_t gi = 0;
+        for (int t = 0; t < NT / 2; ++t) yacc[t] = make_float2(0.0f, 0.0f);
+        const int w_first = start.w;
+        uint32_t pb = 0;
         bool ok = true;
-        for (uint32_t i = 0; i < nchunks && ok; ++i) {
+        ChunkPos cp = start;
+        for (uint32_t i = 0; i < nchunks && ok; ++i, advance(cp)) {
             int w, g0, ng;
-            chunk_groups(u0 + i, w, g0, ng);
+            chunk_groups(cp, w, g0, ng);
+            const int np = (ng + 1) >> 1;
             const int n = w * BW + r;
-            const int q0 = static_cast<int>((par - gi) & 1u);
+            const int j0 = first_pair(pb, copy, kDrainCopies);   // this copy's pairs: j0, j0 + 2
             const int pr = static_cast<int>(i % PR);
             bool got = ptx::mbar_wait(&p_full[pr], (i / PR) & 1u, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
             const uint8_t* pt = smem + L::kOffPar + pr * L::kParBytes;
-            // this copy's scales and biases of row r (groups q0, q0 + 2, ...)
-            __half sv[CG / 2], bv[CG / 2];
+            // scales and biases of row r for this copy's pairs j0 and j0 + 2: word jj holds the f16 values
+            // of groups 2 (j0 + 2 jj) (low half) and 2 (j0 + 2 jj) + 1 (high half)
+            uint32_t sw[2], bw[2];
             if (p.param_tma) {
-                __align__(16) __half sa[CG], ba[CG];
-#pragma unroll
-                for (int c = 0; c < CG / 8; ++c) {
-                    *reinterpret_cast<uint4*>(sa + 8 * c) = reinterpret_cast<const uint4*>(pt + r * CG * 2)[c];
-                    *reinterpret_cast<uint4*>(ba + 8 * c) = reinterpret_cast<const uint4*>(pt + kParHalf + r * CG * 2)[c];
-                }
-#pragma unroll
-                for (int k = 0; k < CG / 2; ++k) {
-                    sv[k] = q0 ? sa[2 * k + 1] : sa[2 * k];
-                    bv[k] = q0 ? ba[2 * k + 1] : ba[2 * k];
-                }
+                const uint4 sq = *reinterpret_cast<const uint4*>(pt + r * CG * 2);
+                const uint4 bq = *reinterpret_cast<const uint4*>(pt + kParHalf + r * CG * 2);
+                sw[0] = j0 ? sq.y : sq.x;
+                sw[1] = j0 ? sq.w : sq.z;
+                bw[0] = j0 ? bq.y : bq.x;
+                bw[1] = j0 ? bq.w : bq.z;
             } else {
 #pragma unroll
-                for (int k = 0; k < CG / 2; ++k) {
-                    const int q = q0 + 2 * k;
-                    const bool in = n < p.N && q < ng;
-                    sv[k] = in ? __ldg(p.scales + static_cast<int64_t>(n) * p.G + g0 + q) : __float2half_rn(0.0f);
-                    bv[k] = in ? __ldg(p.biases + static_cast<int64_t>(n) * p.G + g0 + q) : __float2half_rn(0.0f);
+                for (int jj = 0; jj < 2; ++jj) {
+                    uint32_t sp = 0u, bp = 0u;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int q = 2 * (j0 + 2 * jj) + h;
+                        if (n < p.N && q < ng) {
+                            const int64_t at = static_cast<int64_t>(n) * p.G + g0 + q;
+                            sp |= static_cast<uint32_t>(__half_as_ushort(__ldg(p.scales + at))) << (16 * h);
+                            bp |= static_cast<uint32_t>(__half_as_ushort(__ldg(p.biases + at))) << (16 * h);
+                        }
+                    }
+                    sw[jj] = sp;
+                    bw[jj] = bp;
                 }
             }
             const float* xsp = reinterpret_cast<const float*>(pt + 2 * kParHalf);     // [CG][NT]
 #pragma unroll
-            for (int k = 0; k < CG / 2; ++k) {
-                const int q = q0 + 2 * k;
-                if (q >= ng) break;
-                const uint32_t gq = gi + static_cast<uint32_t>(q);
-                const int sl = static_cast<int>(gq % NS);
-                float sc = 0.0f, cc = 0.0f;
-                if (n < p.N) {
-                    sc = __half2float(sv[k]);
-                    cc = fmaf(-128.0f, sc, __half2float(bv[k]));
-                }
-                // the activation-sum term first (few live registers), then the tensor-core sums
-                const float4* xsq = reinterpret_cast<const float4*>(xsp + q * NT);
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j = j0 + 2 * jj;
+                if (j >= np) break;
+                const uint32_t pc = pb + static_cast<uint32_t>(j);
+                const int sl = static_cast<int>(pc % NS);
+                float sc[2];
+                // the bias terms first (few live registers), then the tensor-core sums
 #pragma unroll
-                for (int t4 = 0; t4 < NT / 4; ++t4) {
-                    const float4 v = xsq[t4];
-                    yacc[4 * t4 + 0] = fmaf(cc, v.x, yacc[4 * t4 + 0]);
-                    yacc[4 * t4 + 1] = fmaf(cc, v.y, yacc[4 * t4 + 1]);
-                    yacc[4 * t4 + 2] = fmaf(cc, v.z, yacc[4 * t4 + 2]);
-                    yacc[4 * t4 + 3] = fmaf(cc, v.w, yacc[4 * t4 + 3]);
+                for (int h = 0; h < 2; ++h) {
+                    const int q = 2 * j + h;
+                    sc[h] = 0.0f;
+                    if (q < ng) {
+                        float bb = 0.0f;
+                        if (n < p.N) {
+                            sc[h] = __half2float(__ushort_as_half(static_cast<unsigned short>(sw[jj] >> (16 * h))));
+                            bb = __half2float(__ushort_as_half(static_cast<unsigned short>(bw[jj] >> (16 * h))));
+                        }
+                        const float2 b2 = make_float2(bb, bb);
+                        const float4* xsq = reinterpret_cast<const float4*>(xsp + q * NT);
+#pragma unroll
+                        for (int t4 = 0; t4 < NT / 4; ++t4) {
+                            const float4 v = xsq[t4];
+                            yacc[2 * t4] = fma2(b2, make_float2(v.x, v.y), yacc[2 * t4]);
+                            yacc[2 * t4 + 1] = fma2(b2, make_float2(v.z, v.w), yacc[2 * t4 + 1]);
+                        }
+                    }
                 }
-                got = ptx::mbar_wait(&done[sl], (gq / NS) & 1u, abort_flag);
+                got = ptx::mbar_wait(&done[sl], (pc / NS) & 1u, abort_flag);
                 if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
                 ptx::tc_fence_after_sync();
-                uint32_t dv[NT];
-                if constexpr (NT == 32) {
-                    ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + L::kAccCol + static_cast<uint32_t>(sl * NT),
-                                            *reinterpret_cast<uint32_t(*)[32]>(dv));
-                } else {
-                    ptx::tmem_ld_32x32b_x16(tmem_base + lane_addr + L::kAccCol + static_cast<uint32_t>(sl * NT),
-                                            *reinterpret_cast<uint32_t(*)[16]>(dv));
-                }
-                ptx::tmem_wait_ld();
 #pragma unroll
-                for (int t = 0; t < NT; ++t) yacc[t] = fmaf(sc, __uint_as_float(dv[t]), yacc[t]);
+                for (int h = 0; h < 2; ++h) {
+                    if (2 * j + h < ng) {
+                        const float2 s2 = make_float2(sc[h], sc[h]);
+#pragma unroll
+                        for (int half = 0; half < NT / 16; ++half) {
+                            uint32_t dv[16];
+                            ptx::tmem_ld_32x32b_x16(tmem_base + lane_addr + L::kAccCol +
+                                                        static_cast<uint32_t>((2 * sl + h) * NT + 16 * half), dv);
+                            ptx::tmem_wait_ld();
+#pragma unroll
+                            for (int t2 = 0; t2 < 8; ++t2)
+                                yacc[8 * half + t2] = fma2(s2, make_float2(__uint_as_float(dv[2 * t2]), __uint_as_float(dv[2 * t2 + 1])),
+                                                           yacc[8 * half + t2]);
+                        }
+                    }
+                }
                 ptx::tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&ready[sl]);
@@ -451,17 +558,17 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
             if (!ok) break;
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&p_empty[pr]);
-            gi += static_cast<uint32_t>(ng);
+            pb += static_cast<uint32_t>(np);
             // end of this tile's segment: write this copy's partial and start over
-            const bool seg_end = (i + 1 == nchunks) || ((u0 + i + 1) % p.cpt == 0);
+            const bool seg_end = (i + 1 == nchunks) || (cp.cq + 1 == p.cpt);
             if (seg_end) {
                 float* dst = p.partial +
-                             (((static_cast<int64_t>(blockIdx.x) * p.segmax + (w - w_first)) * 2 + par) * p.M) * BW;
+                             (((static_cast<int64_t>(blockIdx.x) * p.segmax + (w - w_first)) * 2 + copy) * p.M) * BW;
 #pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    if (t < p.M) dst[static_cast<int64_t>(t) * BW + r] = yacc[t];
-                    yacc[t] = 0.0f;
-                }
+                for (int t = 0; t < NT; ++t)
+                    if (t < p.M) dst[static_cast<int64_t>(t) * BW + r] = (t & 1) ? yacc[t >> 1].y : yacc[t >> 1].x;
+#pragma unroll
+                for (int t = 0; t < NT / 2; ++t) yacc[t] = make_float2(0.0f, 0.0f);
             }
         }
     }
@@ -475,9 +582,11 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     }
 }
 
-// y[t][n] = sum over the CTAs whose runs cover tile n/128, in CTA order, of their two partials for that tile.
+// y[t][n] = 2^rowexp[t] * (sum over the CTAs whose runs cover tile n/128, in CTA order, of their two
+// partials for that tile).
 template <bool kBf16Out>
-__global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restrict__ partial, void* __restrict__ y,
+__global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restrict__ partial,
+                                                            const int* __restrict__ rowexp, void* __restrict__ y,
                                                             int M, int N, int cpt, int64_t units, int P, int segmax) {
     ptx::grid_dependency_wait();
     const int64_t total = static_cast<int64_t>(M) * N;
@@ -498,6 +607,7 @@ __global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restr
             acc += partial[((seg + 0) * M + t) * BW + r];
             acc += partial[((seg + 1) * M + t) * BW + r];
         }
+        acc = ldexpf(acc, rowexp[t]);
         if constexpr (kBf16Out) {
             reinterpret_cast<__nv_bfloat16*>(y)[e] = __float2bfloat16_rn(acc);
         } else {
