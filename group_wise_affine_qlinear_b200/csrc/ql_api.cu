@@ -147,8 +147,10 @@ struct Plan {
     size_t workspace = 0;
     // fused path workspace carve-up
     size_t off_xh = 0, off_rs = 0, off_sb = 0;
-    // skinny path workspace carve-up: partials, scaled f16 activations, activation sums, row exponents
-    size_t off_xp = 0, off_xs = 0, off_re = 0;
+    // skinny path workspace carve-up: partials, scaled f16 activations, activation sums, row exponents,
+    // per-slice row maxima
+    size_t off_xp = 0, off_xs = 0, off_re = 0, off_pm = 0;
+    int slices = 0;
 };
 
 ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int sm_count, Plan* plan) {
@@ -174,7 +176,9 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         plan->off_xp = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * 2 * M * skinny::BW * sizeof(float), 256);
         plan->off_xs = plan->off_xp + round_up(static_cast<size_t>(M) * K * 2, 256);
         plan->off_re = plan->off_xs + round_up(static_cast<size_t>(G) * plan->nt * sizeof(float), 256);
-        plan->workspace = plan->off_re + round_up(static_cast<size_t>(plan->nt) * sizeof(int), 256);
+        plan->slices = static_cast<int>((K / 8 + 255) / 256);
+        plan->off_pm = plan->off_re + round_up(static_cast<size_t>(plan->nt) * sizeof(int), 256);
+        plan->workspace = plan->off_pm + round_up(static_cast<size_t>(M) * plan->slices * sizeof(float), 256);
         return QL_OK;
     }
     if (path == QL_PATH_TC_FUSED) {
@@ -274,10 +278,10 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
 // Launches with programmatic stream serialization: the kernel may start while the previous
 // kernel on the stream is still running and waits for it (griddepcontrol.wait) where it must.
 template <typename... KArgs, typename... Args>
-ql_status launch_dependent(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st,
+ql_status launch_dependent(void (*kernel)(KArgs...), dim3 grid, int block, size_t smem, cudaStream_t st,
                            Args&&... args) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.gridDim = grid;
     cfg.blockDim = dim3(static_cast<unsigned>(block));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
@@ -297,6 +301,7 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     void* xp = wsb + pl.off_xp;
     float* xs = reinterpret_cast<float*>(wsb + pl.off_xs);
     int* rowexp = reinterpret_cast<int*>(wsb + pl.off_re);
+    float* pmax = reinterpret_cast<float*>(wsb + pl.off_pm);
     CUtensorMap mc, mx, mxs;
     ql_status s;
     if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K / 8, N, K / 2,
@@ -331,31 +336,46 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     p.cpt = static_cast<int>((G + skinny::CG - 1) / skinny::CG);
     p.units = pl.units;
     p.segmax = pl.segmax;
-    // scaled and reordered f16 activations, per-group activation sums, row exponents: one CTA per row
-    skinny::skinny_prepass_kernel<<<static_cast<unsigned>(pl.nt), 256, 0, st>>>(
-        static_cast<const uint4*>(x), static_cast<uint4*>(xp), xs, rowexp, p.M, static_cast<int>(K), pl.nt);
+    // row maxima, then scaled and reordered f16 activations, per-group activation sums, row exponents
+    const dim3 pre_grid(static_cast<unsigned>(pl.slices), static_cast<unsigned>(M));
+    skinny::skinny_rowmax_kernel<<<pre_grid, 256, 0, st>>>(static_cast<const uint4*>(x), pmax, static_cast<int>(K));
     if ((s = launch_status()) != QL_OK) return s;
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = pre_grid;
+        cfg.blockDim = dim3(256);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const float* pm = pmax;
+        if (cudaLaunchKernelEx(&cfg, skinny::skinny_prepass_kernel, static_cast<const uint4*>(x), pm,
+                               static_cast<uint4*>(xp), xs, rowexp, static_cast<int>(K), pl.nt) != cudaSuccess)
+            return QL_ERR_CUDA;
+    }
     prof_begin(st);
     if (pl.nt == 16)
-        s = launch_dependent(skinny::skinny_kernel<16>, pl.ctas, skinny::kThreads, skinny::Layout<16>::kSmemBytes, st,
+        s = launch_dependent(skinny::skinny_kernel<16>, dim3(static_cast<unsigned>(pl.ctas)), skinny::kThreads, skinny::Layout<16>::kSmemBytes, st,
                              mc, mx, ms, mb, mxs, p);
     else
-        s = launch_dependent(skinny::skinny_kernel<32>, pl.ctas, skinny::kThreads, skinny::Layout<32>::kSmemBytes, st,
+        s = launch_dependent(skinny::skinny_kernel<32>, dim3(static_cast<unsigned>(pl.ctas)), skinny::kThreads, skinny::Layout<32>::kSmemBytes, st,
                              mc, mx, ms, mb, mxs, p);
     if (s != QL_OK) return s;
     prof_end(st);
-    const int64_t total = M * N;
-    const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4 * sm_count));
     const float* part = p.partial;
     const int* rexp = rowexp;
+    const dim3 red_grid(static_cast<unsigned>(p.num_w), static_cast<unsigned>((M + 1) / 2));
     if (bf16_out)
-        s = launch_dependent(skinny::skinny_reduce_kernel<true>, blocks, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
+        s = launch_dependent(skinny::skinny_reduce_kernel<true>, red_grid, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
                              p.units, pl.ctas, pl.segmax);
     else
-        s = launch_dependent(skinny::skinny_reduce_kernel<false>, blocks, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
+        s = launch_dependent(skinny::skinny_reduce_kernel<false>, red_grid, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
                              p.units, pl.ctas, pl.segmax);
     if (s != QL_OK) return s;
-    set_dispatch("path=tc_skinny nt=%d ctas=%d segmax=%d units=%lld launches=3", pl.nt, pl.ctas, pl.segmax,
+    (void)sm_count;
+    set_dispatch("path=tc_skinny nt=%d ctas=%d segmax=%d units=%lld launches=4", pl.nt, pl.ctas, pl.segmax,
                  static_cast<long long>(pl.units));
     return launch_status();
 }

@@ -21,10 +21,10 @@
 //   D_g[n][t] = sum_{k in g} A[n][k] x'[t][k] = 2^(e_t - 24) sum_{k in g} q(n,k) x[t][k].
 // The prepass also writes xs_g[t] = 2^(e_t - 24) sum_{k in g} x[t][k], so the drain
 // accumulates s * D + b * xs, all scaled by 2^(e_t - 24), and the reduce kernel
-// scales back by 2^(24 - e_t) (ldexpf, exact).  Activation entries below 2^-25 of
+// scales back by 2^(24 - e_t) (ldexpf, exact).  Activation entries below 2^-24 of
 // the row maximum lose bits as f16 subnormals; nothing else is rounded before the
-// fp32 accumulation.  The prepass runs under programmatic dependent launch: the
-// main kernel starts streaming codes at once and waits for the prepass only
+// fp32 accumulation.  The prepass kernels run under programmatic dependent launch:
+// the main kernel starts streaming codes at once and waits for the prepass only
 // before its first activation load.
 //
 // Stream-K schedule: the work is cut into chunks of CG = 8 consecutive groups of
@@ -136,65 +136,73 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
     return *reinterpret_cast<float2*>(&d);
 }
 
-// Per activation row t (one CTA each, t < NT): e_t puts max_k |x[t][k]| in [2^14, 2^15) (0 for a
-// zero or non-finite row); xp[t][k] = f16(x * 2^e_t), times 2^-4 at odd k, in the order
-// 0,4,1,5,2,6,3,7 of each 8-block; xs[g][t] = 2^(e_t - 24) * sum over group g of x[t][k] in fp32
-// (zero for t >= M); rowexp[t] = 24 - e_t.
-__global__ void __launch_bounds__(256) skinny_prepass_kernel(const uint4* __restrict__ x, uint4* __restrict__ xp,
-                                                             float* __restrict__ xs, int* __restrict__ rowexp,
-                                                             int M, int K, int NT) {
+// Activation prepass, two kernels over a grid of (slice, row): one thread per 8-block of k, 256 per
+// CTA, so every 8-block of a row is read in parallel.
+
+// pmax[t][slice] = max |x[t][k]| over the slice's 8-blocks.
+__global__ void __launch_bounds__(256) skinny_rowmax_kernel(const uint4* __restrict__ x, float* __restrict__ pmax,
+                                                            int K) {
     ptx::launch_dependents();
     __shared__ float red[8];
-    const int t = blockIdx.x;
-    const int kb = K / 8;                                      // 8-blocks per row, a multiple of 8
-    const bool row = t < M;
-    const uint4* xr = x + static_cast<int64_t>(t) * kb;
+    const int t = blockIdx.y, kb = K / 8;
+    const int c = blockIdx.x * 256 + threadIdx.x;
     float m = 0.0f;
-    if (row)
-        for (int c = threadIdx.x; c < kb; c += blockDim.x) {
-            const uint4 v = xr[c];
-            m = fmaxf(m, fmaxf(fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))),
-                               fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w))))));
-        }
+    if (c < kb) {
+        const uint4 v = x[static_cast<int64_t>(t) * kb + c];
+        m = fmaxf(fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))),
+                  fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     __syncthreads();
-    m = red[0];
-    for (int i = 1; i < static_cast<int>(blockDim.x >> 5); ++i) m = fmaxf(m, red[i]);
+    if (threadIdx.x == 0) {
+        for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
+        pmax[static_cast<int64_t>(t) * gridDim.x + blockIdx.x] = fmaxf(m, red[0]);
+    }
+}
+
+// For row t: e_t puts max_k |x[t][k]| in [2^14, 2^15) (0 for a zero or non-finite row);
+// xp[t][k] = f16(x * 2^e_t), times 2^-4 at odd k, in the order 0,4,1,5,2,6,3,7 of each 8-block;
+// xs[g][t] = 2^(e_t - 24) * (sum over group g of x[t][k], fp32); rowexp[t] = 24 - e_t.  The 8
+// blocks of a group are 8 aligned lanes.  Columns t >= M of xs are never read back.
+__global__ void __launch_bounds__(256) skinny_prepass_kernel(const uint4* __restrict__ x, const float* __restrict__ pmax,
+                                                             uint4* __restrict__ xp, float* __restrict__ xs,
+                                                             int* __restrict__ rowexp, int K, int NT) {
+    ptx::launch_dependents();
+    ptx::grid_dependency_wait();                               // pmax comes from the kernel before
+    const int t = blockIdx.y, kb = K / 8;
+    const int c = blockIdx.x * 256 + threadIdx.x;
+    float m = 0.0f;
+    for (int i = 0; i < static_cast<int>(gridDim.x); ++i) m = fmaxf(m, pmax[static_cast<int64_t>(t) * gridDim.x + i]);
     int ex = 0;
     if (m > 0.0f && m <= 3.4028235e38f) {
         int E;
         frexpf(m, &E);                                         // m = f 2^E, f in [0.5, 1)
         ex = 15 - E;
     }
-    if (threadIdx.x == 0) rowexp[t] = 24 - ex;
-    // the 8 blocks of a group are 8 consecutive threads (blockDim.x is a multiple of 8)
-    const int iters = (kb + static_cast<int>(blockDim.x) - 1) / static_cast<int>(blockDim.x);
-    for (int it = 0; it < iters; ++it) {
-        const int c = it * static_cast<int>(blockDim.x) + static_cast<int>(threadIdx.x);
-        const bool in = c < kb;
-        float sum = 0.0f;
-        if (in && row) {
-            const uint4 v = xr[c];
-            const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                                bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-            sum = ((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]));
-            // slot pairs (k0, k4) (k1, k5) (k2, k6) (k3, k7); odd k carry the extra 2^-4
-            uint32_t o[4];
+    if (blockIdx.x == 0 && threadIdx.x == 0) rowexp[t] = 24 - ex;
+    const bool in = c < kb;
+    float sum = 0.0f;
+    if (in) {
+        const uint4 v = x[static_cast<int64_t>(t) * kb + c];
+        const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                            bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+        sum = ((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]));
+        // slot pairs (k0, k4) (k1, k5) (k2, k6) (k3, k7); odd k carry the extra 2^-4
+        uint32_t o[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int sh = ex - ((j & 1) ? 4 : 0);
-                const __half2 h = __halves2half2(__float2half_rn(ldexpf(f[j], sh)), __float2half_rn(ldexpf(f[j + 4], sh)));
-                o[j] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            xp[static_cast<int64_t>(t) * kb + c] = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int j = 0; j < 4; ++j) {
+            const int sh = ex - ((j & 1) ? 4 : 0);
+            const __half2 h = __halves2half2(__float2half_rn(ldexpf(f[j], sh)), __float2half_rn(ldexpf(f[j + 4], sh)));
+            o[j] = *reinterpret_cast<const uint32_t*>(&h);
         }
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
-        if (in && (c & 7) == 0) xs[static_cast<int64_t>(c >> 3) * NT + t] = row ? ldexpf(sum, ex - 24) : 0.0f;
+        xp[static_cast<int64_t>(t) * kb + c] = make_uint4(o[0], o[1], o[2], o[3]);
     }
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+    sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
+    if (in && (c & 7) == 0) xs[static_cast<int64_t>(c >> 3) * NT + t] = ldexpf(sum, ex - 24);
 }
 
 template <int NT>
@@ -583,36 +591,45 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
 }
 
 // y[t][n] = 2^rowexp[t] * (sum over the CTAs whose runs cover tile n/128, in CTA order, of their two
-// partials for that tile).
+// partials for that tile).  One CTA per (tile, 2 tokens): the tile's CTA range is found once.
 template <bool kBf16Out>
 __global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restrict__ partial,
                                                             const int* __restrict__ rowexp, void* __restrict__ y,
                                                             int M, int N, int cpt, int64_t units, int P, int segmax) {
-    ptx::grid_dependency_wait();
-    const int64_t total = static_cast<int64_t>(M) * N;
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
-        const int t = static_cast<int>(e / N), n = static_cast<int>(e % N);
-        const int w = n / BW, r = n % BW;
+    __shared__ int range[3];
+    const int w = blockIdx.x;
+    if (threadIdx.x == 0) {
         // CTAs whose run of chunks [first(c), first(c+1)) meets [w*cpt, (w+1)*cpt)
         const int64_t lo = static_cast<int64_t>(w) * cpt, hi = lo + cpt;
         int c = static_cast<int>((lo * P) / units);
         while (c > 0 && run_first(units, P, c) > lo) --c;
         while (c + 1 <= P && run_first(units, P, c + 1) <= lo) ++c;
-        float acc = 0.0f;
-        for (; c < P && run_first(units, P, c) < hi; ++c) {
-            if (run_first(units, P, c + 1) <= run_first(units, P, c)) continue;      // empty run
-            const int w_first = static_cast<int>(run_first(units, P, c) / cpt);
-            const int64_t seg = (static_cast<int64_t>(c) * segmax + (w - w_first)) * 2;
-            acc += partial[((seg + 0) * M + t) * BW + r];
-            acc += partial[((seg + 1) * M + t) * BW + r];
-        }
-        acc = ldexpf(acc, rowexp[t]);
-        if constexpr (kBf16Out) {
-            reinterpret_cast<__nv_bfloat16*>(y)[e] = __float2bfloat16_rn(acc);
-        } else {
-            reinterpret_cast<float*>(y)[e] = acc;
-        }
+        int c1 = c;
+        while (c1 < P && run_first(units, P, c1) < hi) ++c1;
+        range[0] = c;
+        range[1] = c1;
+    }
+    ptx::grid_dependency_wait();                               // partials come from the kernel before
+    __syncthreads();
+    const int c0 = range[0], c1 = range[1];
+    const int t = blockIdx.y * 2 + (threadIdx.x >> 7), r = threadIdx.x & 127;
+    const int n = w * BW + r;
+    if (t >= M || n >= N) return;
+    float acc = 0.0f;
+    for (int c = c0; c < c1; ++c) {
+        const int64_t f0 = run_first(units, P, c), f1 = run_first(units, P, c + 1);
+        if (f1 <= f0) continue;                                // empty run
+        const int w_first = static_cast<int>(f0 / cpt);
+        const int64_t seg = (static_cast<int64_t>(c) * segmax + (w - w_first)) * 2;
+        acc += partial[((seg + 0) * M + t) * BW + r];
+        acc += partial[((seg + 1) * M + t) * BW + r];
+    }
+    acc = ldexpf(acc, rowexp[t]);
+    const int64_t e = static_cast<int64_t>(t) * N + n;
+    if constexpr (kBf16Out) {
+        reinterpret_cast<__nv_bfloat16*>(y)[e] = __float2bfloat16_rn(acc);
+    } else {
+        reinterpret_cast<float*>(y)[e] = acc;
     }
 }
 
