@@ -169,7 +169,7 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         plan->nt = M <= 16 ? 16 : 32;
         const int64_t cpt = (G + skinny::CG - 1) / skinny::CG;
         plan->units = ((N + skinny::BW - 1) / skinny::BW) * cpt;
-        plan->ctas = static_cast<int>(std::min<int64_t>(sm_count, plan->units));
+        plan->ctas = static_cast<int>(std::min<int64_t>(std::min(sm_count, skinny::kMaxCtas), plan->units));
         const int64_t run = (plan->units + plan->ctas - 1) / plan->ctas;
         plan->segmax = static_cast<int>((run + cpt - 1) / cpt + 1);
         plan->split_k = 1;
@@ -222,6 +222,24 @@ ql_status run_gemv(const Plan& pl, const void* x, const uint32_t* codes, const v
     return launch_status();
 }
 
+// Launches with programmatic stream serialization: the kernel may start while the previous
+// kernel on the stream is still running and waits for it (griddepcontrol.wait) where it must.
+template <typename... KArgs, typename... Args>
+ql_status launch_dependent(void (*kernel)(KArgs...), dim3 grid, int block, size_t smem, cudaStream_t st,
+                           Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(static_cast<unsigned>(block));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}
+
 ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const void* scales, const void* biases,
                     void* y, bool bf16_out, int64_t M, int64_t K, int64_t N, void* ws, cudaStream_t st,
                     int sm_count) {
@@ -249,9 +267,13 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
 
     convert_x_kernel<<<static_cast<unsigned>(M), kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), xh, rs,
                                                                         static_cast<int>(K));
+    if ((s = launch_status()) != QL_OK) return s;
+    // the transpose, then the fused kernel, start under programmatic dependent launch (each waits
+    // for the kernels before it where it reads their output)
     const dim3 tgrid(static_cast<unsigned>((G + 31) / 32), static_cast<unsigned>((N + 31) / 32));
-    transpose_params_kernel<<<tgrid, 256, 0, st>>>(static_cast<const __half*>(scales), static_cast<const __half*>(biases),
-                                                   sb, static_cast<int>(N), static_cast<int>(G));
+    if ((s = launch_dependent(transpose_params_kernel, tgrid, 256, 0, st, static_cast<const __half*>(scales),
+                              static_cast<const __half*>(biases), sb, static_cast<int>(N), static_cast<int>(G))) != QL_OK)
+        return s;
     fused::Params p;
     p.rowscale = rs;
     p.y = y;
@@ -265,32 +287,17 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     using FC = fused::DefaultCfg;
     prof_begin(st);
     if (bf16_out)
-        fused::fused_gemm_kernel<true, FC><<<grid, fused::kThreads, FC::kSmemBytes, st>>>(mx, mc, mp, my, p);
+        s = launch_dependent(fused::fused_gemm_kernel<true, FC>, dim3(static_cast<unsigned>(grid)), fused::kThreads,
+                             FC::kSmemBytes, st, mx, mc, mp, my, p);
     else
-        fused::fused_gemm_kernel<false, FC><<<grid, fused::kThreads, FC::kSmemBytes, st>>>(mx, mc, mp, my, p);
+        s = launch_dependent(fused::fused_gemm_kernel<false, FC>, dim3(static_cast<unsigned>(grid)), fused::kThreads,
+                             FC::kSmemBytes, st, mx, mc, mp, my, p);
+    if (s != QL_OK) return s;
     prof_end(st);
     set_dispatch("path=tc_fused tile=%dw x %dt x %dk stages=x%d/c%d/a%d ctas=%d splitk=1 launches=3", fused::BW,
                  fused::BT, fused::BK, FC::kNX, FC::kNC, fused::NA, grid);
     (void)codes;
     return launch_status();
-}
-
-// Launches with programmatic stream serialization: the kernel may start while the previous
-// kernel on the stream is still running and waits for it (griddepcontrol.wait) where it must.
-template <typename... KArgs, typename... Args>
-ql_status launch_dependent(void (*kernel)(KArgs...), dim3 grid, int block, size_t smem, cudaStream_t st,
-                           Args&&... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(static_cast<unsigned>(block));
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
 ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const void* scales, const void* biases,

@@ -15,7 +15,7 @@
 //    can be fetched by the tensor memory accelerator.
 #pragma once
 
-#include "ql_common.cuh"
+#include "ql_ptx.cuh"
 
 namespace ql {
 
@@ -25,6 +25,7 @@ constexpr int kPrepThreads = 256;
 __global__ void __launch_bounds__(kPrepThreads) convert_x_kernel(const __nv_bfloat16* __restrict__ x,
                                                                  __half* __restrict__ xh,
                                                                  float* __restrict__ rowscale, int K) {
+    ptx::launch_dependents();
     __shared__ float red[kPrepThreads / 32];
     __shared__ int row_exp;
     const int64_t m = blockIdx.x;
@@ -76,10 +77,13 @@ __global__ void __launch_bounds__(kPrepThreads) convert_x_kernel(const __nv_bflo
     }
 }
 
-// sb[g][n] = (scale[n][g], bias[n][g]); 32x32 tiles through shared memory.
+// sb[g][n] = (scale[n][g], bias[n][g]); 32x32 tiles through shared memory.  Launched behind
+// convert_x_kernel under programmatic dependent launch: it does not read that kernel's output, so it
+// runs alongside it, and waits for it only before finishing, so that its own completion implies both.
 __global__ void __launch_bounds__(256) transpose_params_kernel(const __half* __restrict__ scales,
                                                                const __half* __restrict__ biases,
                                                                uint32_t* __restrict__ sb, int N, int G) {
+    ptx::launch_dependents();
     __shared__ uint32_t tile[32][33];
     const int g0 = blockIdx.x * 32, n0 = blockIdx.y * 32;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;     // 8 rows per pass
@@ -98,6 +102,7 @@ __global__ void __launch_bounds__(256) transpose_params_kernel(const __half* __r
         const int g = g0 + r, n = n0 + tx;
         if (g < G && n < N) sb[static_cast<int64_t>(g) * N + n] = tile[tx][r];
     }
+    ptx::grid_dependency_wait();
 }
 
 }  // namespace ql

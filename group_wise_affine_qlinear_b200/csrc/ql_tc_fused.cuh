@@ -236,10 +236,34 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             uint64_t* empty = is_x ? x_empty : c_empty;
             uint32_t i = 0;
             bool ok = true;
+            // The activations and the parameter pairs come from the kernels before this one on the
+            // stream (programmatic dependent launch): the code loads of the first NC stages go out
+            // at once, their parameter loads (same stage barrier) once those kernels are done.
+            const uint32_t first_steps = static_cast<uint32_t>(p.G) * static_cast<uint32_t>(
+                (num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x));
+            const uint32_t early = is_x ? 0u : min(static_cast<uint32_t>(NC), first_steps);
+            auto step_coords = [&](uint32_t step, int& kb, int& w_blk, int& t_blk) {
+                const int t = static_cast<int>(blockIdx.x) + static_cast<int>(step / p.G) * static_cast<int>(gridDim.x);
+                kb = static_cast<int>(step % p.G);
+                tile_coords(t, p.num_w, t_blk, w_blk);
+            };
+            for (uint32_t e = 0; e < early; ++e) {       // fresh stages: no empty wait
+                int kb, w_blk, t_blk;
+                step_coords(e, kb, w_blk, t_blk);
+                ptx::mbar_arrive_expect_tx(&full[e], kCBytes + kPBytes);
+                ptx::tma_load_2d(smem + C::kOffC + e * kCBytes, &map_codes, &full[e], kb * (BK / 8), w_blk * BW);
+            }
+            ptx::grid_dependency_wait();
+            for (uint32_t e = 0; e < early; ++e) {
+                int kb, w_blk, t_blk;
+                step_coords(e, kb, w_blk, t_blk);
+                ptx::tma_load_2d(smem + C::kOffP + e * kPBytes, &map_params, &full[e], w_blk * BW, kb);
+            }
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 int t_blk, w_blk;
                 tile_coords(t, p.num_w, t_blk, w_blk);
                 for (int kb = 0; kb < p.G; ++kb, ++i) {
+                    if (i < early) continue;
                     const int s = static_cast<int>(i % depth);
                     const uint32_t ph = (i / depth) & 1u;
                     if (!ptx::mbar_wait(&empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
@@ -311,6 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         uint8_t* epi_stage = smem + C::kOffEpi + (warp - kWarpEpi0) * 2 * kStageBytes;
         uint32_t nstore = 0;
         int j = 0;
+        ptx::grid_dependency_wait();               // the row scales come from the kernels before this one
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++j) {
             int t_blk, w_blk;
             tile_coords(t, p.num_w, t_blk, w_blk);

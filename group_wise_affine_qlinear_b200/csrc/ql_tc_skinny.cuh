@@ -591,36 +591,44 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
 }
 
 // y[t][n] = 2^rowexp[t] * (sum over the CTAs whose runs cover tile n/128, in CTA order, of their two
-// partials for that tile).  One CTA per (tile, 2 tokens): the tile's CTA range is found once.
+// partials for that tile).  One CTA per (tile, 2 tokens): thread 0 lists the covering CTAs' segment
+// bases once, the other threads only load and add.
+constexpr int kMaxCtas = 256;                // the planner launches at most this many CTAs, so every
+                                             // tile's covering CTAs fit the reduce kernel's list
 template <bool kBf16Out>
 __global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restrict__ partial,
                                                             const int* __restrict__ rowexp, void* __restrict__ y,
                                                             int M, int N, int cpt, int64_t units, int P, int segmax) {
-    __shared__ int range[3];
+    __shared__ int64_t seg_base[kMaxCtas];
+    __shared__ int count;
     const int w = blockIdx.x;
     if (threadIdx.x == 0) {
-        // CTAs whose run of chunks [first(c), first(c+1)) meets [w*cpt, (w+1)*cpt)
+        // CTAs whose run of chunks [first(c), first(c+1)) meets [w*cpt, (w+1)*cpt), in CTA order
         const int64_t lo = static_cast<int64_t>(w) * cpt, hi = lo + cpt;
         int c = static_cast<int>((lo * P) / units);
         while (c > 0 && run_first(units, P, c) > lo) --c;
         while (c + 1 <= P && run_first(units, P, c + 1) <= lo) ++c;
-        int c1 = c;
-        while (c1 < P && run_first(units, P, c1) < hi) ++c1;
-        range[0] = c;
-        range[1] = c1;
+        int k = 0;
+        int64_t f0 = run_first(units, P, c);
+        for (; c < P && f0 < hi; ++c) {
+            const int64_t f1 = run_first(units, P, c + 1);
+            if (f1 > f0) {                                        // non-empty run
+                const int w_first = static_cast<int>(f0 / cpt);
+                seg_base[k++] = (static_cast<int64_t>(c) * segmax + (w - w_first)) * 2;
+            }
+            f0 = f1;
+        }
+        count = k;
     }
-    ptx::grid_dependency_wait();                               // partials come from the kernel before
+    ptx::grid_dependency_wait();                                  // partials come from the kernel before
     __syncthreads();
-    const int c0 = range[0], c1 = range[1];
     const int t = blockIdx.y * 2 + (threadIdx.x >> 7), r = threadIdx.x & 127;
     const int n = w * BW + r;
     if (t >= M || n >= N) return;
     float acc = 0.0f;
-    for (int c = c0; c < c1; ++c) {
-        const int64_t f0 = run_first(units, P, c), f1 = run_first(units, P, c + 1);
-        if (f1 <= f0) continue;                                // empty run
-        const int w_first = static_cast<int>(f0 / cpt);
-        const int64_t seg = (static_cast<int64_t>(c) * segmax + (w - w_first)) * 2;
+    const int k_end = count;
+    for (int k = 0; k < k_end; ++k) {
+        const int64_t seg = seg_base[k];
         acc += partial[((seg + 0) * M + t) * BW + r];
         acc += partial[((seg + 1) * M + t) * BW + r];
     }

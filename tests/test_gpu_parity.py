@@ -139,14 +139,42 @@ def test_skinny_rejects_large_m():
 
 
 @pytest.mark.parametrize("M", [1, 8, 16, 17, 32])
-@pytest.mark.parametrize("K,N", [(64, 8), (128, 4608), (4096, 264), (8192, 1032)])
+@pytest.mark.parametrize("K,N", [(64, 8), (128, 4608), (4096, 264), (8192, 1032), (65536, 128), (4160, 200)])
 def test_skinny_stream_k_shapes(M, K, N):
-    """Runs that start and end inside tiles, tiles shorter than a run, ragged N."""
+    """Runs that start and end inside tiles, tiles shorter than a run, ragged N, one tile shared by
+    128 CTAs (65536 x 128), and a group count that is not a whole number of chunks (4160 = 65 groups)."""
     rng = np.random.default_rng(M * 7 + K + N)
     x, codes, s, b = random_layer(rng, M, K, N)
     y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=ql.PATH_TC_SKINNY)
     _check_tol(y, O.forward_ref(x, codes, s, b))
     assert ql.last_dispatch().startswith("path=tc_skinny")
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_activation_dynamic_range(path):
+    """Rows of very different magnitude: the tensor-core paths scale each activation row by its own
+    power of two before rounding it to f16, so every row must meet the tolerance on its own, a zero
+    row must give exact zeros, and a row of one spike plus tiny values must stay within tolerance."""
+    rng = np.random.default_rng(11)
+    K, N = 1024, 264
+    _, codes, s, b = random_layer(rng, 6, K, N)
+    base = rng.standard_normal((6, K))
+    rows = np.empty((6, K))
+    rows[0] = base[0]
+    rows[1] = 0.0
+    rows[2] = base[2] * 1e30
+    rows[3] = base[3] * 1e-30
+    rows[4] = np.sign(base[4]) * np.exp2(rng.uniform(-40, 40, K))
+    rows[5] = 1e-6 * base[5]
+    rows[5, 17] = 1e4
+    x = S.f32_to_bf16_bits(rows.astype(np.float32))
+    y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=PATHS[path])
+    ref = O.forward_ref(x, codes, s, b)
+    got = O.decode_bf16(bf16_bits(y))
+    assert np.all(got[1] == 0.0)
+    for t in (0, 2, 3, 4, 5):
+        tol = O.tolerance(got[t:t + 1], ref[t:t + 1], bf16_output=True)
+        assert tol["relF"] <= 4e-3 and tol["max_gate"] <= 1.5e-2, (t, tol)
 
 
 @pytest.mark.parametrize("path", list(PATHS))
