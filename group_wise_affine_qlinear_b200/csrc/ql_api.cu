@@ -147,9 +147,8 @@ struct Plan {
     size_t workspace = 0;
     // fused path workspace carve-up
     size_t off_xh = 0, off_rs = 0, off_sb = 0;
-    // skinny path workspace carve-up: partials, scaled f16 activations, activation sums, row exponents,
-    // per-slice row maxima
-    size_t off_xp = 0, off_xs = 0, off_re = 0, off_pm = 0;
+    // skinny path workspace carve-up: partials, scaled f16 activations, row exponents, per-slice row maxima
+    size_t off_xp = 0, off_re = 0, off_pm = 0;
     int slices = 0;
 };
 
@@ -173,9 +172,8 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         const int64_t run = (plan->units + plan->ctas - 1) / plan->ctas;
         plan->segmax = static_cast<int>((run + cpt - 1) / cpt + 1);
         plan->split_k = 1;
-        plan->off_xp = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * 2 * M * skinny::BW * sizeof(float), 256);
-        plan->off_xs = plan->off_xp + round_up(static_cast<size_t>(M) * K * 2, 256);
-        plan->off_re = plan->off_xs + round_up(static_cast<size_t>(G) * plan->nt * sizeof(float), 256);
+        plan->off_xp = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * M * skinny::BW * sizeof(float), 256);
+        plan->off_re = plan->off_xp + round_up(static_cast<size_t>(M) * K * 2, 256);
         plan->slices = static_cast<int>((K / 8 + 255) / 256);
         plan->off_pm = plan->off_re + round_up(static_cast<size_t>(plan->nt) * sizeof(int), 256);
         plan->workspace = plan->off_pm + round_up(static_cast<size_t>(M) * plan->slices * sizeof(float), 256);
@@ -306,19 +304,15 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     const int64_t G = K / kGroup;
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     void* xp = wsb + pl.off_xp;
-    float* xs = reinterpret_cast<float*>(wsb + pl.off_xs);
     int* rowexp = reinterpret_cast<int*>(wsb + pl.off_re);
     float* pmax = reinterpret_cast<float*>(wsb + pl.off_pm);
-    CUtensorMap mc, mx, mxs;
+    CUtensorMap mc, mx;
     ql_status s;
     if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K / 8, N, K / 2,
                        skinny::kBoxGroups * skinny::BK / 8, skinny::BW, CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
     if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xp, K, M, K * 2, skinny::BK, pl.nt,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
-        return s;
-    if ((s = encode_2d(&mxs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, xs, pl.nt, G, pl.nt * 4, pl.nt, skinny::CG,
-                       CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
         return s;
     // scale/bias tiles by TMA need a 16-byte row pitch and chunk-aligned groups
     const bool param_tma = (G % skinny::CG) == 0;
@@ -359,16 +353,16 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
         cfg.numAttrs = 1;
         const float* pm = pmax;
         if (cudaLaunchKernelEx(&cfg, skinny::skinny_prepass_kernel, static_cast<const uint4*>(x), pm,
-                               static_cast<uint4*>(xp), xs, rowexp, static_cast<int>(K), pl.nt) != cudaSuccess)
+                               static_cast<uint4*>(xp), rowexp, static_cast<int>(K)) != cudaSuccess)
             return QL_ERR_CUDA;
     }
     prof_begin(st);
     if (pl.nt == 16)
         s = launch_dependent(skinny::skinny_kernel<16>, dim3(static_cast<unsigned>(pl.ctas)), skinny::kThreads, skinny::Layout<16>::kSmemBytes, st,
-                             mc, mx, ms, mb, mxs, p);
+                             mc, mx, ms, mb, p);
     else
         s = launch_dependent(skinny::skinny_kernel<32>, dim3(static_cast<unsigned>(pl.ctas)), skinny::kThreads, skinny::Layout<32>::kSmemBytes, st,
-                             mc, mx, ms, mb, mxs, p);
+                             mc, mx, ms, mb, p);
     if (s != QL_OK) return s;
     prof_end(st);
     const float* part = p.partial;

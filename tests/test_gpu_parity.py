@@ -192,8 +192,8 @@ def test_forward_tiny(path, out):
 def test_forward_one_hot_bitexact(path):
     """x rows = unit vectors: y selects single weights, so the result is exact.
 
-    CUDA-core and skinny paths (exact codes, fp32 scale and bias): y = RN_bf16(fp32 dequant).
-    Large-M tensor-core path (f16 operand): y = RN_bf16(RN_f16(w)).
+    CUDA-core path (exact codes, fp32 scale and bias): y = RN_bf16(fp32 dequant).
+    Tensor-core paths (weights dequantized to an f16 operand): y = RN_bf16(RN_f16(w)).
     """
     rng = np.random.default_rng(3)
     K, N = 320, 264
@@ -205,7 +205,7 @@ def test_forward_one_hot_bitexact(path):
     x[np.arange(ks.size), ks] = 0x3F80
     y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=PATHS[path])
     got = bf16_bits(y)
-    if path in ("gemv", "tc_skinny"):
+    if path == "gemv":
         ref = O.dequant_bf16(codes, s, b)[:, ks].T
     else:
         ref = O.round_bf16(O.dequant_f16(codes, s, b).astype(np.float64))[:, ks].T
