@@ -35,12 +35,14 @@
 // of a tile segment both issuers commit to acc_full, and the drain warps add the
 // two accumulators and write the partial; the accumulators are double-buffered
 // across segments (acc_empty).
-// Warp roles (736 threads, one CTA per SM; 6 warps per SM sub-partition leave 80 registers a thread):
-//   warp 0        TMA producer: per chunk one stage of codes (128 rows x CG*32 B, 128B swizzle) and
-//                 scale and bias tiles, and one stage of activation tiles (NT x 64 f16 per group)
-//   warps 1, 2    MMA issuers for even / odd pairs (warp 1 also allocates TMEM)
-//   warps 3-18    A builders, copies 0-3 of 4 warps: one weight row per thread
-//   warps 19-22   drain: one weight row per thread, at the end of each tile segment
+// Warp roles (768 threads, one CTA per SM; 6 warps per SM sub-partition leave 80 registers a thread):
+//   warp 0        TMA producer of code chunks (128 rows x CG*32 B, 128B swizzle) with their scale and
+//                 bias tiles
+//   warp 1        TMA producer of activation tiles (NT x 64 f16 per group), its own ring: activation
+//                 loads from L2 take about a microsecond, so they run several chunks ahead
+//   warps 2, 3    MMA issuers for even / odd pairs (warp 2 also allocates TMEM)
+//   warps 4-19    A builders, copies 0-3 of 4 warps: one weight row per thread
+//   warps 20-23   drain: one weight row per thread, at the end of each tile segment
 #pragma once
 
 #include "ql_ptx.cuh"
@@ -53,7 +55,7 @@ constexpr int BW = 128;
 constexpr int BK = 64;
 constexpr int UK = 16;
 constexpr int kBuildCopies = 4, kMmaCopies = 2;
-constexpr int kWarpTma = 0, kWarpMma0 = 1, kWarpBuild0 = 3, kWarpDrain0 = kWarpBuild0 + 4 * kBuildCopies;
+constexpr int kWarpTmaC = 0, kWarpTmaX = 1, kWarpMma0 = 2, kWarpBuild0 = 4, kWarpDrain0 = kWarpBuild0 + 4 * kBuildCopies;
 constexpr int kThreads = (kWarpDrain0 + 4) * 32;
 constexpr int CG = 8;                    // groups per chunk: four pairs, one per builder copy
 constexpr int kBoxGroups = 4;            // groups per code box: 128 bytes of each row (the 128B-swizzle span)
@@ -201,9 +203,9 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == kWarpTma && lane == 0) {
+    if (warp == kWarpTmaX && lane == 0) ptx::prefetch_tensormap(&map_x);
+    if (warp == kWarpTmaC && lane == 0) {
         ptx::prefetch_tensormap(&map_codes);
-        ptx::prefetch_tensormap(&map_x);
         if (p.param_tma) {
             ptx::prefetch_tensormap(&map_scales);
             ptx::prefetch_tensormap(&map_biases);
@@ -244,16 +246,17 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
         return static_cast<int>((static_cast<uint32_t>(copy) + nc - pb % nc) % nc);
     };
 
-    if (warp == kWarpTma) {
-        // ---------------------------------------------------------------- TMA producer
+    if (warp == kWarpTmaC) {
+        // ---------------------------------------------------------------- code + parameter producer
+        // (codes and parameters do not depend on the prepass: no dependency wait)
         if (lane == 0) {
-            uint32_t ci = 0, xi = 0;                 // chunks whose codes / activations were issued
-            ChunkPos cpc = start, cpi = start;       // positions of chunk ci and of chunk i
-            auto issue_codes = [&]() -> bool {
+            uint32_t ci = 0;
+            ChunkPos cp = start;
+            for (; ci < nchunks; ++ci, advance(cp)) {
                 int w, g0, ng;
-                chunk_groups(cpc, w, g0, ng);
+                chunk_groups(cp, w, g0, ng);
                 const int s = static_cast<int>(ci % NC);
-                if (!ptx::mbar_wait(&c_empty[s], ((ci / NC) & 1u) ^ 1u, abort_flag)) return false;
+                if (!ptx::mbar_wait(&c_empty[s], ((ci / NC) & 1u) ^ 1u, abort_flag)) break;
                 uint8_t* st = smem + L::kOffC + s * kStageBytes;
                 ptx::mbar_arrive_expect_tx(&c_full[s], kCBytes + (p.param_tma ? 2 * kParHalf : 0u));
 #pragma unroll
@@ -263,28 +266,26 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
                     ptx::tma_load_2d(st + kCBytes, &map_scales, &c_full[s], g0, w * BW);
                     ptx::tma_load_2d(st + kCBytes + kParHalf, &map_biases, &c_full[s], g0, w * BW);
                 }
-                advance(cpc);
-                ++ci;
-                return true;
-            };
-            // codes and parameters do not depend on the prepass: start streaming them at once
-            bool ok = true;
-            while (ok && ci < nchunks && ci < static_cast<uint32_t>(NC)) ok = issue_codes();
-            ptx::grid_dependency_wait();
-            for (uint32_t i = 0; i < nchunks && ok; ++i, advance(cpi)) {
-                int w, g0, ng;
-                chunk_groups(cpi, w, g0, ng);
-                const int xc = static_cast<int>(i % NXC);
-                if (!ptx::mbar_wait(&x_empty[xc], ((i / NXC) & 1u) ^ 1u, abort_flag)) break;
-                ptx::mbar_arrive_expect_tx(&x_full[xc], static_cast<uint32_t>(ng) * L::kXTile);
-                for (int q = 0; q < ng; ++q)
-                    ptx::tma_load_2d(smem + L::kOffX + xc * L::kXBytes + q * L::kXTile, &map_x, &x_full[xc], (g0 + q) * BK, 0);
-                ++xi;
-                if (ci < nchunks && !issue_codes()) break;     // codes run NC chunks ahead
             }
             // never leave the CTA with bulk copies still landing in its shared memory
             for (uint32_t j = (ci > static_cast<uint32_t>(NC) ? ci - NC : 0u); j < ci; ++j)
                 ptx::mbar_wait(&c_full[j % NC], (j / NC) & 1u, nullptr);
+        }
+    } else if (warp == kWarpTmaX) {
+        // ---------------------------------------------------------------- activation producer
+        if (lane == 0) {
+            ptx::grid_dependency_wait();              // the activations come from the prepass
+            uint32_t xi = 0;
+            ChunkPos cp = start;
+            for (; xi < nchunks; ++xi, advance(cp)) {
+                int w, g0, ng;
+                chunk_groups(cp, w, g0, ng);
+                const int xc = static_cast<int>(xi % NXC);
+                if (!ptx::mbar_wait(&x_empty[xc], ((xi / NXC) & 1u) ^ 1u, abort_flag)) break;
+                ptx::mbar_arrive_expect_tx(&x_full[xc], static_cast<uint32_t>(ng) * L::kXTile);
+                for (int q = 0; q < ng; ++q)
+                    ptx::tma_load_2d(smem + L::kOffX + xc * L::kXBytes + q * L::kXTile, &map_x, &x_full[xc], (g0 + q) * BK, 0);
+            }
             for (uint32_t j = (xi > static_cast<uint32_t>(NXC) ? xi - NXC : 0u); j < xi; ++j)
                 ptx::mbar_wait(&x_full[j % NXC], (j / NXC) & 1u, nullptr);
         }
