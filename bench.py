@@ -63,7 +63,7 @@ def peaks():
 def kernel_source_hash() -> str:
     import hashlib
     d = os.path.join(ROOT, "group_wise_affine_qlinear_b200", "csrc")
-    src = open(os.path.join(d, "ql_tc_fused.cuh"), "rb").read() + open(os.path.join(d, "ql_ptx.cuh"), "rb").read()
+    src = b"".join(open(os.path.join(d, f), "rb").read() for f in ("ql_tc_fused.cuh", "ql_ptx.cuh", "ql_dequant_f16.cuh"))
     return hashlib.sha256(src).hexdigest()[:12]
 
 
