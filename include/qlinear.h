@@ -68,10 +68,13 @@ typedef enum { QL_F32 = 0, QL_BF16 = 1 } ql_dtype;
 typedef enum {
     QL_PATH_AUTO = 0,       /* per-shape choice of the dispatcher */
     QL_PATH_GEMV = 1,       /* CUDA-core split-K weight streaming (any M; meant for M <= 4) */
-    QL_PATH_TC_SKINNY = 2,  /* tcgen05 weight streaming for small M: integer codes as bf16,
-                               per-group scale/bias applied to fp32 partials; M <= 32 */
-    QL_PATH_TC_FUSED = 3    /* tcgen05 fused-dequant GEMM for large M: fp16 operands,
-                               fp32 TMEM accumulators */
+    QL_PATH_TC_SKINNY = 2,  /* tcgen05 weight streaming for small M (M <= 32): stream-K over K,
+                               fp32 partials reduced in a fixed order */
+    QL_PATH_TC_FUSED = 3    /* tcgen05 fused-dequant GEMM for large M */
+    /* Both tcgen05 paths multiply f16 operands with fp32 accumulation in tensor memory: each
+     * weight is rounded once, RN_f16(s * q + b), and each activation row is scaled by a power of
+     * two into f16 (exact for entries above 2^-28 of the row's largest magnitude) and scaled back
+     * after the accumulation.  QL_PATH_GEMV multiplies the exact codes in fp32. */
 } ql_path;
 
 /*
