@@ -321,6 +321,9 @@ def pack_imatrix(w, imatrix, row_chunk: int = 256):
     Every visited triple is scored; the lowest E wins, ties to the lowest index.
     For fixed (s, b) the nearest code is optimal for any imp >= 0 because the
     objective is a sum of independent non-negative terms.
+    Every float64 sum (the imatrix mean, E and the least-squares moments of a
+    group) is taken one term at a time in index order, so a device fit that
+    follows the same steps with correctly rounded operations gives the same bytes.
     """
     w = np.asarray(w, dtype=np.float32)
     if imatrix is None:
@@ -328,7 +331,10 @@ def pack_imatrix(w, imatrix, row_chunk: int = 256):
     N, K = w.shape
     _check_packable(w)
     imp = np.asarray(imatrix, dtype=np.float64)
-    imp = imp + 1e-6 * imp.mean()
+    total = 0.0
+    for v in imp.tolist():                     # index order, one term at a time
+        total = total + v
+    imp = imp + 1e-6 * (total / imp.size)
     codes = np.empty((N, K // 8), dtype=np.uint32)
     scales = np.empty((N, K // GROUP), dtype=np.float16)
     biases = np.empty((N, K // GROUP), dtype=np.float16)
@@ -339,10 +345,18 @@ def pack_imatrix(w, imatrix, row_chunk: int = 256):
     return codes, scales, biases
 
 
+def _seq_sum(t):
+    """Sum over the last axis one term at a time in index order (float64)."""
+    acc = np.zeros(t.shape[:-1], dtype=np.float64)
+    for j in range(t.shape[-1]):
+        acc = acc + t[..., j]
+    return acc
+
+
 def _score(g64, imp_g, q, s16, b16):
     """Weighted error of the triple (q, s16, b16) per group; deq = RN32(s*q + b)."""
     deq = (s16.astype(np.float64)[..., None] * q + b16.astype(np.float64)[..., None]).astype(np.float32)
-    return np.sum(imp_g * (g64 - deq.astype(np.float64)) ** 2, axis=-1)
+    return _seq_sum(imp_g * (g64 - deq.astype(np.float64)) ** 2)
 
 
 def _fit_rows(w, imp):
@@ -369,8 +383,8 @@ def _fit_rows(w, imp):
     mn = g64.min(axis=-1)
     mx = g64.max(axis=-1)
     r = mx - mn
-    sw = imp_g.sum(axis=-1)                                 # sum imp
-    swx = (imp_g * g64).sum(axis=-1)                        # sum imp * w
+    sw = _seq_sum(imp_g)                                    # sum imp
+    swx = _seq_sum(imp_g * g64)                             # sum imp * w
     for a in FIT_SHRINK:
         for bb in FIT_SHRINK:
             if a == 0 and bb == 0:
@@ -384,9 +398,9 @@ def _fit_rows(w, imp):
             active = np.ones(s16.shape, dtype=bool)
             for _ in range(FIT_REFITS):
                 qf = q.astype(np.float64)
-                swq = (imp_g * qf).sum(axis=-1)
-                swqq = (imp_g * qf * qf).sum(axis=-1)
-                swqx = (imp_g * qf * g64).sum(axis=-1)
+                swq = _seq_sum(imp_g * qf)
+                swqq = _seq_sum(imp_g * qf * qf)
+                swqx = _seq_sum(imp_g * qf * g64)
                 det = swqq * sw - swq * swq
                 ok = active & (np.abs(det) > 1e-12 * np.maximum(swqq * sw, 1e-300))
                 with np.errstate(divide="ignore", invalid="ignore"):
