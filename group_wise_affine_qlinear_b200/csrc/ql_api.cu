@@ -14,6 +14,7 @@
 #include "ql_dequant.cuh"
 #include "ql_gemv.cuh"
 #include "ql_pack.cuh"
+#include "ql_pack_fit.cuh"
 #include "ql_prepass.cuh"
 #include "ql_tc_fused.cuh"
 #include "ql_tc_skinny.cuh"
@@ -487,7 +488,7 @@ ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t 
     ql_status s = check_shape(1, K, N, group);
     if (s != QL_OK) return s;
     if (!w || !codes || !scales || !biases) return QL_ERR_INVALID_ARG;
-    if (imatrix != nullptr) return QL_ERR_UNSUPPORTED;
+    if (N > 65535ll * kFitThreads || K / kGroup > 2147483647ll) return QL_ERR_UNSUPPORTED;   // fit grid limits
     if (!aligned16(w) || !aligned16(codes) || !aligned16(scales) || !aligned16(biases)) return QL_ERR_ALIGNMENT;
     const int64_t G = K / kGroup;
     const size_t wb = static_cast<size_t>(N) * K * 4, cb = static_cast<size_t>(N) * K / 2,
@@ -495,6 +496,16 @@ ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t 
     if (overlap(w, wb, codes, cb) || overlap(w, wb, scales, pb) || overlap(w, wb, biases, pb) ||
         overlap(codes, cb, scales, pb) || overlap(codes, cb, biases, pb) || overlap(scales, pb, biases, pb))
         return QL_ERR_INVALID_ARG;
+    if (imatrix != nullptr) {
+        const size_t ib = static_cast<size_t>(K) * 4;
+        if (overlap(imatrix, ib, codes, cb) || overlap(imatrix, ib, scales, pb) || overlap(imatrix, ib, biases, pb))
+            return QL_ERR_INVALID_ARG;
+        const dim3 grid(static_cast<unsigned>(K / kGroup), static_cast<unsigned>((N + kFitThreads - 1) / kFitThreads));
+        pack_fit_kernel<<<grid, kFitThreads, 0, stream>>>(w, imatrix, codes, static_cast<__half*>(scales),
+                                                          static_cast<__half*>(biases), static_cast<int>(K),
+                                                          static_cast<int>(N));
+        return launch_status();
+    }
     DeviceInfo* dev = nullptr;
     if ((s = device_info(&dev)) != QL_OK) return s;
     const int64_t groups = N * G;

@@ -132,7 +132,17 @@ QL_API ql_status qlinear_dequant(const uint32_t* codes, const void* scales, cons
  * bias = RN_f16(min), q = clamp(rint(RN32(RN32(w-bias)/scale)), 0, 15)
  * (ties to even), q = 0 when scale == 0.  Deterministic: equal inputs give
  * equal bytes.
- * imatrix != NULL (importance-weighted fit): QL_ERR_UNSUPPORTED in this build.
+ * imatrix != NULL: importance-weighted fit.  imatrix is fp32 [K], the per-channel
+ * E[x^2] of the layer's activations (device memory, read only).  Per group the
+ * candidates are the RTN triple, then 80 range shrinks (lo = min + a r,
+ * hi = max - c r, a, c in {0, 0.025, ..., 0.2}), each refined by up to two
+ * weighted least-squares refits of (scale, bias) with the codes fixed; the
+ * triple with the lowest sum_j imp_j (w_j - RN32(s q_j + b))^2 (float64,
+ * imp = imatrix + 1e-6 * mean(imatrix)) wins, ties to the earliest, so the fit
+ * is never worse than RTN on that objective.  Deterministic: every float64 sum
+ * is taken in index order with correctly rounded operations.  A negative or
+ * non-finite imatrix entry is an argument error reported through the device
+ * status word (all groups written as zeros).
  * A group holding a non-finite value or |w| > 65504 is written as codes 0,
  * scale 0, bias 0, and the device status word records QL_ERR_INVALID_ARG.
  */

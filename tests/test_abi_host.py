@@ -94,7 +94,8 @@ def test_dequant_and_pack_validation(L):
     assert L.qlinear_dequant(FAKE, FAKE + (1 << 24), FAKE + (2 << 24), 256, 256, 32, FAKE + (3 << 24), 0, None) == 3
     assert L.qlinear_dequant(FAKE, FAKE + (1 << 24), FAKE + (2 << 24), 256, 256, 64, FAKE, 0, None) == 1
     assert L.qlinear_dequant(FAKE + 8, FAKE + (1 << 24), FAKE + (2 << 24), 256, 256, 64, FAKE + (3 << 24), 0, None) == 2
-    assert L.qlinear_pack(FAKE, FAKE, 256, 256, 64, FAKE + (1 << 24), FAKE + (2 << 24), FAKE + (3 << 24), None) == 3
+    # an importance vector overlapping an output is rejected before any launch
+    assert L.qlinear_pack(FAKE, FAKE + (1 << 24), 256, 256, 64, FAKE + (1 << 24), FAKE + (2 << 24), FAKE + (3 << 24), None) == 1
     assert L.qlinear_pack(FAKE, None, 256, 256, 64, FAKE, FAKE + (2 << 24), FAKE + (3 << 24), None) == 1
 
 

@@ -122,11 +122,51 @@ def test_pack_nonfinite_reports_status():
         O.pack_rtn(w)
 
 
-def test_pack_imatrix_unsupported():
-    w = torch.zeros((8, 64), dtype=torch.float32, device="cuda")
-    with pytest.raises(ql.QLinearError) as e:
-        ql.pack(w, imatrix=torch.ones(64, dtype=torch.float32, device="cuda"))
-    assert e.value.status == 3
+def _fit_case():
+    """64 dense rows of N(0, 0.02^2) weights (the fitted MLP rows' recipe) with special groups, and the
+    E[x^2] of 512 synthetic activation rows, rounded to fp32, with some channels never reached."""
+    K = 4608
+    w = S.dense_weight(2, 0, 64, K, 0.02)
+    w[0, :64] = 0.0125                                   # constant group
+    w[1, 64:128] = 0.0
+    w[2, :64] *= 0.01
+    w[2, 7] = 0.3                                        # one outlier dominates the range
+    w[3, :64] = (np.arange(64) % 16).astype(np.float32) * np.float32(0.002) - np.float32(0.01)   # on a grid
+    imp = O.imatrix_from_x(S.activations(2, 0, 512, K)).astype(np.float32)
+    imp[100:164] = 0.0                                   # channels no activation reached
+    imp[4000] = 0.0
+    return w, imp
+
+
+def test_pack_imatrix_bitexact():
+    w, imp = _fit_case()
+    c, s, b = ql.pack(torch.from_numpy(w).cuda(), imatrix=torch.from_numpy(imp).cuda())
+    rc, rs, rb = O.pack_imatrix(w, imp.astype(np.float64))
+    assert ql.device_status() == 0
+    assert np.array_equal(c.cpu().numpy().view(np.uint32), rc)
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), rs.view(np.uint16))
+    assert np.array_equal(b.cpu().numpy().view(np.uint16), rb.view(np.uint16))
+
+
+def test_pack_imatrix_never_worse_than_rtn():
+    """The pages' guarantee, checked on the device result against the oracle's objective."""
+    w, imp = _fit_case()
+    c, s, b = ql.pack(torch.from_numpy(w).cuda(), imatrix=torch.from_numpy(imp).cuda())
+    imp64 = imp.astype(np.float64)
+    imp64 = imp64 + 1e-6 * imp64.mean()
+    e_fit = O.group_weighted_error(w, c.cpu().numpy().view(np.uint32), s.cpu().numpy(), b.cpu().numpy(), imp64)
+    e_rtn = O.group_weighted_error(w, *O.pack_rtn(w), imp64)
+    assert np.all(e_fit <= e_rtn * (1 + 1e-12))
+    assert e_fit.sum() < e_rtn.sum()
+
+
+def test_pack_imatrix_rejects_bad_importance():
+    w = S.dense_weight(2, 1, 8, 128, 0.02)
+    imp = np.ones(128, dtype=np.float32)
+    imp[5] = -1.0
+    c, s, b = ql.pack(torch.from_numpy(w).cuda(), imatrix=torch.from_numpy(imp).cuda())
+    assert ql.device_status() == 1          # QL_ERR_INVALID_ARG
+    assert not c.cpu().numpy().any() and not s.cpu().numpy().view(np.uint16).any()
 
 
 # ------------------------------------------------------------------ forward: small and ragged
