@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--path", type=int, default=0, help="force a kernel path (0 = dispatcher's choice)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-m", action="store_true", help="skip the small-M weight-streaming measurements")
+    ap.add_argument("--no-pack", action="store_true", help="skip the quantizer (qlinear_pack) measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     return ap.parse_args()
 
@@ -78,6 +79,60 @@ def recorded_traffic(path: str, key: str):
         if len(f) == 4 and f[0] == path and f[1] == key and f[2] == h:
             return int(f[3])
     return None
+
+
+# ---------------------------------------------------------------------------- quantizer timing
+
+PACK_ROWS, PACK_K = 4608, 4608
+
+
+def pack_inputs():
+    """DiT-shaped dense weight N(0, 0.02^2) and E[x^2] of 512 synthetic activation rows (fp32)."""
+    w = S.dense_weight(2, 0, PACK_ROWS, PACK_K, 0.02)
+    xb = S.activations(2, 0, 512, PACK_K)
+    xf = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return w, (xf * xf).mean(axis=0).astype(np.float32)
+
+
+def pack_measure(ql, torch, dev, flush, runs=3):
+    """Device time of qlinear_pack on a 4608 x 4608 weight: importance-weighted fit and RTN."""
+    w, imp = pack_inputs()
+    wd = torch.from_numpy(w).to(dev)
+    impd = torch.from_numpy(imp).to(dev)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        ms = []
+        for i in range(runs):
+            flush.fill_(i & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        return sum(ms) / runs
+
+    fit_ms = timed(lambda: ql.pack(wd, imatrix=impd))
+    rtn_ms = timed(lambda: ql.pack(wd))
+    assert ql.device_status() == 0, "qlinear_pack reported an error"
+    groups = PACK_ROWS * PACK_K // 64
+    rtn_bytes = PACK_ROWS * PACK_K * 4 + PACK_ROWS * PACK_K // 2 + groups * 4
+    return {"workload": f"dense N(0, 0.02^2) {PACK_ROWS} x {PACK_K}, imatrix = E[x^2] of 512 synthetic rows",
+            "groups": groups, "fit_ms": fit_ms, "fit_groups_per_s": groups / (fit_ms * 1e-3),
+            "rtn_ms": rtn_ms, "rtn_GBps": rtn_bytes / (rtn_ms * 1e-3) / 1e9}
+
+
+def oracle_fit_rate(rows=4):
+    """CPU oracle's importance-weighted fit on the first rows of the same weight: groups per second."""
+    from oracle import qlinear_oracle as O
+    w, imp = pack_inputs()
+    t0 = time.perf_counter()
+    O.pack_imatrix(w[:rows], imp.astype(np.float64))
+    dt = time.perf_counter() - t0
+    return rows * PACK_K // 64 / dt, f"{rows} rows of the same weight in {dt:.1f} s"
 
 
 # ---------------------------------------------------------------------------- CPU oracle timing
@@ -342,6 +397,9 @@ def main():
             del c
         torch.cuda.synchronize()
 
+    # ---- the quantizer: importance-weighted fit and RTN pack of a DiT-shaped weight
+    pack = None if a.no_pack else pack_measure(ql, torch, dev, flush)
+
     mean_step, mean_main, mean_e2e = max_over_ranks([mean_step, mean_main, mean_e2e], dev)
 
     flops = 2.0 * M * K * N
@@ -380,11 +438,15 @@ def main():
         "clocks": clk,
         "small_m": small,
     }
+    if pack is not None:
+        line["pack"] = pack
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         rate, cores, rows, dt = oracle_rate(w, M, a.cpu_seconds, case.x_np[: min(M, 512)],
                                             (case.codes_np, case.s_np, case.b_np))
         line["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                 "sample": f"{rows} rows x full K x full N of {w.name} in {dt:.1f} s"}
+        if pack is not None:
+            pack["oracle_fit_groups_per_s"], pack["oracle_fit_sample"] = oracle_fit_rate()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg:
