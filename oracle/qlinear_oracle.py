@@ -41,6 +41,13 @@ notes of the repository):
   R5 tolerance: bf16 output is gated on relative Frobenius error <= 4e-3 and
      on max_i(|y_i - y_ref_i| - half_ulp_bf16(max(|y_i|, |y_ref_i|)))^+ <=
      1.5e-2 * rms(y_ref); the literal max error is reported beside it.
+  R9 W8 g64, the 8-bit width the pages keep for the modulation and
+     conditioning projections (aimarketly "Ideogram-4-IQ4_M", Conversion) and
+     ship as a Q8 pack (huggingface "SceneWorks/ideogram-4-mlx", Versions):
+     codes are uint32 [N][K/4] with code (n, k) = (codes[n][k/4] >> 8*(k%4)) &
+     0xFF (low byte first), q in [0, 255]; scales and biases as in R1, so a
+     weight costs 8 + 0.5 bits (the same "+0.5" overhead); RTN as R3 with 255
+     levels in place of 15.
 
 Parity status: the imatrix fit (pack_imatrix) is a search heuristic with no
 printed reference values; only its invariants are pinned ("never worse than
@@ -424,3 +431,85 @@ def _fit_rows(w, imp):
                 best_b = np.where(better, b16, best_b)
                 best_q = np.where(better[..., None], q, best_q)
     return pack_codes(best_q.reshape(n, K)), best_s.astype(np.float16), best_b.astype(np.float16)
+
+
+# --------------------------------------------------------------------------
+# W8 g64 (R9): 8-bit codes with the same per-64 f16 scale and bias
+# --------------------------------------------------------------------------
+
+def unpack_codes8(codes, K: int) -> np.ndarray:
+    """uint32 [N][K/4] -> int64 codes q [N][K], code k%4 in bits 8*(k%4) .. 8*(k%4)+7."""
+    c = np.asarray(codes, dtype=np.uint32).astype(np.int64)
+    N = c.shape[0]
+    assert c.shape[1] * 4 == K
+    shifts = 8 * np.arange(4, dtype=np.int64)
+    q = (c[:, :, None] >> shifts[None, None, :]) & 0xFF
+    return q.reshape(N, K)
+
+
+def pack_codes8(q) -> np.ndarray:
+    """int codes [N][K] in [0, 255] -> uint32 [N][K/4], low byte first."""
+    q = np.asarray(q, dtype=np.uint64)
+    N, K = q.shape
+    assert K % 4 == 0 and q.max(initial=0) <= 255
+    shifts = 8 * np.arange(4, dtype=np.uint64)
+    words = (q.reshape(N, K // 4, 4) << shifts[None, None, :]).sum(axis=-1)
+    return words.astype(np.uint32)
+
+
+def dequant8_exact(codes, scales, biases) -> np.ndarray:
+    """Exact w = s*q + b as float64 [N][K] for 8-bit codes.
+
+    s and b are integer multiples of 2^-24 below 2^16 and q <= 255, so
+    s*q + b = i * 2^-24 with |i| < 2^49: float64 holds it without rounding.
+    """
+    N, G = np.shape(scales)
+    K = G * GROUP
+    q = unpack_codes8(codes, K).astype(np.float64)
+    s = np.repeat(decode_f16(f16_array_bits(scales)), GROUP, axis=1)
+    b = np.repeat(decode_f16(f16_array_bits(biases)), GROUP, axis=1)
+    return s * q + b
+
+
+def dequant8_f32(codes, scales, biases) -> np.ndarray:
+    """fp32 dequant of 8-bit codes: RN_fp32 of the exact value (R2)."""
+    return dequant8_exact(codes, scales, biases).astype(np.float32)
+
+
+def dequant8_bf16(codes, scales, biases) -> np.ndarray:
+    """bf16 dequant of 8-bit codes = RN_bf16(fp32 dequant) as uint16 bits."""
+    return round_bf16(dequant8_f32(codes, scales, biases).astype(np.float64))
+
+
+def forward8_ref(x_bits, codes, scales, biases) -> np.ndarray:
+    """y_ref[m][n] = sum_k x[m][k] * w(n, k) in float64, w the fp32 dequant of 8-bit codes."""
+    x = decode_bf16(x_bits)
+    w = dequant8_f32(codes, scales, biases).astype(np.float64)
+    return x @ w.T
+
+
+def nearest_codes8(w32, scale16, bias16) -> np.ndarray:
+    """q = clamp(round_half_even(RN32(RN32(w - b) / s)), 0, 255) per group; 0 where s == 0."""
+    s = scale16.astype(np.float32)[..., None]
+    b = bias16.astype(np.float32)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (w32 - b) / np.where(s == 0, np.float32(1), s)      # float32 subtract and divide
+    q = np.clip(np.rint(t), 0, 255)
+    q = np.where(s == 0, 0, q)
+    return q.astype(np.int64)
+
+
+def pack8_rtn(w):
+    """Min/max round-to-nearest quantization of float32 W [N][K] to 8-bit codes (R9)."""
+    w = np.asarray(w, dtype=np.float32)
+    N, K = w.shape
+    assert K % GROUP == 0
+    _check_packable(w)
+    g = w.reshape(N, K // GROUP, GROUP)
+    mn = g.min(axis=-1)
+    mx = g.max(axis=-1)
+    s32 = (mx - mn) / np.float32(255.0)                           # float32: RN32(RN32(mx - mn) / 255)
+    scale16 = s32.astype(np.float16)
+    bias16 = mn.astype(np.float16)
+    q = nearest_codes8(g, scale16, bias16)
+    return pack_codes8(q.reshape(N, K)), scale16, bias16

@@ -408,3 +408,172 @@ def test_fit_on_grid_group_has_zero_error():
 def test_imatrix_is_mean_square():
     x = np.array([[0x3F80, 0x4000], [0xBF80, 0x0000]], dtype=np.uint16)   # [[1, 2], [-1, 0]]
     assert np.array_equal(O.imatrix_from_x(x), np.array([1.0, 2.0]))
+
+
+# ---------------------------------------------------------------- W8 g64 (reading R9)
+
+def _w8_layer(rng, M, K, N):
+    codes = rng.integers(0, 1 << 32, size=(N, K // 4), dtype=np.uint32)
+    s = np.exp(rng.uniform(np.log(1e-4), np.log(2e-3), size=(N, K // 64))).astype(np.float16)
+    b = (-127.5 * s.astype(np.float64) + 0.1 * s.astype(np.float64) * rng.standard_normal(s.shape)).astype(np.float16)
+    x = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(torch.bfloat16)
+    return x.view(torch.int16).numpy().view(np.uint16), codes, s, b
+
+
+def test_w8_byte_order_low_first():
+    assert list(O.unpack_codes8(np.array([[0x04030201]], dtype=np.uint32), 4)[0]) == [1, 2, 3, 4]
+    assert O.pack_codes8(np.array([[1, 2, 3, 4]]))[0, 0] == 0x04030201
+
+
+def test_w8_pack_unpack_roundtrip():
+    q = _rng(40).integers(0, 256, size=(5, 192))
+    assert np.array_equal(O.unpack_codes8(O.pack_codes8(q), 192), q)
+
+
+def test_w8_bits_per_weight_is_8_5_golden():
+    """8-bit codes plus the pages' '+0.5' group overhead (one f16 scale and bias per 64)."""
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "format_constants.json")))
+    K = 4608
+    w = np.zeros((1, K), dtype=np.float32)
+    codes, s, b = O.pack8_rtn(w)
+    bits = 8 * (codes.nbytes + s.nbytes + b.nbytes)
+    assert bits == (g["q8_code_bits"]["value"] + g["overhead_bits_per_weight"]["value"]) * K
+
+
+def test_w8_dequant_exact_equals_rational_arithmetic():
+    """All 256 codes x edge f16 values as scale and as bias."""
+    edges = np.array([0.0, -0.0, 2.0 ** -24, 6.1e-5, 1.0, -1.0, 0.0078125, 3.140625, 65504.0, -65504.0,
+                      1e-3, -7.5e-3, 2.0 ** -14, 0.5, -2.0, 1024.0], dtype=np.float16)
+    q = np.arange(256)
+    for sv in edges:
+        for bv in edges:
+            for part in range(4):
+                qq = q[64 * part: 64 * part + 64]
+                codes = O.pack_codes8(qq[None, :])
+                got = O.dequant8_exact(codes, np.array([[sv]]), np.array([[bv]]))[0]
+                for j in range(64):
+                    exact = Fraction(float(sv)) * int(qq[j]) + Fraction(float(bv))
+                    assert Fraction(float(got[j])) == exact
+
+
+def test_w8_dequant_f32_is_correctly_rounded():
+    rng = _rng(41)
+    _, codes, s, b = _w8_layer(rng, 1, 256, 48)
+    w32 = O.dequant8_f32(codes, s, b)
+    q = O.unpack_codes8(codes, 256)
+    for n in range(0, 48, 5):
+        for k in range(0, 256, 7):
+            exact = Fraction(float(s[n, k // 64])) * int(q[n, k]) + Fraction(float(b[n, k // 64]))
+            got = Fraction(float(w32[n, k]))
+            lo = Fraction(float(np.nextafter(w32[n, k], np.float32(-np.inf))))
+            hi = Fraction(float(np.nextafter(w32[n, k], np.float32(np.inf))))
+            assert abs(got - exact) <= abs(lo - exact) and abs(got - exact) <= abs(hi - exact)
+
+
+def test_w8_dequant_bf16_is_bf16_of_f32_dequant():
+    _, codes, s, b = _w8_layer(_rng(42), 1, 128, 16)
+    w32 = O.dequant8_f32(codes, s, b)
+    lib = torch.from_numpy(w32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.dequant8_bf16(codes, s, b), lib)
+
+
+@pytest.mark.parametrize("M,K,N", [(3, 64, 5), (2, 192, 7)])
+def test_w8_forward_equals_triple_loop(M, K, N):
+    """Pure-Python triple loop with exactly rounded sums (math.fsum) against the float64 matrix product."""
+    import math
+    x, codes, s, b = _w8_layer(_rng(43 + M + K + N), M, K, N)
+    y = O.forward8_ref(x, codes, s, b)
+    xf = O.decode_bf16(x)
+    q = O.unpack_codes8(codes, K)
+    for m in range(M):
+        for n in range(N):
+            terms = []
+            for k in range(K):
+                wv = float(np.float32(float(s[n, k // 64]) * int(q[n, k]) + float(b[n, k // 64])))
+                terms.append(float(xf[m, k]) * wv)
+            ref = math.fsum(terms)
+            bound = 1e-14 * math.fsum(abs(t) for t in terms) + 1e-300
+            assert abs(y[m, n] - ref) <= bound
+
+
+def _w8_rtn_case(seed, N=16, K=256):
+    rng = _rng(seed)
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    w[0, :64] *= 100.0
+    w[1, 64:128] = np.abs(w[1, 64:128]) + 1.0
+    return w
+
+
+def test_w8_rtn_codes_are_nearest_grid_point():
+    """Brute force over the 256 grid points: each RTN code is (one of) the nearest."""
+    w = _w8_rtn_case(44)
+    codes, s, b = O.pack8_rtn(w)
+    N, K = w.shape
+    q = O.unpack_codes8(codes, K)
+    sf = s.astype(np.float64)
+    bf = b.astype(np.float64)
+    for n in range(N):
+        for k in range(K):
+            g = k // 64
+            grid = sf[n, g] * np.arange(256) + bf[n, g]
+            d = np.abs(grid - float(w[n, k]))
+            assert d[q[n, k]] <= d.min() + 4e-7 * max(abs(float(w[n, k])), 1e-3)
+
+
+def test_w8_rtn_reconstructs_group_extremes():
+    """R9 bounds: deq(code of min) within half an f16 ulp of min; max within 255*ulp(s)/2 + ulp(min)/2."""
+    w = _w8_rtn_case(45, N=24, K=512)
+    codes, s, b = O.pack8_rtn(w)
+    deq = O.dequant8_f32(codes, s, b).astype(np.float64).reshape(24, 8, 64)
+    g = w.astype(np.float64).reshape(24, 8, 64)
+
+    def half_ulp_f16(v):
+        _, e = np.frexp(np.abs(v))
+        return np.ldexp(1.0, np.maximum(e, -13) - 12)
+
+    i_min, i_max = g.argmin(-1), g.argmax(-1)
+    mn = np.take_along_axis(g, i_min[..., None], -1)[..., 0]
+    mx = np.take_along_axis(g, i_max[..., None], -1)[..., 0]
+    d_min = np.take_along_axis(deq, i_min[..., None], -1)[..., 0]
+    d_max = np.take_along_axis(deq, i_max[..., None], -1)[..., 0]
+    eps = 2.0 ** -23 * np.maximum(np.abs(mn), np.abs(mx))
+    assert np.all(np.abs(d_min - mn) <= half_ulp_f16(mn) + eps)
+    assert np.all(np.abs(d_max - mx) <= 255 * half_ulp_f16(s.astype(np.float64)) + half_ulp_f16(mn) + eps)
+
+
+def test_w8_rtn_constant_group_and_monotone_codes():
+    w = np.full((2, 128), -0.7, dtype=np.float32)
+    codes, s, b = O.pack8_rtn(w)
+    assert np.all(O.unpack_codes8(codes, 128) == 0) and np.all(s == 0)
+    w = _w8_rtn_case(46, N=6, K=128)
+    q = O.unpack_codes8(O.pack8_rtn(w)[0], 128).reshape(6, 2, 64)
+    g = w.reshape(6, 2, 64)
+    for n in range(6):
+        for j in range(2):
+            order = np.argsort(g[n, j], kind="stable")
+            assert np.all(np.diff(q[n, j][order]) >= 0)
+
+
+def test_w8_rtn_on_grid_group_is_exact():
+    """A group on an f16 affine grid that uses codes 0 and 255 is reproduced exactly."""
+    s = np.float16(2.0 ** -10)
+    b = np.float16(-0.125)
+    q = np.concatenate([[0, 255], np.arange(1, 255, 4)[:62]])
+    w = (np.float64(s) * q + np.float64(b)).astype(np.float32)[None, :]
+    codes, s2, b2 = O.pack8_rtn(w)
+    assert s2[0, 0] == s and b2[0, 0] == b
+    assert np.array_equal(O.unpack_codes8(codes, 64)[0], q)
+
+
+def test_w8_and_w4_agree_on_a_shared_grid():
+    """Weights whose 64-groups use only the 16 levels b + 17 s' q (q <= 15) of an 8-bit grid with step
+    s' = s/17: the W4 and W8 packs dequantize to the same values."""
+    s4 = np.float16(0.0078125 * 1.0625 * 17)           # 17 * s8, exact in f16
+    s8 = np.float16(np.float64(s4) / 17)
+    assert np.float64(s8) * 17 == np.float64(s4)
+    b = np.float16(-0.0625)
+    q4 = np.tile(np.arange(16), 4)
+    w = (np.float64(s4) * q4 + np.float64(b)).astype(np.float32)[None, :]
+    d4 = O.dequant_f32(*O.pack_rtn(w))
+    d8 = O.dequant8_f32(*O.pack8_rtn(w))
+    assert np.array_equal(d4, d8)
