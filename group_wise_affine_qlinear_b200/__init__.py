@@ -12,6 +12,9 @@ Tensors follow the ABI layout:
     scales  torch.float16  [N][K/64]
     biases  torch.float16  [N][K/64]
     y       torch.bfloat16 [M][N]     (y = x . W^T, W[n][k] = scale * code + bias)
+The 8-bit variant (forward8, dequant8, pack8, workspace_size8) takes codes as
+torch.int32 [N][K/4] (4 codes per word, low byte first) with the same scales
+and biases.
 """
 from __future__ import annotations
 
@@ -24,14 +27,18 @@ from ._lib import (  # noqa: F401
     QLinearError,
     STATUS,
     dequant,
+    dequant8,
     device_status,
     forward,
+    forward8,
     forward_noalloc,
     last_dispatch,
     lib,
     library_path,
     pack,
+    pack8,
     set_profile_events,
     version,
     workspace_size,
+    workspace_size8,
 )

@@ -73,6 +73,19 @@ def lib() -> ctypes.CDLL:
         L.qlinear_status_string.restype = ctypes.c_char_p
         L.qlinear_version.argtypes = []
         L.qlinear_version.restype = ctypes.c_int32
+        L.qlinear8_workspace_size.argtypes = [i64, i64, i64, i32]
+        L.qlinear8_workspace_size.restype = sz
+        L.qlinear8_workspace_size_config.argtypes = [i64, i64, i64, i32, i32, i32]
+        L.qlinear8_workspace_size_config.restype = sz
+        L.qlinear8_forward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, sz, vp]
+        L.qlinear8_forward.restype = ctypes.c_int
+        L.qlinear8_forward_config.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i32, i32, i32, vp, sz,
+                                              vp]
+        L.qlinear8_forward_config.restype = ctypes.c_int
+        L.qlinear8_dequant.argtypes = [vp, vp, vp, i64, i64, i32, vp, ctypes.c_int, vp]
+        L.qlinear8_dequant.restype = ctypes.c_int
+        L.qlinear8_pack.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp, vp]
+        L.qlinear8_pack.restype = ctypes.c_int
         _lib = L
         return L
 
@@ -98,28 +111,45 @@ def _need_cuda(t: torch.Tensor, name: str, dtype, shape=None) -> None:
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
-def _weights_shape(codes: torch.Tensor, scales: torch.Tensor):
+def _weights_shape(codes: torch.Tensor, scales: torch.Tensor, bits: int = 4):
     N, Kw = codes.shape
-    K = 8 * Kw
+    K = (32 // bits) * Kw
     return N, K
 
 
-def workspace_size(M: int, K: int, N: int, path: int = PATH_AUTO, split_k: int = 0) -> int:
-    v = lib().qlinear_workspace_size_config(M, K, N, GROUP, path, split_k)
+def workspace_size(M: int, K: int, N: int, path: int = PATH_AUTO, split_k: int = 0, bits: int = 4) -> int:
+    fn = lib().qlinear_workspace_size_config if bits == 4 else lib().qlinear8_workspace_size_config
+    v = fn(M, K, N, GROUP, path, split_k)
     if v == ctypes.c_size_t(-1).value:
         raise ValueError("shape or path not supported")
     return int(v)
+
+
+def workspace_size8(M: int, K: int, N: int, path: int = PATH_AUTO, split_k: int = 0) -> int:
+    """Workspace bytes of forward8 (qlinear8_workspace_size_config)."""
+    return workspace_size(M, K, N, path, split_k, bits=8)
 
 
 def forward(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
             out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
             path: int = PATH_AUTO, split_k: int = 0, out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
     """y = x . W^T for the packed W; see include/qlinear.h (qlinear_forward[_config])."""
+    return _forward(x, codes, scales, biases, out, workspace, path, split_k, out_dtype, stream, 4)
+
+
+def forward8(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+             out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+             path: int = PATH_AUTO, split_k: int = 0, out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+    """forward() for 8-bit codes, int32 [N][K/4] (qlinear8_forward[_config])."""
+    return _forward(x, codes, scales, biases, out, workspace, path, split_k, out_dtype, stream, 8)
+
+
+def _forward(x, codes, scales, biases, out, workspace, path, split_k, out_dtype, stream, bits):
     L = lib()
-    N, K = _weights_shape(codes, scales)
+    N, K = _weights_shape(codes, scales, bits)
     M = x.shape[0]
     _need_cuda(x, "x", torch.bfloat16, (M, K))
-    _need_cuda(codes, "codes", torch.int32, (N, K // 8))
+    _need_cuda(codes, "codes", torch.int32, (N, K * bits // 32))
     _need_cuda(scales, "scales", torch.float16, (N, K // GROUP))
     _need_cuda(biases, "biases", torch.float16, (N, K // GROUP))
     if out_dtype not in (torch.bfloat16, torch.float32):
@@ -127,20 +157,21 @@ def forward(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, biases: 
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
     _need_cuda(out, "out", out_dtype, (M, N))
-    need = workspace_size(M, K, N, path, split_k)
+    need = workspace_size(M, K, N, path, split_k, bits)
     if need > 0 and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = _stream_handle(stream)
+    name = "qlinear_forward" if bits == 4 else "qlinear8_forward"
     if path == PATH_AUTO and split_k == 0 and out_dtype == torch.bfloat16:
-        s = L.qlinear_forward(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), biases.data_ptr(), out.data_ptr(),
-                              M, K, N, GROUP, ws_ptr, ws_bytes, st)
+        s = getattr(L, name)(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), biases.data_ptr(), out.data_ptr(),
+                             M, K, N, GROUP, ws_ptr, ws_bytes, st)
     else:
-        s = L.qlinear_forward_config(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), biases.data_ptr(),
-                                     out.data_ptr(), _BF16 if out_dtype == torch.bfloat16 else _F32,
-                                     M, K, N, GROUP, path, split_k, ws_ptr, ws_bytes, st)
-    _check(s, "qlinear_forward")
+        s = getattr(L, name + "_config")(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), biases.data_ptr(),
+                                         out.data_ptr(), _BF16 if out_dtype == torch.bfloat16 else _F32,
+                                         M, K, N, GROUP, path, split_k, ws_ptr, ws_bytes, st)
+    _check(s, name)
     return out
 
 
@@ -165,34 +196,55 @@ def forward_noalloc(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, 
 def dequant(codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor, out_dtype=torch.float32,
             out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """W[n][k] = RN_fp32(scale * q + bias) (optionally rounded again to bf16)."""
+    return _dequant(codes, scales, biases, out_dtype, out, stream, 4)
+
+
+def dequant8(codes: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor, out_dtype=torch.float32,
+             out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """dequant() for 8-bit codes, int32 [N][K/4] (qlinear8_dequant)."""
+    return _dequant(codes, scales, biases, out_dtype, out, stream, 8)
+
+
+def _dequant(codes, scales, biases, out_dtype, out, stream, bits):
     L = lib()
-    N, K = _weights_shape(codes, scales)
-    _need_cuda(codes, "codes", torch.int32, (N, K // 8))
+    N, K = _weights_shape(codes, scales, bits)
+    _need_cuda(codes, "codes", torch.int32, (N, K * bits // 32))
     _need_cuda(scales, "scales", torch.float16, (N, K // GROUP))
     _need_cuda(biases, "biases", torch.float16, (N, K // GROUP))
     if out is None:
         out = torch.empty((N, K), dtype=out_dtype, device=codes.device)
     _need_cuda(out, "out", out_dtype, (N, K))
     dt = {torch.float32: _F32, torch.bfloat16: _BF16}[out_dtype]
-    _check(L.qlinear_dequant(codes.data_ptr(), scales.data_ptr(), biases.data_ptr(), K, N, GROUP, out.data_ptr(), dt,
-                             _stream_handle(stream)), "qlinear_dequant")
+    name = "qlinear_dequant" if bits == 4 else "qlinear8_dequant"
+    _check(getattr(L, name)(codes.data_ptr(), scales.data_ptr(), biases.data_ptr(), K, N, GROUP, out.data_ptr(), dt,
+                            _stream_handle(stream)), name)
     return out
 
 
 def pack(w: torch.Tensor, imatrix: torch.Tensor | None = None, stream=None):
-    """Min/max round-to-nearest quantization of fp32 W [N][K] -> (codes, scales, biases)."""
+    """Quantize fp32 W [N][K] -> (codes, scales, biases): round-to-nearest, or the imatrix-weighted fit."""
+    return _pack(w, imatrix, stream, 4)
+
+
+def pack8(w: torch.Tensor, stream=None):
+    """Round-to-nearest quantization of fp32 W [N][K] to 8-bit codes, int32 [N][K/4] (qlinear8_pack)."""
+    return _pack(w, None, stream, 8)
+
+
+def _pack(w, imatrix, stream, bits):
     L = lib()
     N, K = w.shape
     _need_cuda(w, "w", torch.float32, (N, K))
-    codes = torch.empty((N, K // 8), dtype=torch.int32, device=w.device)
+    codes = torch.empty((N, K * bits // 32), dtype=torch.int32, device=w.device)
     scales = torch.empty((N, K // GROUP), dtype=torch.float16, device=w.device)
     biases = torch.empty((N, K // GROUP), dtype=torch.float16, device=w.device)
     imp = None
     if imatrix is not None:
         _need_cuda(imatrix, "imatrix", torch.float32, (K,))
         imp = imatrix.data_ptr()
-    _check(L.qlinear_pack(w.data_ptr(), imp, K, N, GROUP, codes.data_ptr(), scales.data_ptr(), biases.data_ptr(),
-                          _stream_handle(stream)), "qlinear_pack")
+    name = "qlinear_pack" if bits == 4 else "qlinear8_pack"
+    _check(getattr(L, name)(w.data_ptr(), imp, K, N, GROUP, codes.data_ptr(), scales.data_ptr(), biases.data_ptr(),
+                            _stream_handle(stream)), name)
     return codes, scales, biases
 
 

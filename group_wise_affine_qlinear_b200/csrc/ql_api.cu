@@ -49,6 +49,21 @@ struct DeviceInfo {
     bool fused_attr_set = false;
     bool skinny_attr_set = false;
 };
+
+template <int NT, int B>
+cudaError_t skinny_smem_attr() {
+    return cudaFuncSetAttribute(skinny::skinny_kernel<NT, B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                skinny::Layout<NT, B>::kSmemBytes);
+}
+
+template <class FC>
+cudaError_t fused_smem_attr() {
+    const cudaError_t e = cudaFuncSetAttribute(fused::fused_gemm_kernel<true, FC>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, FC::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(fused::fused_gemm_kernel<false, FC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                FC::kSmemBytes);
+}
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
@@ -63,22 +78,14 @@ ql_status device_info(DeviceInfo** out) {
         d.sm_count = n;
     }
     if (!d.fused_attr_set) {
-        using FC = fused::DefaultCfg;
-        if (cudaFuncSetAttribute(fused::fused_gemm_kernel<true, FC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 FC::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(fused::fused_gemm_kernel<false, FC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 FC::kSmemBytes) != cudaSuccess) {
+        if (fused_smem_attr<fused::DefaultCfg>() != cudaSuccess || fused_smem_attr<fused::Q8Cfg>() != cudaSuccess)
             return QL_ERR_CUDA;
-        }
         d.fused_attr_set = true;
     }
     if (!d.skinny_attr_set) {
-        if (cudaFuncSetAttribute(skinny::skinny_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 skinny::Layout<16>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(skinny::skinny_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 skinny::Layout<32>::kSmemBytes) != cudaSuccess) {
+        if (skinny_smem_attr<16, 4>() != cudaSuccess || skinny_smem_attr<32, 4>() != cudaSuccess ||
+            skinny_smem_attr<16, 8>() != cudaSuccess || skinny_smem_attr<32, 8>() != cudaSuccess)
             return QL_ERR_CUDA;
-        }
         d.skinny_attr_set = true;
     }
     *out = &d;
@@ -132,6 +139,9 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // ------------------------------------------------------------------ shapes and plans
 
+// Bytes of the packed codes of an [N][K] weight with `bits`-bit codes (4 or 8).
+size_t code_bytes(int64_t K, int64_t N, int bits) { return static_cast<size_t>(N) * K * bits / 8; }
+
 ql_status check_shape(int64_t M, int64_t K, int64_t N, int32_t group) {
     if (group != kGroup) return QL_ERR_UNSUPPORTED;
     if (M < 1 || K < kGroup || N < 8 || K % kGroup != 0 || N % 8 != 0) return QL_ERR_INVALID_ARG;
@@ -140,6 +150,7 @@ ql_status check_shape(int64_t M, int64_t K, int64_t N, int32_t group) {
 }
 
 struct Plan {
+    int bits = 4;         // code width: 4 (W4 g64) or 8 (W8 g64)
     int path = QL_PATH_GEMV;
     int split_k = 1;
     // skinny path: stream-K runs
@@ -153,10 +164,11 @@ struct Plan {
     int slices = 0;
 };
 
-ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int sm_count, Plan* plan) {
+ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int sm_count, int bits, Plan* plan) {
     const int64_t G = K / kGroup;
     if (path == QL_PATH_AUTO) path = (M <= 32) ? QL_PATH_TC_SKINNY : QL_PATH_TC_FUSED;
     plan->path = path;
+    plan->bits = bits;
     if (path == QL_PATH_GEMV) {
         int s = split_k > 0 ? split_k : gemv_auto_split(K, N, sm_count);
         if (s > G || s > 65535) return QL_ERR_INVALID_ARG;
@@ -167,7 +179,8 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
     if (path == QL_PATH_TC_SKINNY) {
         if (M > 32 || split_k > 1) return QL_ERR_UNSUPPORTED;
         plan->nt = M <= 16 ? 16 : 32;
-        const int64_t cpt = (G + skinny::CG - 1) / skinny::CG;
+        const int64_t cg = bits == 4 ? skinny::Layout<16, 4>::CG : skinny::Layout<16, 8>::CG;
+        const int64_t cpt = (G + cg - 1) / cg;
         plan->units = ((N + skinny::BW - 1) / skinny::BW) * cpt;
         plan->ctas = static_cast<int>(std::min<int64_t>(std::min(sm_count, skinny::kMaxCtas), plan->units));
         const int64_t run = (plan->units + plan->ctas - 1) / plan->ctas;
@@ -204,10 +217,17 @@ ql_status run_gemv(const Plan& pl, const void* x, const uint32_t* codes, const v
     auto sc = static_cast<const __half*>(scales);
     auto bi = static_cast<const __half*>(biases);
     prof_begin(st);
-    if (bf16_out)
-        gemv_kernel<true><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
-    else
-        gemv_kernel<false><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
+    if (pl.bits == 8) {
+        if (bf16_out)
+            gemv8_kernel<true><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
+        else
+            gemv8_kernel<false><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
+    } else {
+        if (bf16_out)
+            gemv_kernel<true><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
+        else
+            gemv_kernel<false><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
+    }
     prof_end(st);
     if (partial) {
         const int64_t count = M * N;
@@ -217,7 +237,7 @@ ql_status run_gemv(const Plan& pl, const void* x, const uint32_t* codes, const v
         else
             splitk_reduce_kernel<false><<<blocks, 256, 0, st>>>(static_cast<const float*>(ws), y, count, pl.split_k);
     }
-    set_dispatch("path=gemv warps=%d splitk=%d launches=%d", kGemvWarps, pl.split_k, partial ? 2 : 1);
+    set_dispatch("path=gemv bits=%d warps=%d splitk=%d launches=%d", pl.bits, kGemvWarps, pl.split_k, partial ? 2 : 1);
     return launch_status();
 }
 
@@ -253,8 +273,12 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xh, K, M, K * 2, fused::BK, fused::BT,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
-    if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K / 8, N, K / 2, fused::BK / 8, fused::BW,
-                       CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+    // one K-step of codes per box: 32 bytes of each of 256 rows (4-bit codes, unswizzled) or 64 bytes
+    // (8-bit codes, 64-byte swizzle, which the dequantizers undo)
+    const int bits = pl.bits;
+    if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K * bits / 32, N, K * bits / 8,
+                       fused::BK * bits / 32, fused::BW,
+                       bits == 4 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_64B)) != QL_OK)
         return s;
     if ((s = encode_2d(&mp, CU_TENSOR_MAP_DATA_TYPE_UINT32, sb, N, G, N * 4, fused::BW, 1,
                        CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
@@ -264,8 +288,12 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
                        N * (bf16_out ? 2 : 4), 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
         return s;
 
-    convert_x_kernel<<<static_cast<unsigned>(M), kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), xh, rs,
-                                                                        static_cast<int>(K));
+    if (bits == 4)
+        convert_x_kernel<4><<<static_cast<unsigned>(M), kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), xh,
+                                                                              rs, static_cast<int>(K));
+    else
+        convert_x_kernel<8><<<static_cast<unsigned>(M), kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), xh,
+                                                                              rs, static_cast<int>(K));
     if ((s = launch_status()) != QL_OK) return s;
     // the transpose, then the fused kernel, start under programmatic dependent launch (each waits
     // for the kernels before it where it reads their output)
@@ -283,18 +311,27 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     p.num_w = static_cast<int>((N + fused::BW - 1) / fused::BW);
     const int tiles = p.num_t * p.num_w;
     const int grid = std::min(tiles, sm_count);
-    using FC = fused::DefaultCfg;
     prof_begin(st);
-    if (bf16_out)
-        s = launch_dependent(fused::fused_gemm_kernel<true, FC>, dim3(static_cast<unsigned>(grid)), fused::kThreads,
-                             FC::kSmemBytes, st, mx, mc, mp, my, p);
-    else
-        s = launch_dependent(fused::fused_gemm_kernel<false, FC>, dim3(static_cast<unsigned>(grid)), fused::kThreads,
-                             FC::kSmemBytes, st, mx, mc, mp, my, p);
+    const dim3 fgrid(static_cast<unsigned>(grid));
+    if (bits == 4) {
+        using FC = fused::DefaultCfg;
+        s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
+                                        mx, mc, mp, my, p)
+                     : launch_dependent(fused::fused_gemm_kernel<false, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
+                                        mx, mc, mp, my, p);
+    } else {
+        using FC = fused::Q8Cfg;
+        s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
+                                        mx, mc, mp, my, p)
+                     : launch_dependent(fused::fused_gemm_kernel<false, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
+                                        mx, mc, mp, my, p);
+    }
     if (s != QL_OK) return s;
     prof_end(st);
-    set_dispatch("path=tc_fused tile=%dw x %dt x %dk stages=x%d/c%d/a%d ctas=%d splitk=1 launches=3", fused::BW,
-                 fused::BT, fused::BK, FC::kNX, FC::kNC, fused::NA, grid);
+    const int nc = bits == 4 ? fused::DefaultCfg::kNC : fused::Q8Cfg::kNC;
+    const int nx = bits == 4 ? fused::DefaultCfg::kNX : fused::Q8Cfg::kNX;
+    set_dispatch("path=tc_fused bits=%d tile=%dw x %dt x %dk stages=x%d/c%d/a%d ctas=%d splitk=1 launches=3", bits,
+                 fused::BW, fused::BT, fused::BK, nx, nc, fused::NA, grid);
     (void)codes;
     return launch_status();
 }
@@ -309,20 +346,23 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     float* pmax = reinterpret_cast<float*>(wsb + pl.off_pm);
     CUtensorMap mc, mx;
     ql_status s;
-    if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K / 8, N, K / 2,
-                       skinny::kBoxGroups * skinny::BK / 8, skinny::BW, CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
+    const int bits = pl.bits;
+    // code boxes: 128 bytes (32 words) of each of 128 rows, 128-byte swizzle, for either code width
+    if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K * bits / 32, N, K * bits / 8,
+                       skinny::kBoxBytes / skinny::BW / 4, skinny::BW, CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
     if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xp, K, M, K * 2, skinny::BK, pl.nt,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
-    // scale/bias tiles by TMA need a 16-byte row pitch and chunk-aligned groups
-    const bool param_tma = (G % skinny::CG) == 0;
+    // scale/bias boxes of 8 groups by TMA need a 16-byte row pitch (G % 8 == 0); every chunk then
+    // lies inside one box
+    const bool param_tma = (G % skinny::kParGroups) == 0;
     CUtensorMap ms = mc, mb = mc;
     if (param_tma) {
-        if ((s = encode_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, G, N, G * 2, skinny::CG, skinny::BW,
+        if ((s = encode_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, scales, G, N, G * 2, skinny::kParGroups, skinny::BW,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
             return s;
-        if ((s = encode_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, biases, G, N, G * 2, skinny::CG, skinny::BW,
+        if ((s = encode_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, biases, G, N, G * 2, skinny::kParGroups, skinny::BW,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
             return s;
     }
@@ -335,7 +375,8 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     p.N = static_cast<int>(N);
     p.G = static_cast<int>(G);
     p.num_w = static_cast<int>((N + skinny::BW - 1) / skinny::BW);
-    p.cpt = static_cast<int>((G + skinny::CG - 1) / skinny::CG);
+    const int cg = bits == 4 ? skinny::Layout<16, 4>::CG : skinny::Layout<16, 8>::CG;
+    p.cpt = static_cast<int>((G + cg - 1) / cg);
     p.units = pl.units;
     p.segmax = pl.segmax;
     // row maxima, then scaled and reordered f16 activations, per-group activation sums, row exponents
@@ -353,16 +394,26 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         const float* pm = pmax;
-        if (cudaLaunchKernelEx(&cfg, skinny::skinny_prepass_kernel, static_cast<const uint4*>(x), pm,
-                               static_cast<uint4*>(xp), rowexp, static_cast<int>(K)) != cudaSuccess)
-            return QL_ERR_CUDA;
+        const cudaError_t e =
+            bits == 4 ? cudaLaunchKernelEx(&cfg, skinny::skinny_prepass_kernel<4>, static_cast<const uint4*>(x), pm,
+                                           static_cast<uint4*>(xp), rowexp, static_cast<int>(K))
+                      : cudaLaunchKernelEx(&cfg, skinny::skinny_prepass_kernel<8>, static_cast<const uint4*>(x), pm,
+                                           static_cast<uint4*>(xp), rowexp, static_cast<int>(K));
+        if (e != cudaSuccess) return QL_ERR_CUDA;
     }
     prof_begin(st);
-    if (pl.nt == 16)
-        s = launch_dependent(skinny::skinny_kernel<16>, dim3(static_cast<unsigned>(pl.ctas)), skinny::kThreads, skinny::Layout<16>::kSmemBytes, st,
+    const dim3 sgrid(static_cast<unsigned>(pl.ctas));
+    if (bits == 4 && pl.nt == 16)
+        s = launch_dependent(skinny::skinny_kernel<16, 4>, sgrid, skinny::kThreads, skinny::Layout<16, 4>::kSmemBytes, st,
+                             mc, mx, ms, mb, p);
+    else if (bits == 4)
+        s = launch_dependent(skinny::skinny_kernel<32, 4>, sgrid, skinny::kThreads, skinny::Layout<32, 4>::kSmemBytes, st,
+                             mc, mx, ms, mb, p);
+    else if (pl.nt == 16)
+        s = launch_dependent(skinny::skinny_kernel<16, 8>, sgrid, skinny::kThreads, skinny::Layout<16, 8>::kSmemBytes, st,
                              mc, mx, ms, mb, p);
     else
-        s = launch_dependent(skinny::skinny_kernel<32>, dim3(static_cast<unsigned>(pl.ctas)), skinny::kThreads, skinny::Layout<32>::kSmemBytes, st,
+        s = launch_dependent(skinny::skinny_kernel<32, 8>, sgrid, skinny::kThreads, skinny::Layout<32, 8>::kSmemBytes, st,
                              mc, mx, ms, mb, p);
     if (s != QL_OK) return s;
     prof_end(st);
@@ -377,14 +428,14 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
                              p.units, pl.ctas, pl.segmax);
     if (s != QL_OK) return s;
     (void)sm_count;
-    set_dispatch("path=tc_skinny nt=%d ctas=%d segmax=%d units=%lld launches=4", pl.nt, pl.ctas, pl.segmax,
-                 static_cast<long long>(pl.units));
+    set_dispatch("path=tc_skinny bits=%d nt=%d ctas=%d segmax=%d units=%lld launches=4", bits, pl.nt, pl.ctas,
+                 pl.segmax, static_cast<long long>(pl.units));
     return launch_status();
 }
 
 ql_status forward_impl(const void* x, const uint32_t* codes, const void* scales, const void* biases, void* y,
                        ql_dtype out_dtype, int64_t M, int64_t K, int64_t N, int32_t group, int32_t path,
-                       int32_t split_k, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                       int32_t split_k, void* workspace, size_t workspace_bytes, cudaStream_t stream, int bits) {
     ql_status s = check_shape(M, K, N, group);
     if (s != QL_OK) return s;
     if (!x || !codes || !scales || !biases || !y) return QL_ERR_INVALID_ARG;
@@ -393,7 +444,7 @@ ql_status forward_impl(const void* x, const uint32_t* codes, const void* scales,
     if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(biases) || !aligned16(y))
         return QL_ERR_ALIGNMENT;
     const int64_t G = K / kGroup;
-    const size_t xb = static_cast<size_t>(M) * K * 2, cb = static_cast<size_t>(N) * K / 2,
+    const size_t xb = static_cast<size_t>(M) * K * 2, cb = code_bytes(K, N, bits),
                  pb = static_cast<size_t>(N) * G * 2,
                  yb = static_cast<size_t>(M) * N * (out_dtype == QL_BF16 ? 2 : 4);
     if (overlap(y, yb, x, xb) || overlap(y, yb, codes, cb) || overlap(y, yb, scales, pb) || overlap(y, yb, biases, pb))
@@ -401,7 +452,7 @@ ql_status forward_impl(const void* x, const uint32_t* codes, const void* scales,
     DeviceInfo* dev = nullptr;
     if ((s = device_info(&dev)) != QL_OK) return s;
     Plan pl;
-    if ((s = make_plan(M, K, N, path, split_k, dev->sm_count, &pl)) != QL_OK) return s;
+    if ((s = make_plan(M, K, N, path, split_k, dev->sm_count, bits, &pl)) != QL_OK) return s;
     if (pl.workspace > 0) {
         if (!workspace || workspace_bytes < pl.workspace) return QL_ERR_WORKSPACE;
         if (!aligned16(workspace)) return QL_ERR_ALIGNMENT;
@@ -418,48 +469,18 @@ ql_status forward_impl(const void* x, const uint32_t* codes, const void* scales,
     return run_fused(pl, x, codes, scales, biases, y, bf16, M, K, N, workspace, stream, dev->sm_count);
 }
 
-size_t workspace_impl(int64_t M, int64_t K, int64_t N, int32_t group, int32_t path, int32_t split_k) {
+size_t workspace_impl(int64_t M, int64_t K, int64_t N, int32_t group, int32_t path, int32_t split_k, int bits) {
     if (check_shape(M, K, N, group) != QL_OK) return static_cast<size_t>(-1);
     DeviceInfo* dev = nullptr;
     int sms = 148;
     if (device_info(&dev) == QL_OK) sms = dev->sm_count;
     Plan pl;
-    if (make_plan(M, K, N, path, split_k, sms, &pl) != QL_OK) return static_cast<size_t>(-1);
+    if (make_plan(M, K, N, path, split_k, sms, bits, &pl) != QL_OK) return static_cast<size_t>(-1);
     return pl.workspace;
 }
 
-}  // namespace
-}  // namespace ql
-
-using namespace ql;
-
-extern "C" {
-
-size_t qlinear_workspace_size(int64_t M, int64_t K, int64_t N, int32_t group) {
-    return workspace_impl(M, K, N, group, QL_PATH_AUTO, 0);
-}
-
-size_t qlinear_workspace_size_config(int64_t M, int64_t K, int64_t N, int32_t group, int32_t path, int32_t split_k) {
-    return workspace_impl(M, K, N, group, path, split_k);
-}
-
-ql_status qlinear_forward(const void* x, const uint32_t* codes, const void* scales, const void* biases, void* y,
-                          int64_t M, int64_t K, int64_t N, int32_t group, void* workspace, size_t workspace_bytes,
-                          cudaStream_t stream) {
-    return forward_impl(x, codes, scales, biases, y, QL_BF16, M, K, N, group, QL_PATH_AUTO, 0, workspace,
-                        workspace_bytes, stream);
-}
-
-ql_status qlinear_forward_config(const void* x, const uint32_t* codes, const void* scales, const void* biases,
-                                 void* y, ql_dtype out_dtype, int64_t M, int64_t K, int64_t N, int32_t group,
-                                 int32_t path, int32_t split_k, void* workspace, size_t workspace_bytes,
-                                 cudaStream_t stream) {
-    return forward_impl(x, codes, scales, biases, y, out_dtype, M, K, N, group, path, split_k, workspace,
-                        workspace_bytes, stream);
-}
-
-ql_status qlinear_dequant(const uint32_t* codes, const void* scales, const void* biases, int64_t K, int64_t N,
-                          int32_t group, void* out, ql_dtype out_dtype, cudaStream_t stream) {
+ql_status dequant_impl(const uint32_t* codes, const void* scales, const void* biases, int64_t K, int64_t N,
+                       int32_t group, void* out, ql_dtype out_dtype, cudaStream_t stream, int bits) {
     ql_status s = check_shape(1, K, N, group);
     if (s != QL_OK) return s;
     if (!codes || !scales || !biases || !out) return QL_ERR_INVALID_ARG;
@@ -467,31 +488,39 @@ ql_status qlinear_dequant(const uint32_t* codes, const void* scales, const void*
     if (!aligned16(codes) || !aligned16(scales) || !aligned16(biases) || !aligned16(out)) return QL_ERR_ALIGNMENT;
     const int64_t G = K / kGroup;
     const size_t ob = static_cast<size_t>(N) * K * (out_dtype == QL_BF16 ? 2 : 4);
-    if (overlap(out, ob, codes, static_cast<size_t>(N) * K / 2) || overlap(out, ob, scales, static_cast<size_t>(N) * G * 2) ||
+    if (overlap(out, ob, codes, code_bytes(K, N, bits)) || overlap(out, ob, scales, static_cast<size_t>(N) * G * 2) ||
         overlap(out, ob, biases, static_cast<size_t>(N) * G * 2))
         return QL_ERR_INVALID_ARG;
     DeviceInfo* dev = nullptr;
     if ((s = device_info(&dev)) != QL_OK) return s;
-    const int64_t words = N * K / 8;
+    const int64_t words = N * K * bits / 32;
     const int blocks = static_cast<int>(std::min<int64_t>((words + 255) / 256, 16 * dev->sm_count));
     auto sc = static_cast<const __half*>(scales);
     auto bi = static_cast<const __half*>(biases);
-    if (out_dtype == QL_BF16)
-        dequant_kernel<true><<<blocks, 256, 0, stream>>>(codes, sc, bi, out, words);
-    else
-        dequant_kernel<false><<<blocks, 256, 0, stream>>>(codes, sc, bi, out, words);
+    if (bits == 8) {
+        if (out_dtype == QL_BF16)
+            dequant8_kernel<true><<<blocks, 256, 0, stream>>>(codes, sc, bi, out, words);
+        else
+            dequant8_kernel<false><<<blocks, 256, 0, stream>>>(codes, sc, bi, out, words);
+    } else {
+        if (out_dtype == QL_BF16)
+            dequant_kernel<true><<<blocks, 256, 0, stream>>>(codes, sc, bi, out, words);
+        else
+            dequant_kernel<false><<<blocks, 256, 0, stream>>>(codes, sc, bi, out, words);
+    }
     return launch_status();
 }
 
-ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group, uint32_t* codes,
-                       void* scales, void* biases, cudaStream_t stream) {
+ql_status pack_impl(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group, uint32_t* codes,
+                    void* scales, void* biases, cudaStream_t stream, int bits) {
     ql_status s = check_shape(1, K, N, group);
     if (s != QL_OK) return s;
     if (!w || !codes || !scales || !biases) return QL_ERR_INVALID_ARG;
+    if (imatrix != nullptr && bits != 4) return QL_ERR_UNSUPPORTED;   // the weighted fit is built for 4-bit codes
     if (N > 65535ll * kFitThreads || K / kGroup > 2147483647ll) return QL_ERR_UNSUPPORTED;   // fit grid limits
     if (!aligned16(w) || !aligned16(codes) || !aligned16(scales) || !aligned16(biases)) return QL_ERR_ALIGNMENT;
     const int64_t G = K / kGroup;
-    const size_t wb = static_cast<size_t>(N) * K * 4, cb = static_cast<size_t>(N) * K / 2,
+    const size_t wb = static_cast<size_t>(N) * K * 4, cb = code_bytes(K, N, bits),
                  pb = static_cast<size_t>(N) * G * 2;
     if (overlap(w, wb, codes, cb) || overlap(w, wb, scales, pb) || overlap(w, wb, biases, pb) ||
         overlap(codes, cb, scales, pb) || overlap(codes, cb, biases, pb) || overlap(scales, pb, biases, pb))
@@ -510,9 +539,86 @@ ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t 
     if ((s = device_info(&dev)) != QL_OK) return s;
     const int64_t groups = N * G;
     const int blocks = static_cast<int>(std::min<int64_t>((groups + 7) / 8, 32 * dev->sm_count));
-    pack_rtn_kernel<<<blocks, 256, 0, stream>>>(w, codes, static_cast<__half*>(scales), static_cast<__half*>(biases),
-                                                groups);
+    if (bits == 8)
+        pack8_rtn_kernel<<<blocks, 256, 0, stream>>>(w, codes, static_cast<__half*>(scales),
+                                                     static_cast<__half*>(biases), groups);
+    else
+        pack_rtn_kernel<<<blocks, 256, 0, stream>>>(w, codes, static_cast<__half*>(scales),
+                                                    static_cast<__half*>(biases), groups);
     return launch_status();
+}
+
+}  // namespace
+}  // namespace ql
+
+using namespace ql;
+
+extern "C" {
+
+size_t qlinear_workspace_size(int64_t M, int64_t K, int64_t N, int32_t group) {
+    return workspace_impl(M, K, N, group, QL_PATH_AUTO, 0, 4);
+}
+
+size_t qlinear_workspace_size_config(int64_t M, int64_t K, int64_t N, int32_t group, int32_t path, int32_t split_k) {
+    return workspace_impl(M, K, N, group, path, split_k, 4);
+}
+
+ql_status qlinear_forward(const void* x, const uint32_t* codes, const void* scales, const void* biases, void* y,
+                          int64_t M, int64_t K, int64_t N, int32_t group, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream) {
+    return forward_impl(x, codes, scales, biases, y, QL_BF16, M, K, N, group, QL_PATH_AUTO, 0, workspace,
+                        workspace_bytes, stream, 4);
+}
+
+ql_status qlinear_forward_config(const void* x, const uint32_t* codes, const void* scales, const void* biases,
+                                 void* y, ql_dtype out_dtype, int64_t M, int64_t K, int64_t N, int32_t group,
+                                 int32_t path, int32_t split_k, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream) {
+    return forward_impl(x, codes, scales, biases, y, out_dtype, M, K, N, group, path, split_k, workspace,
+                        workspace_bytes, stream, 4);
+}
+
+ql_status qlinear_dequant(const uint32_t* codes, const void* scales, const void* biases, int64_t K, int64_t N,
+                          int32_t group, void* out, ql_dtype out_dtype, cudaStream_t stream) {
+    return dequant_impl(codes, scales, biases, K, N, group, out, out_dtype, stream, 4);
+}
+
+ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group, uint32_t* codes,
+                       void* scales, void* biases, cudaStream_t stream) {
+    return pack_impl(w, imatrix, K, N, group, codes, scales, biases, stream, 4);
+}
+
+size_t qlinear8_workspace_size(int64_t M, int64_t K, int64_t N, int32_t group) {
+    return workspace_impl(M, K, N, group, QL_PATH_AUTO, 0, 8);
+}
+
+size_t qlinear8_workspace_size_config(int64_t M, int64_t K, int64_t N, int32_t group, int32_t path, int32_t split_k) {
+    return workspace_impl(M, K, N, group, path, split_k, 8);
+}
+
+ql_status qlinear8_forward(const void* x, const uint32_t* codes, const void* scales, const void* biases, void* y,
+                           int64_t M, int64_t K, int64_t N, int32_t group, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+    return forward_impl(x, codes, scales, biases, y, QL_BF16, M, K, N, group, QL_PATH_AUTO, 0, workspace,
+                        workspace_bytes, stream, 8);
+}
+
+ql_status qlinear8_forward_config(const void* x, const uint32_t* codes, const void* scales, const void* biases,
+                                  void* y, ql_dtype out_dtype, int64_t M, int64_t K, int64_t N, int32_t group,
+                                  int32_t path, int32_t split_k, void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream) {
+    return forward_impl(x, codes, scales, biases, y, out_dtype, M, K, N, group, path, split_k, workspace,
+                        workspace_bytes, stream, 8);
+}
+
+ql_status qlinear8_dequant(const uint32_t* codes, const void* scales, const void* biases, int64_t K, int64_t N,
+                           int32_t group, void* out, ql_dtype out_dtype, cudaStream_t stream) {
+    return dequant_impl(codes, scales, biases, K, N, group, out, out_dtype, stream, 8);
+}
+
+ql_status qlinear8_pack(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group, uint32_t* codes,
+                        void* scales, void* biases, cudaStream_t stream) {
+    return pack_impl(w, imatrix, K, N, group, codes, scales, biases, stream, 8);
 }
 
 ql_status qlinear_get_device_status(cudaStream_t stream) {

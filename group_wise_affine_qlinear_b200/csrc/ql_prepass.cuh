@@ -7,9 +7,10 @@
 //    in the f16 normal range; only entries more than ~2^29 below the row
 //    maximum are rounded (to f16 subnormals).  rowscale[m] = 2^e_m undoes the
 //    scaling in the epilogue.  Within every 8 consecutive k the f16 copy is
-//    stored in the order (0,4,1,5,2,6,3,7), which matches the order the
-//    dequantizer produces code pairs in (codes j and j+4 share one 32-bit
-//    word); permuting both operands alike leaves every dot product unchanged.
+//    stored in the order the dequantizer produces weight pairs in, so that
+//    permuting both operands alike leaves every dot product unchanged:
+//    (0,4,1,5,2,6,3,7) for 4-bit codes (codes j and j+4 share one 32-bit
+//    word's f16x2 pair), (0,2,1,3,4,6,5,7) for 8-bit codes (bytes j and j+2).
 // 2) Group parameters: scales/biases [N][G] -> sb[G][N] of (scale, bias) f16
 //    pairs, so one K-step's parameters for a run of N rows are contiguous and
 //    can be fetched by the tensor memory accelerator.
@@ -22,6 +23,8 @@ namespace ql {
 constexpr int kPrepThreads = 256;
 
 // One CTA per row.  Pass 1 reads the row for max|x|, pass 2 re-reads (L2) and converts.
+// kBits: width of the weight codes the activations will meet (4 or 8), which fixes the k order.
+template <int kBits>
 __global__ void __launch_bounds__(kPrepThreads) convert_x_kernel(const __nv_bfloat16* __restrict__ x,
                                                                  __half* __restrict__ xh,
                                                                  float* __restrict__ rowscale, int K) {
@@ -69,10 +72,18 @@ __global__ void __launch_bounds__(kPrepThreads) convert_x_kernel(const __nv_bflo
         const float f4 = bf16_lo(v.z) * inv, f5 = bf16_hi(v.z) * inv;
         const float f6 = bf16_lo(v.w) * inv, f7 = bf16_hi(v.w) * inv;
         uint4 o;
-        o.x = bits_of(__floats2half2_rn(f0, f4));
-        o.y = bits_of(__floats2half2_rn(f1, f5));
-        o.z = bits_of(__floats2half2_rn(f2, f6));
-        o.w = bits_of(__floats2half2_rn(f3, f7));
+        if constexpr (kBits == 4) {
+            o.x = bits_of(__floats2half2_rn(f0, f4));
+            o.y = bits_of(__floats2half2_rn(f1, f5));
+            o.z = bits_of(__floats2half2_rn(f2, f6));
+            o.w = bits_of(__floats2half2_rn(f3, f7));
+        } else {
+            static_assert(kBits == 8, "4- or 8-bit codes");
+            o.x = bits_of(__floats2half2_rn(f0, f2));
+            o.y = bits_of(__floats2half2_rn(f1, f3));
+            o.z = bits_of(__floats2half2_rn(f4, f6));
+            o.w = bits_of(__floats2half2_rn(f5, f7));
+        }
         dst[i] = o;
     }
 }

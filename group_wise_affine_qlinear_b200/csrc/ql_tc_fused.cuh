@@ -4,7 +4,9 @@
 //   xh    f16 activations prescaled per row by a power of two (prepass)
 //   wh    RN_f16(s * q + b): the affine grid of aimarketly "Ideogram-4-IQ4_M",
 //         "What IQ4 means here", formed by one fused f16x2 multiply-add from the
-//         exact code q, i.e. rounded once
+//         exact code q, i.e. rounded once; q is a 4-bit code, or an 8-bit code of
+//         the Q8 pack (huggingface "SceneWorks/ideogram-4-mlx", Versions) with the
+//         same per-64 scale and bias
 // Operands are f16 (A and B must share a type in kind::f16); the accumulator is
 // fp32 in tensor memory.  One K-step is exactly one 64-wide quantization group,
 // so every weight row needs one (scale, bias) pair per step.
@@ -67,14 +69,16 @@ constexpr int NA = 2;                   // TMEM weight stages
 static_assert(kAStageCol + NA * NG * 32 <= kTmemCols, "tensor memory budget");
 
 constexpr uint32_t kXBytes = BT * BK * 2;   // 24 KB
-constexpr uint32_t kCBytes = BW * BK / 2;   // 8 KB of codes
 constexpr uint32_t kPBytes = BW * 4;        // 1 KB of (scale, bias)
 constexpr uint32_t kStageBytes = 32 * 32 * 4;   // one epilogue staging block (fp32 worst case)
 constexpr uint32_t kEpiBytes = kEpiWarps * 2 * kStageBytes;   // 2 buffers per epilogue warp
 
-template <int NX, int NC>
+// NX activation stages, NC code stages, B-bit codes (4: 8 KB of codes per stage; 8: 16 KB, stored
+// with the 64-byte swizzle).
+template <int NX, int NC, int B = 4>
 struct Cfg {
-    static constexpr int kNX = NX, kNC = NC;
+    static constexpr int kNX = NX, kNC = NC, kBits = B;
+    static constexpr uint32_t kCBytes = BW * BK * B / 8;
     static constexpr uint32_t kOffX = 0;
     static constexpr uint32_t kOffC = kOffX + NX * kXBytes;
     static constexpr uint32_t kOffP = kOffC + NC * kCBytes;
@@ -88,6 +92,7 @@ struct Cfg {
 };
 
 using DefaultCfg = Cfg<4, 6>;
+using Q8Cfg = Cfg<4, 3, 8>;
 
 struct Params {
     float* rowscale;      // [M] 2^e_m
@@ -115,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
     const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
     const __grid_constant__ CUtensorMap map_params, const __grid_constant__ CUtensorMap map_y, const Params p) {
     constexpr int NX = C::kNX, NC = C::kNC;
+    constexpr int kCodeWords = BK * C::kBits / 32;      // 32-bit code words of one row per K-step
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
@@ -183,21 +189,44 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             // and wait for the TMEM stage only when the result is ready to be written.
             bool got = ptx::mbar_wait(&c_full[cs], cph, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
-            const uint4* crow = reinterpret_cast<const uint4*>(smem + C::kOffC + cs * kCBytes + r * 32);
-            const uint4 first = crow[h];
-            const uint4 second = crow[h ^ 1];
-            const uint32_t sb = reinterpret_cast<const uint32_t*>(smem + C::kOffP + cs * kPBytes)[r];
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&c_empty[cs]);     // codes and parameters are in registers
-            const uint4 c0 = h ? second : first;
-            const uint4 c1 = h ? first : second;
-            const __half2 sb2 = half2_of(sb);
-            const __half2 s2 = __low2half2(sb2);
-            const __half2 b2 = __high2half2(sb2);
-            const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
             uint32_t a[32];
+            if constexpr (C::kBits == 4) {
+                const uint4* crow = reinterpret_cast<const uint4*>(smem + C::kOffC + cs * C::kCBytes + r * 32);
+                const uint4 first = crow[h];
+                const uint4 second = crow[h ^ 1];
+                const uint32_t sb = reinterpret_cast<const uint32_t*>(smem + C::kOffP + cs * kPBytes)[r];
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&c_empty[cs]);     // codes and parameters are in registers
+                const uint4 c0 = h ? second : first;
+                const uint4 c1 = h ? first : second;
+                const __half2 sb2 = half2_of(sb);
+                const __half2 s2 = __low2half2(sb2);
+                const __half2 b2 = __high2half2(sb2);
+                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-            for (int c = 0; c < 8; ++c) dequant_word(words[c], s2, b2, &a[4 * c]);
+                for (int c = 0; c < 8; ++c) dequant_word(words[c], s2, b2, &a[4 * c]);
+            } else {
+                // Row r's 64 code bytes are four 16-byte pieces stored with the 64-byte swizzle (piece c
+                // at c ^ ((r >> 1) & 3)), so every 8 lanes of a load touch 8 distinct bank groups.
+                const uint8_t* crow = smem + C::kOffC + cs * C::kCBytes + r * 64;
+                const int sw = (r >> 1) & 3;
+                uint4 cv[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) cv[c] = *reinterpret_cast<const uint4*>(crow + ((c ^ sw) << 4));
+                const uint32_t sb = reinterpret_cast<const uint32_t*>(smem + C::kOffP + cs * kPBytes)[r];
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&c_empty[cs]);     // codes and parameters are in registers
+                const __half2 sb2 = half2_of(sb);
+                const __half2 s2 = __low2half2(sb2);
+                const __half2 b2 = __high2half2(sb2);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    dequant_word8(cv[c].x, s2, b2, &a[8 * c + 0]);
+                    dequant_word8(cv[c].y, s2, b2, &a[8 * c + 2]);
+                    dequant_word8(cv[c].z, s2, b2, &a[8 * c + 4]);
+                    dequant_word8(cv[c].w, s2, b2, &a[8 * c + 6]);
+                }
+            }
             got = ptx::mbar_wait(&a_empty[as], aph ^ 1, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
             ptx::tc_fence_after_sync();
@@ -230,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             for (uint32_t e = 0; e < early; ++e) {       // fresh stages: no empty wait
                 int kb, w_blk, t_blk;
                 step_coords(e, kb, w_blk, t_blk);
-                ptx::mbar_arrive_expect_tx(&full[e], kCBytes + kPBytes);
-                ptx::tma_load_2d(smem + C::kOffC + e * kCBytes, &map_codes, &full[e], kb * (BK / 8), w_blk * BW);
+                ptx::mbar_arrive_expect_tx(&full[e], C::kCBytes + kPBytes);
+                ptx::tma_load_2d(smem + C::kOffC + e * C::kCBytes, &map_codes, &full[e], kb * kCodeWords, w_blk * BW);
             }
             ptx::grid_dependency_wait();
             for (uint32_t e = 0; e < early; ++e) {
@@ -251,8 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                         ptx::mbar_arrive_expect_tx(&full[s], kXBytes);
                         ptx::tma_load_2d(smem + C::kOffX + s * kXBytes, &map_x, &full[s], kb * BK, t_blk * BT);
                     } else {
-                        ptx::mbar_arrive_expect_tx(&full[s], kCBytes + kPBytes);
-                        ptx::tma_load_2d(smem + C::kOffC + s * kCBytes, &map_codes, &full[s], kb * (BK / 8), w_blk * BW);
+                        ptx::mbar_arrive_expect_tx(&full[s], C::kCBytes + kPBytes);
+                        ptx::tma_load_2d(smem + C::kOffC + s * C::kCBytes, &map_codes, &full[s], kb * kCodeWords, w_blk * BW);
                         ptx::tma_load_2d(smem + C::kOffP + s * kPBytes, &map_params, &full[s], w_blk * BW, kb);
                     }
                 }

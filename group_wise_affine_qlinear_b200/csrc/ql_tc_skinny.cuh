@@ -5,8 +5,9 @@
 // The weight of row n, column k is w = s(n,g) q(n,k) + b(n,g) for the 64-group g
 // holding k (aimarketly "Ideogram-4-IQ4_M", "What IQ4 means here": w = scale * q +
 // bias).  Builder warps dequantize each group of a 128-row weight tile to the f16
-// operand RN_f16(s q + b) (dequant_word: one shift, four LOP3, four HSUB2 and four
-// HFMA2 per 8 weights) straight into tensor memory, and tcgen05.mma (kind::f16,
+// operand RN_f16(s q + b) (4-bit codes, dequant_word: one shift, four LOP3, four
+// HSUB2 and four HFMA2 per 8 weights; 8-bit codes, dequant_word8: two byte permutes,
+// two HSUB2 and two HFMA2 per 4 weights) straight into tensor memory, and tcgen05.mma (kind::f16,
 // M = 128 weight rows, N = 16 or 32 tokens, fp32 accumulation) accumulates the
 // whole run of groups the CTA owns in one tile, so nothing but the tensor core
 // touches the partial sums until the CTA leaves the tile.  This is the large-M
@@ -15,13 +16,14 @@
 //
 // The activations come from a prepass pair under programmatic dependent launch:
 // per-slice row maxima, then x' = f16(x * 2^e_t) with e_t putting the row maximum
-// in [2^14, 2^15), in the order 0,4,1,5,2,6,3,7 of every 8-block that dequant_word
-// emits its pairs in.  The main kernel starts streaming codes and parameters at
+// in [2^14, 2^15), in the order the dequantizer emits its pairs in (0,4,1,5,2,6,3,7
+// of every 8-block for 4-bit codes, 0,2,1,3,4,6,5,7 for 8-bit codes).  The main kernel starts streaming codes and parameters at
 // once and waits for the prepass only before its first activation load.
 //
-// Stream-K schedule: the work is cut into chunks of CG = 8 consecutive groups of
-// one 128-row tile (a tile has ceil(G/CG) chunks; a tile's last chunk may be
-// partial).  The chunks, tile-major, are split into one equal contiguous run per
+// Stream-K schedule: the work is cut into chunks of CG consecutive groups of one
+// 128-row tile (CG = 8 for 4-bit codes, 4 for the 8-bit codes of the Q8 pack,
+// huggingface "SceneWorks/ideogram-4-mlx", Versions; either way 32 KB of codes; a
+// tile has ceil(G/CG) chunks; a tile's last chunk may be partial).  The chunks, tile-major, are split into one equal contiguous run per
 // CTA; each tile segment a run covers leaves one fp32 partial [tokens][128]
 // (scaled by 2^e_t) in the workspace, and the reduce kernel sums, per output, the
 // partials of the CTAs that covered its tile in CTA order (deterministic) and
@@ -36,7 +38,7 @@
 // two accumulators and write the partial; the accumulators are double-buffered
 // across segments (acc_empty).
 // Warp roles (768 threads, one CTA per SM; 6 warps per SM sub-partition leave 80 registers a thread):
-//   warp 0        TMA producer of code chunks (128 rows x CG*32 B, 128B swizzle) with their scale and
+//   warp 0        TMA producer of code chunks (128 rows x 256 B, 128B swizzle) with their scale and
 //                 bias tiles
 //   warp 1        TMA producer of activation tiles (NT x 64 f16 per group), its own ring: activation
 //                 loads from L2 take about a microsecond, so they run several chunks ahead
@@ -57,24 +59,27 @@ constexpr int UK = 16;
 constexpr int kBuildCopies = 4, kMmaCopies = 2;
 constexpr int kWarpTmaC = 0, kWarpTmaX = 1, kWarpMma0 = 2, kWarpBuild0 = 4, kWarpDrain0 = kWarpBuild0 + 4 * kBuildCopies;
 constexpr int kThreads = (kWarpDrain0 + 4) * 32;
-constexpr int CG = 8;                    // groups per chunk: four pairs, one per builder copy
-constexpr int kBoxGroups = 4;            // groups per code box: 128 bytes of each row (the 128B-swizzle span)
 constexpr int NA = 4;                    // A pair stages in tensor memory
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kBoxBytes = BW * BK / 2 * kBoxGroups;     // 16 KB: one code box
-constexpr uint32_t kCBytes = kBoxBytes * (CG / kBoxGroups);  // codes per chunk
-constexpr uint32_t kParHalf = BW * CG * 2;                   // one chunk's scales (or biases): [128][CG] f16
-constexpr uint32_t kStageBytes = kCBytes + 2 * kParHalf;     // [codes | scales | biases]
+constexpr uint32_t kBoxBytes = BW * 128;                     // 16 KB: one code box, 128 bytes of each row
+constexpr int kParGroups = 8;                                // groups per scale (bias) box: 16-byte rows
+constexpr uint32_t kParHalf = BW * kParGroups * 2;           // one box of scales (or biases): [128][8] f16
 constexpr int kMaxCtas = 256;                // the planner launches at most this many CTAs, so every
                                              // tile's covering CTAs fit the reduce kernel's list
-static_assert(CG == 2 * kBuildCopies && kBoxGroups == 4, "one pair of every chunk per builder copy");
 static_assert(NA % kBuildCopies == 0 && NA % kMmaCopies == 0, "every A stage serves one copy of each role");
-static_assert(kStageBytes % 1024 == 0, "swizzled code boxes need 1 KB alignment");
 
-template <int NT>
+// NT tokens, B-bit codes.  A chunk is CG groups: 8 for 4-bit codes (four pairs, one per builder copy),
+// 4 for 8-bit codes (two pairs), so either way a chunk's codes are 32 KB in two 128-byte-wide boxes.
+template <int NT, int B = 4>
 struct Layout {
-    static constexpr int NC = NT == 16 ? 4 : 3;                          // code/parameter chunk stages
-    static constexpr int NXC = NT == 16 ? 4 : 3;                         // activation chunk stages
+    static constexpr int kBits = B;
+    static constexpr int CG = B == 4 ? 8 : 4;                            // groups per chunk
+    static constexpr int kGroupWords = BK * B / 32;                      // code words of one row per group
+    static constexpr int kBoxGroups = 128 / (4 * kGroupWords);           // groups per code box
+    static constexpr uint32_t kCBytes = kBoxBytes * (CG / kBoxGroups);   // codes per chunk
+    static constexpr uint32_t kStageBytes = kCBytes + 2 * kParHalf;      // [codes | scales | biases]
+    static constexpr int NC = B == 4 ? (NT == 16 ? 4 : 3) : (NT == 16 ? 5 : 4);    // code/parameter chunk stages
+    static constexpr int NXC = B == 4 ? (NT == 16 ? 4 : 3) : (NT == 16 ? 5 : 4);   // activation chunk stages
     static constexpr uint32_t kXTile = NT * BK * 2;                      // one group's activation tile (f16)
     static constexpr uint32_t kXBytes = CG * kXTile;                     // one chunk's activation tiles
     static constexpr uint32_t kOffC = 0;                                  // [NC][codes | scales | biases]
@@ -85,6 +90,10 @@ struct Layout {
     static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
     static constexpr uint32_t kAccCol = 0;                                // accumulator (set e, issuer c) at (2e+c)*NT
     static constexpr uint32_t kACol = 4 * NT;                             // A stage st, half h at kACol + 32(2st+h)
+    static_assert(B == 4 || B == 8, "4- or 8-bit codes");
+    static_assert(CG <= 2 * kBuildCopies && CG % kBoxGroups == 0 && kParGroups % CG == 0,
+                  "at most one pair of a chunk per builder copy; whole code boxes; whole chunks per parameter box");
+    static_assert(kStageBytes % 1024 == 0, "swizzled code boxes need 1 KB alignment");
     static_assert(kXTile % 1024 == 0, "swizzled activation tiles need 1 KB alignment");
     static_assert(kACol + 2 * NA * 32 <= kTmemCols, "tensor memory budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -94,7 +103,7 @@ struct Params {
     float* partial;          // [P][segmax][M][128] fp32, scaled by 2^e_t
     const __half* scales;    // [N][G]
     const __half* biases;    // [N][G]
-    int param_tma;           // 1: scales/biases arrive as TMA tiles (needs G % CG == 0); 0: direct loads
+    int param_tma;           // 1: scales/biases arrive as TMA tiles (needs G % 8 == 0); 0: direct loads
     int M, N, G, num_w;
     int cpt;                 // chunks per tile = ceil(G / CG)
     int64_t units;           // num_w * cpt chunks
@@ -133,7 +142,9 @@ __global__ void __launch_bounds__(256) skinny_rowmax_kernel(const uint4* __restr
 }
 
 // For row t: e_t puts max_k |x[t][k]| in [2^14, 2^15) (0 for a zero or non-finite row);
-// xp[t][k] = f16(x * 2^e_t) in the order 0,4,1,5,2,6,3,7 of each 8-block; rowexp[t] = -e_t.
+// xp[t][k] = f16(x * 2^e_t) in the order the dequantizer of kBits-bit codes emits its pairs in
+// (0,4,1,5,2,6,3,7 of each 8-block for 4-bit codes, 0,2,1,3,4,6,5,7 for 8-bit codes); rowexp[t] = -e_t.
+template <int kBits>
 __global__ void __launch_bounds__(256) skinny_prepass_kernel(const uint4* __restrict__ x, const float* __restrict__ pmax,
                                                              uint4* __restrict__ xp, int* __restrict__ rowexp, int K) {
     ptx::launch_dependents();
@@ -155,23 +166,30 @@ __global__ void __launch_bounds__(256) skinny_prepass_kernel(const uint4* __rest
                             bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
         uint32_t o[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {                           // slot pairs (k0, k4) (k1, k5) (k2, k6) (k3, k7)
-            const __half2 h = __halves2half2(__float2half_rn(ldexpf(f[j], ex)), __float2half_rn(ldexpf(f[j + 4], ex)));
+        for (int j = 0; j < 4; ++j) {
+            // 4-bit: slot pairs (k0, k4) (k1, k5) (k2, k6) (k3, k7); 8-bit: (k0, k2) (k1, k3) (k4, k6) (k5, k7)
+            const int lo = kBits == 4 ? j : 2 * (j & 2) + (j & 1);
+            const int hi = kBits == 4 ? j + 4 : lo + 2;
+            const __half2 h = __halves2half2(__float2half_rn(ldexpf(f[lo], ex)), __float2half_rn(ldexpf(f[hi], ex)));
             o[j] = *reinterpret_cast<const uint32_t*>(&h);
         }
         xp[static_cast<int64_t>(t) * kb + c] = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
 
-template <int NT>
+template <int NT, int B>
 __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_constant__ CUtensorMap map_codes,
                                                             const __grid_constant__ CUtensorMap map_x,
                                                             const __grid_constant__ CUtensorMap map_scales,
                                                             const __grid_constant__ CUtensorMap map_biases,
                                                             const Params p) {
-    using L = Layout<NT>;
+    using L = Layout<NT, B>;
     constexpr int NC = L::NC;
     constexpr int NXC = L::NXC;
+    constexpr int CG = L::CG;
+    constexpr int kBoxGroups = L::kBoxGroups;
+    constexpr uint32_t kCBytes = L::kCBytes;
+    constexpr uint32_t kStageBytes = L::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
@@ -261,10 +279,13 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
                 ptx::mbar_arrive_expect_tx(&c_full[s], kCBytes + (p.param_tma ? 2 * kParHalf : 0u));
 #pragma unroll
                 for (int bx = 0; bx < CG / kBoxGroups; ++bx)   // consecutive boxes: long contiguous row segments
-                    ptx::tma_load_2d(st + bx * kBoxBytes, &map_codes, &c_full[s], (g0 + bx * kBoxGroups) * (BK / 8), w * BW);
+                    ptx::tma_load_2d(st + bx * kBoxBytes, &map_codes, &c_full[s], (g0 + bx * kBoxGroups) * L::kGroupWords,
+                                     w * BW);
                 if (p.param_tma) {
-                    ptx::tma_load_2d(st + kCBytes, &map_scales, &c_full[s], g0, w * BW);
-                    ptx::tma_load_2d(st + kCBytes + kParHalf, &map_biases, &c_full[s], g0, w * BW);
+                    // the 8-group box holding the chunk (a chunk of 4 groups uses half of it)
+                    const int gp = g0 - g0 % kParGroups;
+                    ptx::tma_load_2d(st + kCBytes, &map_scales, &c_full[s], gp, w * BW);
+                    ptx::tma_load_2d(st + kCBytes + kParHalf, &map_biases, &c_full[s], gp, w * BW);
                 }
             }
             // never leave the CTA with bulk copies still landing in its shared memory
@@ -370,27 +391,30 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
             const int s = static_cast<int>(i % NC);
             bool got = ptx::mbar_wait(&c_full[s], (i / NC) & 1u, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
-            // row r's 32 code bytes of group q sit in code box q / 4 at the 16-byte pieces 2 (q % 4) and
-            // 2 (q % 4) + 1 of its box row, stored with the 128-byte swizzle (piece c at c ^ (r % 8)), so
-            // every 8 lanes of a load touch 8 bank groups; its scales and biases of groups 2j, 2j + 1
-            // are one 32-bit word each
-            uint4 cw[4];
+            // row r's code bytes of group q (32 for 4-bit codes, 64 for 8-bit codes) sit in code box
+            // q / kBoxGroups at the 16-byte pieces kPieces (q % kBoxGroups) .. of its box row, stored with
+            // the 128-byte swizzle (piece c at c ^ (r % 8)), so every 8 lanes of a load touch 8 bank
+            // groups; its scales and biases of groups 2j, 2j + 1 are one 32-bit word each
+            constexpr int kPieces = L::kGroupWords / 4;       // 16-byte pieces per group row: 2 or 4
+            uint4 cw[2 * kPieces];
             uint32_t sp = 0u, bp = 0u;
             if (mine) {
                 const uint8_t* st = smem + L::kOffC + s * kStageBytes;
-                const uint8_t* crow = st + (j >> 1) * kBoxBytes + r * 128;
+                const uint8_t* crow = st + ((2 * j) / kBoxGroups) * kBoxBytes + r * 128;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int c = 2 * ((2 * j + h) & 3);
+                    const int c = kPieces * ((2 * j + h) % kBoxGroups);
                     if (2 * j + h < ng) {
-                        cw[2 * h] = *reinterpret_cast<const uint4*>(crow + ((c ^ (r & 7)) << 4));
-                        cw[2 * h + 1] = *reinterpret_cast<const uint4*>(crow + (((c + 1) ^ (r & 7)) << 4));
+#pragma unroll
+                        for (int e = 0; e < kPieces; ++e)
+                            cw[kPieces * h + e] = *reinterpret_cast<const uint4*>(crow + (((c + e) ^ (r & 7)) << 4));
                     }
                 }
                 const int n = w * BW + r;
                 if (p.param_tma) {
-                    sp = *reinterpret_cast<const uint32_t*>(st + kCBytes + r * CG * 2 + 4 * j);
-                    bp = *reinterpret_cast<const uint32_t*>(st + kCBytes + kParHalf + r * CG * 2 + 4 * j);
+                    const int pc0 = g0 % kParGroups + 2 * j;        // the pair's first column in the parameter box
+                    sp = *reinterpret_cast<const uint32_t*>(st + kCBytes + r * kParGroups * 2 + 2 * pc0);
+                    bp = *reinterpret_cast<const uint32_t*>(st + kCBytes + kParHalf + r * kParGroups * 2 + 2 * pc0);
                 } else {
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
@@ -417,11 +441,22 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
                     if (2 * j + h < ng) {
                         const __half2 s2 = h ? __high2half2(half2_of(sp)) : __low2half2(half2_of(sp));
                         const __half2 b2 = h ? __high2half2(half2_of(bp)) : __low2half2(half2_of(bp));
-                        const uint4 c0 = cw[2 * h], c1 = cw[2 * h + 1];
-                        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
                         uint32_t a[32];
+                        if constexpr (B == 4) {
+                            const uint4 c0 = cw[2 * h], c1 = cw[2 * h + 1];
+                            const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) dequant_word(words[c], s2, b2, &a[4 * c]);
+                            for (int c = 0; c < 8; ++c) dequant_word(words[c], s2, b2, &a[4 * c]);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const uint4 cv = cw[4 * h + c];
+                                dequant_word8(cv.x, s2, b2, &a[8 * c + 0]);
+                                dequant_word8(cv.y, s2, b2, &a[8 * c + 2]);
+                                dequant_word8(cv.z, s2, b2, &a[8 * c + 4]);
+                                dequant_word8(cv.w, s2, b2, &a[8 * c + 6]);
+                            }
+                        }
                         ptx::tmem_st_32x32b_x32(tmem_base + lane_addr + L::kACol + 32u * static_cast<uint32_t>(2 * st + h), a);
                     }
                 }

@@ -21,6 +21,13 @@ Recipe (shared by every workload):
   * activations x[m][j] = RN_bf16(z * sigma_j), z ~ N(0, 1), sigma_j = exp(N(mu_j, 1)),
     mu_j = 0, except the long-K text projection, whose 13 channel blocks of
     4096 get mu = -1.5 + 0.25 * block to mimic 13 concatenated encoder layers.
+
+8-bit workloads (the Q8 pack of huggingface "SceneWorks/ideogram-4-mlx",
+Versions; aimarketly "Ideogram-4-IQ4_M", Conversion, keeps the conditioning
+projection at 8 bits): codes uint32 [N][K/4], each word 4 uniform codes in
+[0, 255], low byte first; scale s = RN_f16(exp(U(ln 1e-3, ln 2e-2)) / 17) and
+bias b = RN_f16(-127.5 * s + N(0, (1.7 * s)^2)), so a group spans the same
+range of weights as a 4-bit group (255 s = 15 * 17 s).
 """
 from __future__ import annotations
 
@@ -69,6 +76,19 @@ def weights(seed: int, widx: int, N: int, K: int):
     return codes, s, b
 
 
+def weights8(seed: int, widx: int, N: int, K: int):
+    """8-bit packed codes uint32 [N][K/4], scales float16 [N][K/64], biases float16 [N][K/64]."""
+    assert K % GROUP == 0
+    G = K // GROUP
+    codes = _rng(seed, _TID_CODES, widx).integers(0, 1 << 32, size=(N, K // 4), dtype=np.uint32)
+    lo, hi = np.log(1e-3), np.log(2e-2)
+    s = (np.exp(_rng(seed, _TID_SCALES, widx).uniform(lo, hi, size=(N, G))) / 17.0).astype(np.float16)
+    s64 = s.astype(np.float64)
+    noise = _rng(seed, _TID_BIASES, widx).standard_normal(size=(N, G))
+    b = (-127.5 * s64 + noise * (1.7 * s64)).astype(np.float16)
+    return codes, s, b
+
+
 def channel_sigma(seed: int, xidx: int, K: int, block_means: bool = False) -> np.ndarray:
     z = _rng(seed, _TID_SIGMA, xidx).standard_normal(size=K)
     mu = np.zeros(K)
@@ -112,6 +132,7 @@ class Workload:
     xidx: int = 0
     block_means: bool = False
     fitted_rows: int = 0          # leading rows of W that come from an imatrix fit of dense floats
+    bits: int = 4                 # code width: 4 (W4 g64) or 8 (W8 g64)
     note: str = ""
 
     @property
@@ -120,12 +141,14 @@ class Workload:
 
     @property
     def weight_bytes(self) -> int:
-        return self.N * self.K // 2 + 4 * self.N * (self.K // GROUP)
+        return self.N * self.K * self.bits // 8 + 4 * self.N * (self.K // GROUP)
 
     def x(self, M: int | None = None) -> np.ndarray:
         return activations(self.seed, self.xidx, self.M if M is None else M, self.K, self.block_means)
 
     def w(self):
+        if self.bits == 8:
+            return weights8(self.seed, self.widx, self.N, self.K)
         return weights(self.seed, self.widx, self.N, self.K)
 
 
@@ -140,6 +163,8 @@ WORKLOADS = {
                  note="DiT SwiGLU down projection"),
         Workload("text_proj", 512, 53248, 4608, seed=3, block_means=True,
                  note="llm_cond_proj 53248->4608; M swept over 1, 8, 32, 512 (leading rows)"),
+        Workload("text_proj_w8", 512, 53248, 4608, seed=3, widx=1, block_means=True, bits=8,
+                 note="llm_cond_proj 53248->4608 at 8 bits; M swept over 1, 8, 32, 512 (leading rows)"),
         Workload("canvas2048_n4608", 33792, 4608, 4608, seed=4, widx=0,
                  note="2048^2 canvas, two packed samples"),
         Workload("canvas2048_n13824", 33792, 4608, 13824, seed=4, widx=1,

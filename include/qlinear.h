@@ -1,5 +1,6 @@
 /*
- * qlinear.h -- C ABI of the group-wise affine W4 g64 quantized linear layer (sm_100a).
+ * qlinear.h -- C ABI of the group-wise affine W4 g64 quantized linear layer (sm_100a),
+ * with its W8 g64 variant (qlinear8_*, at the end).
  *
  * The packed format (aimarketly "Ideogram-4-IQ4_M", intro: one f16 scale and one
  * f16 bias per 64 weights on top of 4-bit codes, 4.5 bits per weight;
@@ -198,6 +199,46 @@ QL_API ql_status qlinear_forward_noalloc(const void* x, const uint32_t* codes, c
  * caller owns both events; NULL, NULL turns the hook off.  Thread-local.
  */
 QL_API ql_status qlinear_set_profile_events(cudaEvent_t start, cudaEvent_t stop);
+
+/*
+ * W8 g64: the 8-bit variant of the same format.  The pages ship an 8-bit pack beside the 4-bit one
+ * (huggingface "SceneWorks/ideogram-4-mlx", Versions: Q8) and keep the modulation and conditioning
+ * projections at 8 bits (aimarketly "Ideogram-4-IQ4_M", Conversion); the scale and bias stay one f16
+ * pair per 64 weights, so a weight costs 8.5 bits.
+ *
+ *   codes   uint32   [N][K/4]    code (n, k) = (codes[n][k/4] >> 8*(k%4)) & 0xFF, low byte first
+ *   scales, biases, x, y          as for the 4-bit calls; w = s * q + b with q in [0, 255]
+ *
+ * Each qlinear8_* call has the arguments, preconditions, errors and arithmetic of the 4-bit call of
+ * the same name, with the code tensor above in place of the 4-bit one:
+ *   qlinear8_forward / _config   y = x . W^T; the same kernel paths (QL_PATH_GEMV multiplies exact
+ *                                codes in fp32; both tcgen05 paths multiply RN_f16(s * q + b) by f16
+ *                                activations scaled per row by a power of two, fp32 accumulation)
+ *   qlinear8_workspace_size[_config]
+ *   qlinear8_dequant             out = RN_fp32(s * q + b) (bf16: rounded once more), bit-exact
+ *   qlinear8_pack                min/max round-to-nearest with 255 levels:
+ *                                s = RN32(RN32(max-min)/255), scale = RN_f16(s), bias = RN_f16(min),
+ *                                q = clamp(rint(RN32(RN32(w-bias)/scale)), 0, 255) (ties to even),
+ *                                q = 0 when scale == 0; imatrix must be NULL (QL_ERR_UNSUPPORTED
+ *                                otherwise: the importance-weighted fit is built for 4-bit codes)
+ */
+QL_API size_t qlinear8_workspace_size(int64_t M, int64_t K, int64_t N, int32_t group);
+QL_API size_t qlinear8_workspace_size_config(int64_t M, int64_t K, int64_t N, int32_t group,
+                                             int32_t path, int32_t split_k);
+QL_API ql_status qlinear8_forward(const void* x, const uint32_t* codes, const void* scales,
+                                  const void* biases, void* y, int64_t M, int64_t K, int64_t N,
+                                  int32_t group, void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream);
+QL_API ql_status qlinear8_forward_config(const void* x, const uint32_t* codes, const void* scales,
+                                         const void* biases, void* y, ql_dtype out_dtype,
+                                         int64_t M, int64_t K, int64_t N, int32_t group,
+                                         int32_t path, int32_t split_k,
+                                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
+QL_API ql_status qlinear8_dequant(const uint32_t* codes, const void* scales, const void* biases,
+                                  int64_t K, int64_t N, int32_t group, void* out, ql_dtype out_dtype,
+                                  cudaStream_t stream);
+QL_API ql_status qlinear8_pack(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group,
+                               uint32_t* codes, void* scales, void* biases, cudaStream_t stream);
 
 /* Static, human-readable name of a status code. */
 QL_API const char* qlinear_status_string(ql_status status);

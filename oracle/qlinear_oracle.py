@@ -476,6 +476,11 @@ def dequant8_f32(codes, scales, biases) -> np.ndarray:
     return dequant8_exact(codes, scales, biases).astype(np.float32)
 
 
+def dequant8_f16(codes, scales, biases) -> np.ndarray:
+    """RN_f16 of the exact s*q + b for 8-bit codes: the weight operand of the tensor-core paths (R7)."""
+    return dequant8_exact(codes, scales, biases).astype(np.float16)
+
+
 def dequant8_bf16(codes, scales, biases) -> np.ndarray:
     """bf16 dequant of 8-bit codes = RN_bf16(fp32 dequant) as uint16 bits."""
     return round_bf16(dequant8_f32(codes, scales, biases).astype(np.float64))
@@ -484,6 +489,13 @@ def dequant8_bf16(codes, scales, biases) -> np.ndarray:
 def forward8_ref(x_bits, codes, scales, biases) -> np.ndarray:
     """y_ref[m][n] = sum_k x[m][k] * w(n, k) in float64, w the fp32 dequant of 8-bit codes."""
     x = decode_bf16(x_bits)
+    w = dequant8_f32(codes, scales, biases).astype(np.float64)
+    return x @ w.T
+
+
+def forward8_rows(x_bits, codes, scales, biases, rows) -> np.ndarray:
+    """forward8_ref restricted to the given rows of x (rows are independent)."""
+    x = decode_bf16(np.asarray(x_bits)[np.asarray(rows)])
     w = dequant8_f32(codes, scales, biases).astype(np.float64)
     return x @ w.T
 

@@ -33,6 +33,16 @@ def random_layer(rng: np.random.Generator, M: int, K: int, N: int):
     return x, codes, s, b
 
 
+def random_layer8(rng: np.random.Generator, M: int, K: int, N: int):
+    """Small random layer with 8-bit codes, drawn as in the synthetic module's 8-bit recipe."""
+    codes = rng.integers(0, 1 << 32, size=(N, K // 4), dtype=np.uint32)
+    s = (np.exp(rng.uniform(np.log(1e-3), np.log(2e-2), size=(N, K // 64))) / 17.0).astype(np.float16)
+    b = (-127.5 * s.astype(np.float64) + 1.7 * s.astype(np.float64) * rng.standard_normal(s.shape)).astype(np.float16)
+    sigma = np.exp(rng.standard_normal(K)).astype(np.float32)
+    x = S.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32) * sigma[None, :])
+    return x, codes, s, b
+
+
 def sample_rows(M: int, n_random: int = 64, seed: int = 0, tile: int = 128) -> np.ndarray:
     """Row 0, row M-1, both sides of every tile boundary, and random rows."""
     rows = {0, M - 1}

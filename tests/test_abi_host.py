@@ -25,13 +25,15 @@ def _declared():
     for f in os.listdir(inc):
         if f.endswith(".h"):
             txt = open(os.path.join(inc, f)).read()
-            names += re.findall(r"QL_API\s+[\w\s\*]+?\b(qlinear_\w+)\s*\(", txt)
+            names += re.findall(r"QL_API\s+[\w\s\*]+?\b(qlinear8?_\w+)\s*\(", txt)
     return sorted(set(names))
 
 
 def test_header_declares_entry_points():
     names = _declared()
-    for n in ("qlinear_forward", "qlinear_dequant", "qlinear_pack", "qlinear_workspace_size"):
+    for n in ("qlinear_forward", "qlinear_dequant", "qlinear_pack", "qlinear_workspace_size",
+              "qlinear8_forward", "qlinear8_forward_config", "qlinear8_dequant", "qlinear8_pack",
+              "qlinear8_workspace_size", "qlinear8_workspace_size_config"):
         assert n in names
 
 
@@ -112,3 +114,44 @@ def test_workspace_size_values(L):
 def test_profile_events_pairing(L):
     assert L.qlinear_set_profile_events(FAKE, None) == 1
     assert L.qlinear_set_profile_events(None, None) == 0
+
+
+# ---------------------------------------------------------------- 8-bit codes (codes [N][K/4])
+
+def _fwd8(L, x=FAKE, c=FAKE + (1 << 24), s=FAKE + (2 << 24), b=FAKE + (3 << 24), y=FAKE + (4 << 24),
+          M=16, K=256, N=256, group=64):
+    return L.qlinear8_forward(x, c, s, b, y, M, K, N, group, None, 0, None)
+
+
+def test_forward8_rejects_bad_arguments(L):
+    assert _fwd8(L, group=32) == 3
+    assert _fwd8(L, K=100) == 1
+    assert _fwd8(L, N=12) == 1
+    assert _fwd8(L, M=0) == 1
+    assert _fwd8(L, x=0) == 1
+    assert _fwd8(L, c=FAKE + (1 << 24) + 4) == 2
+    assert _fwd8(L, y=FAKE) == 1
+
+
+def test_forward8_counts_one_byte_per_code(L):
+    # 256 x 256 8-bit codes span 64 KiB: a y starting 40000 bytes in lies inside them (it would not
+    # for 4-bit codes, which span 32 KiB)
+    assert _fwd8(L, y=FAKE + (1 << 24) + 40000) == 1
+    assert L.qlinear8_dequant(FAKE, FAKE + (1 << 24), FAKE + (2 << 24), 256, 256, 64, FAKE + 40000, 0, None) == 1
+
+
+def test_pack8_validation(L):
+    # the importance-weighted fit is built for 4-bit codes only
+    assert L.qlinear8_pack(FAKE, FAKE + (4 << 24), 256, 256, 64, FAKE + (1 << 24), FAKE + (2 << 24),
+                           FAKE + (3 << 24), None) == 3
+    assert L.qlinear8_pack(FAKE, None, 256, 256, 32, FAKE + (1 << 24), FAKE + (2 << 24), FAKE + (3 << 24), None) == 3
+    # codes (64 KiB) running into the scales
+    assert L.qlinear8_pack(FAKE, None, 256, 256, 64, FAKE + (1 << 24), FAKE + (1 << 24) + 40000, FAKE + (3 << 24),
+                           None) == 1
+
+
+def test_workspace_size8_values(L):
+    M, K, N = 4608, 4608, 13824
+    assert ql.workspace_size8(M, K, N, ql.PATH_TC_FUSED) == M * K * 2 + M * 4 + (K // 64) * N * 4
+    assert ql.workspace_size8(2, 4096, 64, ql.PATH_GEMV, 4) == 4 * 2 * 64 * 4
+    assert L.qlinear8_workspace_size(16, 100, 256, 64) == ctypes.c_size_t(-1).value

@@ -470,6 +470,26 @@ def test_w8_dequant_f32_is_correctly_rounded():
             assert abs(got - exact) <= abs(lo - exact) and abs(got - exact) <= abs(hi - exact)
 
 
+def test_w8_dequant_f16_is_correctly_rounded():
+    """f16 operand of 8-bit codes = binary16 nearest to the exact rational s*q + b."""
+    _, codes, s, b = _w8_layer(_rng(47), 1, 128, 24)
+    w16 = O.dequant8_f16(codes, s, b)
+    q = O.unpack_codes8(codes, 128)
+    for n in range(24):
+        for k in range(0, 128, 3):
+            exact = Fraction(float(s[n, k // 64])) * int(q[n, k]) + Fraction(float(b[n, k // 64]))
+            got = Fraction(float(w16[n, k]))
+            lo = Fraction(float(np.nextafter(w16[n, k], np.float16(-np.inf))))
+            hi = Fraction(float(np.nextafter(w16[n, k], np.float16(np.inf))))
+            assert abs(got - exact) <= abs(lo - exact) and abs(got - exact) <= abs(hi - exact)
+
+
+def test_w8_forward_rows_equals_full_forward():
+    x, codes, s, b = _w8_layer(_rng(48), 9, 192, 16)
+    rows = np.array([0, 4, 8])
+    assert np.array_equal(O.forward8_rows(x, codes, s, b, rows), O.forward8_ref(x, codes, s, b)[rows])
+
+
 def test_w8_dequant_bf16_is_bf16_of_f32_dequant():
     _, codes, s, b = _w8_layer(_rng(42), 1, 128, 16)
     w32 = O.dequant8_f32(codes, s, b)
