@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-m", action="store_true", help="skip the small-M weight-streaming measurements")
     ap.add_argument("--no-pack", action="store_true", help="skip the quantizer (qlinear_pack) measurement")
+    ap.add_argument("--w8", action="store_true",
+                    help="also measure the 8-bit conditioning projection (text_proj_w8) at M = 1, 8, 32")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     return ap.parse_args()
 
@@ -153,7 +155,7 @@ def oracle_rate(w: S.Workload, M: int, seconds: float, x_bits=None, weights=None
     while True:
         r0 = (chunk * 64) % x.shape[0]
         rows = np.arange(r0, min(r0 + 64, x.shape[0]))
-        O.forward_rows(x, codes, s, b, rows)
+        (O.forward8_rows if w.bits == 8 else O.forward_rows)(x, codes, s, b, rows)
         rows_done += rows.size
         chunk += 1
         if time.perf_counter() - t0 >= seconds:
@@ -279,11 +281,12 @@ class Case:
         self.sc = torch.from_numpy(self.s_np).to(dev)
         self.bi = torch.from_numpy(self.b_np).to(dev)
         self.y = torch.empty((M, self.N), dtype=torch.bfloat16, device=dev)
-        ws_bytes = ql.workspace_size(M, self.K, self.N, path)
+        ws_bytes = ql.workspace_size(M, self.K, self.N, path, bits=w.bits)
         self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.fwd = ql.forward8 if w.bits == 8 else ql.forward
 
     def step(self):
-        self.ql.forward(self.x, self.codes, self.sc, self.bi, out=self.y, workspace=self.ws, path=self.path)
+        self.fwd(self.x, self.codes, self.sc, self.bi, out=self.y, workspace=self.ws, path=self.path)
 
     def warm(self, n):
         for _ in range(n):
@@ -400,7 +403,7 @@ def main():
         if i >= 2:
             s_c.wait_event(out_done[i - 2])             # step i-2's y buffer has been copied out
         flush.fill_(i & 0xFF)
-        ql.forward(xb[b], case.codes, case.sc, case.bi, out=yb[b], workspace=case.ws, path=case.path)
+        case.fwd(xb[b], case.codes, case.sc, case.bi, out=yb[b], workspace=case.ws, path=case.path)
         comp_done[i].record(s_c)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[i])
@@ -412,18 +415,22 @@ def main():
     mean_e2e = t_begin.elapsed_time(t_end) / a.steps
 
     # ---- the small-M half of the metric: weight streaming on the 53248 -> 4608 text projection
-    small = []
-    if not a.no_small_m:
-        tp = S.WORKLOADS["text_proj"]
+    def small_m(name):
+        out = []
+        tp = S.WORKLOADS[name]
         for Ms in (1, 8, 32):
             c = Case(ql, torch, tp, Ms, 0, dev, flush)
             c.warm(3)
             st, mn = c.timed(max(10, a.steps))
-            small.append({"M": Ms, "dispatch": c.dispatch, "step_us": st * 1e3, "kernel_us": mn * 1e3,
-                          "weight_GBps": tp.weight_bytes / (st * 1e-3) / 1e9,
-                          "algorithmic_GBps": c.algorithmic_bytes() / (st * 1e-3) / 1e9})
+            out.append({"M": Ms, "dispatch": c.dispatch, "step_us": st * 1e3, "kernel_us": mn * 1e3,
+                        "weight_GBps": tp.weight_bytes / (st * 1e-3) / 1e9,
+                        "algorithmic_GBps": c.algorithmic_bytes() / (st * 1e-3) / 1e9})
             del c
         torch.cuda.synchronize()
+        return out
+
+    small = [] if a.no_small_m else small_m("text_proj")
+    small_w8 = small_m("text_proj_w8") if a.w8 else []
 
     # ---- the quantizer: importance-weighted fit and RTN pack of a DiT-shaped weight
     pack = None if a.no_pack else pack_measure(ql, torch, dev, flush)
@@ -449,8 +456,8 @@ def main():
         roof = {"bound": "hbm", "achieved": main_rate, "peak": peak_gbs, "unit": "GB/s",
                 "frac": main_rate / peak_gbs, "traffic": traffic, "kernel": kernel, "kernel_ms": mean_main,
                 "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                "algorithmic": "packed W (0.5625 B/weight) + x + y bytes per launch"}
-    for sm in small:
+                "algorithmic": f"packed W ({w.bits / 8 + 0.0625:g} B/weight) + x + y bytes per launch"}
+    for sm in small + small_w8:
         sm["frac_hbm_weight"] = sm["weight_GBps"] / peak_gbs
 
     line = {
@@ -466,6 +473,8 @@ def main():
         "clocks": clk,
         "small_m": small,
     }
+    if small_w8:
+        line["small_m_w8"] = small_w8
     if pack is not None:
         line["pack"] = pack
     if rank == 0 and world == 1 and not a.no_cpu_baseline:

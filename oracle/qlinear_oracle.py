@@ -48,6 +48,17 @@ notes of the repository):
      0xFF (low byte first), q in [0, 255]; scales and biases as in R1, so a
      weight costs 8 + 0.5 bits (the same "+0.5" overhead); RTN as R3 with 255
      levels in place of 15.
+  R10 SwiGLU up/gate pair: the DiT block's MLP is a SwiGLU of three Linears
+     with intermediate size 12288 (jimmysue "Ideogram 4" notes, sec. 2.1
+     block diagram and sec. 2.8 spec table); the pages print no formula, so
+     the plain one: h = silu(x . W_gate^T) * (x . W_up^T) elementwise, with
+     silu(z) = z / (1 + exp(-z)); gate and up are two packed [I][K] weights of
+     the same format, and h is rounded once to bf16.
+  R11 tolerance of h: each linear output may err by R5's per-element allowance
+     d = 1.5e-2 * rms of that output; since |silu'| <= 1.1 everywhere, the mean
+     value theorem gives |dh| <= 1.1 * d_g * (|u| + d_u) + |silu(g)| * d_u per
+     element (plus half a bf16 ulp of h), and relative Frobenius error <= 8e-3
+     (two factors, each within R5's 4e-3).
 
 Parity status: the imatrix fit (pack_imatrix) is a search heuristic with no
 printed reference values; only its invariants are pinned ("never worse than
@@ -525,3 +536,60 @@ def pack8_rtn(w):
     bias16 = mn.astype(np.float16)
     q = nearest_codes8(g, scale16, bias16)
     return pack_codes8(q.reshape(N, K)), scale16, bias16
+
+
+# --------------------------------------------------------------------------
+# SwiGLU up/gate pair (R10, R11)
+# --------------------------------------------------------------------------
+
+SILU_SLOPE_MAX = 1.1      # max_z silu'(z) = 1.0998... (at z = 2.3994...); min is -0.0998...
+
+
+def silu(z) -> np.ndarray:
+    """silu(z) = z * sigmoid(z) = z / (1 + exp(-z)) in float64 (-0 for very negative z)."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def swiglu_linears(x_bits, gate, up, rows=None, bits: int = 4):
+    """(g, u) = (x . W_gate^T, x . W_up^T) in float64 over the given rows of x.
+
+    gate and up are (codes, scales, biases) triples of [I][K] weights with `bits`-bit codes.
+    """
+    x_bits = np.asarray(x_bits)
+    rows = np.arange(x_bits.shape[0]) if rows is None else np.asarray(rows)
+    fwd = forward_rows if bits == 4 else forward8_rows
+    return fwd(x_bits, *gate, rows), fwd(x_bits, *up, rows)
+
+
+def swiglu_ref(x_bits, gate, up, rows=None, bits: int = 4) -> np.ndarray:
+    """h = silu(g) * u (R10), float64 [rows][I]."""
+    g, u = swiglu_linears(x_bits, gate, up, rows, bits)
+    return silu(g) * u
+
+
+def swiglu_tolerance(h, g_ref, u_ref, bf16_output: bool = True) -> dict:
+    """Error metrics of reading R11 for h against the float64 reference built from g_ref, u_ref.
+
+    relF      = ||h - h_ref||_F / ||h_ref||_F                              (gate <= 8e-3)
+    max_ratio = max_i (|h_i - h_ref_i| - half_ulp_i)^+ / bound_i             (gate <= 1)
+    bound_i   = 1.1 * d_g * (|u_i| + d_u) + |silu(g_i)| * d_u,  d = 1.5e-2 * rms(output)
+    """
+    h = np.asarray(h, dtype=np.float64)
+    g_ref = np.asarray(g_ref, dtype=np.float64)
+    u_ref = np.asarray(u_ref, dtype=np.float64)
+    h_ref = silu(g_ref) * u_ref
+    d_g = 1.5e-2 * float(np.sqrt(np.mean(g_ref * g_ref)))
+    d_u = 1.5e-2 * float(np.sqrt(np.mean(u_ref * u_ref)))
+    bound = SILU_SLOPE_MAX * d_g * (np.abs(u_ref) + d_u) + np.abs(silu(g_ref)) * d_u
+    d = np.abs(h - h_ref)
+    allowance = half_ulp_bf16(np.maximum(np.abs(h), np.abs(h_ref))) if bf16_output else 0.0
+    excess = np.maximum(d - allowance, 0.0)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = np.where(excess > 0, excess / np.where(bound > 0, bound, 1.0), 0.0)
+        ratio = np.where((excess > 0) & (bound <= 0), np.inf, ratio)
+    ref_norm = float(np.linalg.norm(h_ref))
+    relF = float(np.linalg.norm(h - h_ref) / ref_norm) if ref_norm > 0 else float(np.linalg.norm(h - h_ref))
+    max_ratio = float(ratio.max(initial=0.0))
+    return {"relF": relF, "max_ratio": max_ratio, "ok": bool(relF <= 8e-3 and max_ratio <= 1.0)}

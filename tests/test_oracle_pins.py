@@ -597,3 +597,88 @@ def test_w8_and_w4_agree_on_a_shared_grid():
     d4 = O.dequant_f32(*O.pack_rtn(w))
     d8 = O.dequant8_f32(*O.pack8_rtn(w))
     assert np.array_equal(d4, d8)
+
+
+# ---------------------------------------------------------------- SwiGLU pair (readings R10, R11)
+
+def test_silu_matches_library_sigmoid():
+    """silu(z) = z * expit(z), expit being scipy's logistic sigmoid (a library routine)."""
+    from scipy.special import expit
+    z = np.concatenate([np.linspace(-50, 50, 20001), [0.0, -0.0, 1e-300, -1e-300, 700.0, -700.0, 745.0, -745.0,
+                                                      800.0, -800.0]])
+    ours = O.silu(z)
+    lib = z * expit(z)
+    assert np.all(np.abs(ours - lib) <= 4 * np.spacing(np.abs(lib)) + 1e-320)
+    assert O.silu(np.array([-800.0]))[0] == 0.0 and O.silu(np.array([800.0]))[0] == 800.0
+
+
+def test_silu_slope_bound_is_tight():
+    """The constant R11 uses: max silu' = sigma(z)(1 + z(1 - sigma(z))) <= 1.1, attained near 1.0998."""
+    from scipy.special import expit
+    z = np.linspace(-40, 40, 800001)
+    sg = expit(z)
+    d = sg * (1 + z * (1 - sg))
+    assert d.max() <= O.SILU_SLOPE_MAX and d.max() > 1.0998 and d.min() > -0.1
+
+
+def test_swiglu_equals_brute_force():
+    """Pure-Python h[m][n] = silu(sum_k x w_g) * sum_k x w_u with exactly rounded sums and math.exp."""
+    import math
+    rng = _rng(60)
+    x, cg, sg, bg = _random_layer(rng, 3, 128, 5)
+    _, cu, su, bu = _random_layer(rng, 3, 128, 5)
+    h = O.swiglu_ref(x, (cg, sg, bg), (cu, su, bu))
+    xf = O.decode_bf16(x)
+    wg = O.dequant_f32(cg, sg, bg).astype(np.float64)
+    wu = O.dequant_f32(cu, su, bu).astype(np.float64)
+    for m in range(3):
+        for n in range(5):
+            g = math.fsum(float(xf[m, k]) * float(wg[n, k]) for k in range(128))
+            u = math.fsum(float(xf[m, k]) * float(wu[n, k]) for k in range(128))
+            ref = g / (1.0 + math.exp(-g)) * u
+            assert abs(h[m, n] - ref) <= 1e-12 * (abs(ref) + 1e-6)
+
+
+def test_swiglu_one_hot_selects_weights():
+    """x = e_k: g = w_g(n, k) and u = w_u(n, k) exactly, so h = w_g * expit(w_g) * w_u (scipy's sigmoid)."""
+    from scipy.special import expit
+    rng = _rng(61)
+    _, cg, sg, bg = _random_layer(rng, 1, 192, 24)
+    _, cu, su, bu = _random_layer(rng, 1, 192, 24)
+    ks = np.array([0, 5, 63, 64, 130, 191])
+    x = np.zeros((ks.size, 192), dtype=np.uint16)
+    x[np.arange(ks.size), ks] = 0x3F80
+    h = O.swiglu_ref(x, (cg, sg, bg), (cu, su, bu))
+    wg = O.dequant_f32(cg, sg, bg).astype(np.float64)[:, ks].T
+    wu = O.dequant_f32(cu, su, bu).astype(np.float64)[:, ks].T
+    ref = wg * expit(wg) * wu
+    assert np.all(np.abs(h - ref) <= 4 * np.spacing(np.abs(ref)) + 1e-300)
+
+
+def test_swiglu_negated_up_weight_negates_output():
+    """(s, b) -> (-s, -b) negates every up weight exactly, hence u and h exactly."""
+    rng = _rng(62)
+    x, cg, sg, bg = _random_layer(rng, 4, 256, 8)
+    _, cu, su, bu = _random_layer(rng, 4, 256, 8)
+    h = O.swiglu_ref(x, (cg, sg, bg), (cu, su, bu))
+    hn = O.swiglu_ref(x, (cg, sg, bg), (cu, -su, -bu))
+    assert np.array_equal(hn, -h)
+
+
+def test_swiglu_tolerance_gates():
+    """R11's gate: the reference rounded to bf16 passes; an error of twice the bound, or a relF above 8e-3, fails."""
+    rng = _rng(63)
+    x, cg, sg, bg = _random_layer(rng, 6, 256, 16)
+    _, cu, su, bu = _random_layer(rng, 6, 256, 16)
+    g, u = O.swiglu_linears(x, (cg, sg, bg), (cu, su, bu))
+    h_ref = O.silu(g) * u
+    h_bf16 = O.decode_bf16(O.round_bf16(h_ref))
+    assert O.swiglu_tolerance(h_bf16, g, u)["ok"]
+    d_g = 1.5e-2 * np.sqrt(np.mean(g * g))
+    d_u = 1.5e-2 * np.sqrt(np.mean(u * u))
+    bound = 1.1 * d_g * (abs(u[2, 3]) + d_u) + abs(O.silu(g[2, 3])) * d_u
+    bad = h_ref.copy()
+    bad[2, 3] += 2 * bound + 2 * abs(h_ref[2, 3])
+    t = O.swiglu_tolerance(bad, g, u, bf16_output=False)
+    assert not t["ok"] and t["max_ratio"] > 1.0
+    assert not O.swiglu_tolerance(h_ref * 1.01, g, u, bf16_output=False)["ok"]     # relF = 1e-2
