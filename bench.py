@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-m", action="store_true", help="skip the small-M weight-streaming measurements")
     ap.add_argument("--no-pack", action="store_true", help="skip the quantizer (qlinear_pack) measurement")
+    ap.add_argument("--swiglu", action="store_true",
+                    help="also measure the fused SwiGLU pair on the MLP at the pages' width (I = 12288)")
     ap.add_argument("--w8", action="store_true",
                     help="also measure the 8-bit conditioning projection (text_proj_w8) at M = 1, 8, 32")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -125,6 +127,47 @@ def pack_measure(ql, torch, dev, flush, runs=3):
     return {"workload": f"dense N(0, 0.02^2) {PACK_ROWS} x {PACK_K}, imatrix = E[x^2] of 512 synthetic rows",
             "groups": groups, "fit_ms": fit_ms, "fit_groups_per_s": groups / (fit_ms * 1e-3),
             "rtn_ms": rtn_ms, "rtn_GBps": rtn_bytes / (rtn_ms * 1e-3) / 1e9}
+
+
+def swiglu_measure(ql, torch, dev, flush, peak_tf, steps=10):
+    """Device time of the fused SwiGLU pair on the MLP at the pages' width (4608 tokens, K 4608, I 12288)."""
+    w = S.WORKLOADS["mlp_gate_up_12288"]
+    x = torch.from_numpy(w.x().view(np.int16)).view(torch.bfloat16).to(dev)
+    gate, up = w.w_pair()
+    dev3 = lambda c, s, b: (torch.from_numpy(c.view(np.int32)).to(dev), torch.from_numpy(s).to(dev),  # noqa: E731
+                            torch.from_numpy(b).to(dev))
+    gd, ud = dev3(*gate), dev3(*up)
+    h = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(ql.swiglu_workspace_size(w.M, w.K, w.N), dtype=torch.uint8, device=dev)
+    step = lambda: ql.swiglu(x, gd, ud, out=h, workspace=ws)  # noqa: E731
+    for _ in range(3):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    dispatch = ql.last_dispatch()
+    call_ms, main_ms = [], []
+    for i in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.fill_(i & 0xFF)
+        e0.record()
+        step()
+        e1.record()
+        flush.fill_(i & 0xFF)
+        m0.record()
+        m1.record()
+        ql.set_profile_events(m0, m1)
+        step()
+        ql.set_profile_events(None, None)
+        torch.cuda.synchronize()
+        call_ms.append(e0.elapsed_time(e1))
+        main_ms.append(m0.elapsed_time(m1))
+    assert ql.device_status() == 0, "the SwiGLU pair reported an error"
+    flops = 2.0 * w.M * w.K * 2 * w.N
+    call, main = sum(call_ms) / steps, sum(main_ms) / steps
+    return {"workload": f"{w.name} M={w.M} K={w.K} I={w.N} (gate + up)", "dispatch": dispatch,
+            "step_ms": call, "kernel_ms": main, "TFLOPs": flops / (call * 1e-3) / 1e12,
+            "kernel_TFLOPs": flops / (main * 1e-3) / 1e12, "kernel_frac": flops / (main * 1e-3) / 1e12 / peak_tf}
 
 
 def oracle_fit_rate(rows=4):
@@ -434,6 +477,7 @@ def main():
 
     # ---- the quantizer: importance-weighted fit and RTN pack of a DiT-shaped weight
     pack = None if a.no_pack else pack_measure(ql, torch, dev, flush)
+    swiglu = swiglu_measure(ql, torch, dev, flush, peaks()[0]) if a.swiglu else None
 
     mean_step, mean_main, mean_e2e = max_over_ranks([mean_step, mean_main, mean_e2e], dev)
 
@@ -475,6 +519,8 @@ def main():
     }
     if small_w8:
         line["small_m_w8"] = small_w8
+    if swiglu is not None:
+        line["swiglu"] = swiglu
     if pack is not None:
         line["pack"] = pack
     if rank == 0 and world == 1 and not a.no_cpu_baseline:

@@ -14,7 +14,8 @@ Tensors follow the ABI layout:
     y       torch.bfloat16 [M][N]     (y = x . W^T, W[n][k] = scale * code + bias)
 The 8-bit variant (forward8, dequant8, pack8, workspace_size8) takes codes as
 torch.int32 [N][K/4] (4 codes per word, low byte first) with the same scales
-and biases.
+and biases.  swiglu(x, gate, up) runs a SwiGLU up/gate pair of two packed
+[I][K] weights in one call: h = silu(x . W_gate^T) * (x . W_up^T).
 """
 from __future__ import annotations
 
@@ -38,6 +39,8 @@ from ._lib import (  # noqa: F401
     pack,
     pack8,
     set_profile_events,
+    swiglu,
+    swiglu_workspace_size,
     version,
     workspace_size,
     workspace_size8,

@@ -86,6 +86,10 @@ def lib() -> ctypes.CDLL:
         L.qlinear8_dequant.restype = ctypes.c_int
         L.qlinear8_pack.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp, vp]
         L.qlinear8_pack.restype = ctypes.c_int
+        L.qlinear_swiglu_workspace_size.argtypes = [i64, i64, i64, i32]
+        L.qlinear_swiglu_workspace_size.restype = sz
+        L.qlinear_swiglu_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i32, vp, sz, vp]
+        L.qlinear_swiglu_forward.restype = ctypes.c_int
         _lib = L
         return L
 
@@ -246,6 +250,46 @@ def _pack(w, imatrix, stream, bits):
     _check(getattr(L, name)(w.data_ptr(), imp, K, N, GROUP, codes.data_ptr(), scales.data_ptr(), biases.data_ptr(),
                             _stream_handle(stream)), name)
     return codes, scales, biases
+
+
+def swiglu_workspace_size(M: int, K: int, I: int) -> int:
+    """Workspace bytes of swiglu() (qlinear_swiglu_workspace_size)."""
+    v = lib().qlinear_swiglu_workspace_size(M, K, I, GROUP)
+    if v == ctypes.c_size_t(-1).value:
+        raise ValueError("shape not supported")
+    return int(v)
+
+
+def swiglu(x: torch.Tensor, gate, up, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+           out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+    """h = silu(x . W_gate^T) * (x . W_up^T) for two packed [I][K] weights (qlinear_swiglu_forward).
+
+    gate and up are (codes int32 [I][K/8], scales f16 [I][K/64], biases f16 [I][K/64]) triples.
+    """
+    L = lib()
+    gc, gs, gb = gate
+    uc, us, ub = up
+    I, K = _weights_shape(gc, gs)
+    M = x.shape[0]
+    _need_cuda(x, "x", torch.bfloat16, (M, K))
+    for name, c, s, b in (("gate", gc, gs, gb), ("up", uc, us, ub)):
+        _need_cuda(c, name + " codes", torch.int32, (I, K // 8))
+        _need_cuda(s, name + " scales", torch.float16, (I, K // GROUP))
+        _need_cuda(b, name + " biases", torch.float16, (I, K // GROUP))
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bfloat16 or float32")
+    if out is None:
+        out = torch.empty((M, I), dtype=out_dtype, device=x.device)
+    _need_cuda(out, "out", out_dtype, (M, I))
+    need = swiglu_workspace_size(M, K, I)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check(L.qlinear_swiglu_forward(x.data_ptr(), gc.data_ptr(), gs.data_ptr(), gb.data_ptr(), uc.data_ptr(),
+                                    us.data_ptr(), ub.data_ptr(), out.data_ptr(),
+                                    _BF16 if out_dtype == torch.bfloat16 else _F32, M, K, I, GROUP,
+                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                    _stream_handle(stream)), "qlinear_swiglu_forward")
+    return out
 
 
 def device_status(stream=None) -> int:

@@ -56,13 +56,13 @@ cudaError_t skinny_smem_attr() {
                                 skinny::Layout<NT, B>::kSmemBytes);
 }
 
-template <class FC>
+template <class FC, bool kSwiGLU = false>
 cudaError_t fused_smem_attr() {
-    const cudaError_t e = cudaFuncSetAttribute(fused::fused_gemm_kernel<true, FC>,
+    const cudaError_t e = cudaFuncSetAttribute(fused::fused_gemm_kernel<true, FC, kSwiGLU>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, FC::kSmemBytes);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(fused::fused_gemm_kernel<false, FC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                FC::kSmemBytes);
+    return cudaFuncSetAttribute(fused::fused_gemm_kernel<false, FC, kSwiGLU>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, FC::kSmemBytes);
 }
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -78,7 +78,8 @@ ql_status device_info(DeviceInfo** out) {
         d.sm_count = n;
     }
     if (!d.fused_attr_set) {
-        if (fused_smem_attr<fused::DefaultCfg>() != cudaSuccess || fused_smem_attr<fused::Q8Cfg>() != cudaSuccess)
+        if (fused_smem_attr<fused::DefaultCfg>() != cudaSuccess || fused_smem_attr<fused::Q8Cfg>() != cudaSuccess ||
+            fused_smem_attr<fused::DefaultCfg, true>() != cudaSuccess)
             return QL_ERR_CUDA;
         d.fused_attr_set = true;
     }
@@ -316,15 +317,15 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     if (bits == 4) {
         using FC = fused::DefaultCfg;
         s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
-                                        mx, mc, mp, my, p)
+                                        mx, mc, mc, mp, my, p)
                      : launch_dependent(fused::fused_gemm_kernel<false, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
-                                        mx, mc, mp, my, p);
+                                        mx, mc, mc, mp, my, p);
     } else {
         using FC = fused::Q8Cfg;
         s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
-                                        mx, mc, mp, my, p)
+                                        mx, mc, mc, mp, my, p)
                      : launch_dependent(fused::fused_gemm_kernel<false, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
-                                        mx, mc, mp, my, p);
+                                        mx, mc, mc, mp, my, p);
     }
     if (s != QL_OK) return s;
     prof_end(st);
@@ -431,6 +432,113 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     set_dispatch("path=tc_skinny bits=%d nt=%d ctas=%d segmax=%d units=%lld launches=4", bits, pl.nt, pl.ctas,
                  pl.segmax, static_cast<long long>(pl.units));
     return launch_status();
+}
+
+// ------------------------------------------------------------------ SwiGLU pair (gate and up in one GEMM)
+
+struct SwigluPlan {
+    int num_w = 0;            // tiles of 128 intermediate columns
+    int64_t ncols = 0;        // columns of the interleaved parameter array: 256 per tile
+    size_t off_rs = 0, off_sb = 0, workspace = 0;
+};
+
+SwigluPlan swiglu_plan(int64_t M, int64_t K, int64_t I) {
+    SwigluPlan pl;
+    const int64_t G = K / kGroup;
+    pl.num_w = static_cast<int>((I + fused::BWG - 1) / fused::BWG);
+    pl.ncols = static_cast<int64_t>(pl.num_w) * fused::BW;
+    pl.off_rs = round_up(static_cast<size_t>(M) * K * 2, 256);
+    pl.off_sb = pl.off_rs + round_up(static_cast<size_t>(M) * 4, 256);
+    pl.workspace = pl.off_sb + round_up(static_cast<size_t>(G) * pl.ncols * 4, 256);
+    return pl;
+}
+
+ql_status run_swiglu(const SwigluPlan& pl, const void* x, const uint32_t* gc, const void* gs, const void* gb,
+                     const uint32_t* uc, const void* us, const void* ub, void* h, bool bf16_out, int64_t M, int64_t K,
+                     int64_t I, void* ws, cudaStream_t st, int sm_count) {
+    const int64_t G = K / kGroup;
+    auto* base = static_cast<uint8_t*>(ws);
+    auto* xh = reinterpret_cast<__half*>(base);
+    auto* rs = reinterpret_cast<float*>(base + pl.off_rs);
+    auto* sb = reinterpret_cast<uint32_t*>(base + pl.off_sb);
+    CUtensorMap mx, mcg, mcu, mp, my;
+    ql_status s;
+    if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xh, K, M, K * 2, fused::BK, fused::BT,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
+        return s;
+    // 128-row code boxes: a tile's gate rows, then the same rows of the up weight
+    if ((s = encode_2d(&mcg, CU_TENSOR_MAP_DATA_TYPE_UINT32, gc, K / 8, I, K / 2, fused::BK / 8, fused::BWG,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+        return s;
+    if ((s = encode_2d(&mcu, CU_TENSOR_MAP_DATA_TYPE_UINT32, uc, K / 8, I, K / 2, fused::BK / 8, fused::BWG,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+        return s;
+    if ((s = encode_2d(&mp, CU_TENSOR_MAP_DATA_TYPE_UINT32, sb, pl.ncols, G, pl.ncols * 4, fused::BW, 1,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+        return s;
+    if ((s = encode_2d(&my, bf16_out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, h, I, M,
+                       I * (bf16_out ? 2 : 4), 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+        return s;
+    convert_x_kernel<4><<<static_cast<unsigned>(M), kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), xh, rs,
+                                                                          static_cast<int>(K));
+    if ((s = launch_status()) != QL_OK) return s;
+    const dim3 tgrid(static_cast<unsigned>((G + 31) / 32), static_cast<unsigned>(pl.ncols / 32));
+    if ((s = launch_dependent(transpose_params_pair_kernel, tgrid, 256, 0, st, static_cast<const __half*>(gs),
+                              static_cast<const __half*>(gb), static_cast<const __half*>(us),
+                              static_cast<const __half*>(ub), sb, static_cast<int>(I), static_cast<int>(G),
+                              static_cast<int>(pl.ncols))) != QL_OK)
+        return s;
+    fused::Params p;
+    p.rowscale = rs;
+    p.y = h;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(I);
+    p.G = static_cast<int>(G);
+    p.num_t = static_cast<int>((M + fused::BT - 1) / fused::BT);
+    p.num_w = pl.num_w;
+    const int tiles = p.num_t * p.num_w;
+    const int grid = std::min(tiles, sm_count);
+    using FC = fused::DefaultCfg;
+    const dim3 fgrid(static_cast<unsigned>(grid));
+    prof_begin(st);
+    s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, FC, true>, fgrid, fused::kThreads, FC::kSmemBytes,
+                                    st, mx, mcg, mcu, mp, my, p)
+                 : launch_dependent(fused::fused_gemm_kernel<false, FC, true>, fgrid, fused::kThreads, FC::kSmemBytes,
+                                    st, mx, mcg, mcu, mp, my, p);
+    if (s != QL_OK) return s;
+    prof_end(st);
+    set_dispatch("path=tc_fused_swiglu bits=4 tile=%dg+%du x %dt x %dk stages=x%d/c%d/a%d ctas=%d launches=3",
+                 fused::BWG, fused::BWG, fused::BT, fused::BK, FC::kNX, FC::kNC, fused::NA, grid);
+    return launch_status();
+}
+
+ql_status swiglu_impl(const void* x, const uint32_t* gc, const void* gs, const void* gb, const uint32_t* uc,
+                      const void* us, const void* ub, void* h, ql_dtype out_dtype, int64_t M, int64_t K, int64_t I,
+                      int32_t group, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    ql_status s = check_shape(M, K, I, group);
+    if (s != QL_OK) return s;
+    if (!x || !gc || !gs || !gb || !uc || !us || !ub || !h) return QL_ERR_INVALID_ARG;
+    if (out_dtype != QL_BF16 && out_dtype != QL_F32) return QL_ERR_INVALID_ARG;
+    const void* in[7] = {x, gc, gs, gb, uc, us, ub};
+    for (const void* q : in)
+        if (!aligned16(q)) return QL_ERR_ALIGNMENT;
+    if (!aligned16(h)) return QL_ERR_ALIGNMENT;
+    const int64_t G = K / kGroup;
+    const size_t xb = static_cast<size_t>(M) * K * 2, cb = code_bytes(K, I, 4), pb = static_cast<size_t>(I) * G * 2,
+                 hb = static_cast<size_t>(M) * I * (out_dtype == QL_BF16 ? 2 : 4);
+    const size_t in_bytes[7] = {xb, cb, pb, pb, cb, pb, pb};
+    for (int i = 0; i < 7; ++i)
+        if (overlap(h, hb, in[i], in_bytes[i])) return QL_ERR_INVALID_ARG;
+    const SwigluPlan pl = swiglu_plan(M, K, I);
+    if (!workspace || workspace_bytes < pl.workspace) return QL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QL_ERR_ALIGNMENT;
+    if (overlap(workspace, pl.workspace, h, hb)) return QL_ERR_INVALID_ARG;
+    for (int i = 0; i < 7; ++i)
+        if (overlap(workspace, pl.workspace, in[i], in_bytes[i])) return QL_ERR_INVALID_ARG;
+    DeviceInfo* dev = nullptr;
+    if ((s = device_info(&dev)) != QL_OK) return s;
+    return run_swiglu(pl, x, gc, gs, gb, uc, us, ub, h, out_dtype == QL_BF16, M, K, I, workspace, stream,
+                      dev->sm_count);
 }
 
 ql_status forward_impl(const void* x, const uint32_t* codes, const void* scales, const void* biases, void* y,
@@ -586,6 +694,19 @@ ql_status qlinear_dequant(const uint32_t* codes, const void* scales, const void*
 ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group, uint32_t* codes,
                        void* scales, void* biases, cudaStream_t stream) {
     return pack_impl(w, imatrix, K, N, group, codes, scales, biases, stream, 4);
+}
+
+size_t qlinear_swiglu_workspace_size(int64_t M, int64_t K, int64_t I, int32_t group) {
+    if (check_shape(M, K, I, group) != QL_OK) return static_cast<size_t>(-1);
+    return swiglu_plan(M, K, I).workspace;
+}
+
+ql_status qlinear_swiglu_forward(const void* x, const uint32_t* gate_codes, const void* gate_scales,
+                                 const void* gate_biases, const uint32_t* up_codes, const void* up_scales,
+                                 const void* up_biases, void* h, ql_dtype out_dtype, int64_t M, int64_t K, int64_t I,
+                                 int32_t group, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return swiglu_impl(x, gate_codes, gate_scales, gate_biases, up_codes, up_scales, up_biases, h, out_dtype, M, K, I,
+                       group, workspace, workspace_bytes, stream);
 }
 
 size_t qlinear8_workspace_size(int64_t M, int64_t K, int64_t N, int32_t group) {

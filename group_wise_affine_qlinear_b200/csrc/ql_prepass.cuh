@@ -116,4 +116,41 @@ __global__ void __launch_bounds__(256) transpose_params_kernel(const __half* __r
     ptx::grid_dependency_wait();
 }
 
+// SwiGLU pair: sb[g][256 w + r] = (scale, bias) of gate row 128 w + r for r < 128, of up row
+// 128 w + (r - 128) for r >= 128 (zeros past row I-1), so that one K-step's parameters of tile w are
+// one contiguous run of 256 pairs in the fused kernel's row order.  32x32 tiles as above; a tile's 32
+// destination columns never straddle a 128-row half, so they come from 32 consecutive rows of one
+// weight.  grid: (ceil(G / 32), num_w * 8).
+__global__ void __launch_bounds__(256) transpose_params_pair_kernel(const __half* __restrict__ gate_scales,
+                                                                    const __half* __restrict__ gate_biases,
+                                                                    const __half* __restrict__ up_scales,
+                                                                    const __half* __restrict__ up_biases,
+                                                                    uint32_t* __restrict__ sb, int I, int G,
+                                                                    int ncols) {
+    ptx::launch_dependents();
+    __shared__ uint32_t tile[32][33];
+    const int g0 = blockIdx.x * 32, c0 = blockIdx.y * 32;     // c0: first destination column
+    const int w = c0 >> 8, rr = c0 & 255;
+    const bool up = rr >= 128;
+    const int n0 = w * 128 + (rr & 127);                      // first source row
+    const __half* sc = up ? up_scales : gate_scales;
+    const __half* bi = up ? up_biases : gate_biases;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    for (int r = ty; r < 32; r += 8) {
+        const int n = n0 + r, g = g0 + tx;
+        uint32_t v = 0;
+        if (n < I && g < G) {
+            const int64_t i = static_cast<int64_t>(n) * G + g;
+            v = static_cast<uint32_t>(__half_as_ushort(sc[i])) | (static_cast<uint32_t>(__half_as_ushort(bi[i])) << 16);
+        }
+        tile[r][tx] = v;
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {
+        const int g = g0 + r, c = c0 + tx;
+        if (g < G && c < ncols) sb[static_cast<int64_t>(g) * ncols + c] = tile[tx][r];
+    }
+    ptx::grid_dependency_wait();
+}
+
 }  // namespace ql

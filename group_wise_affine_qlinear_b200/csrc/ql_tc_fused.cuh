@@ -40,6 +40,16 @@
 // Rings: X (activation tiles, freed by MMA completion), C (codes + parameters,
 // freed once read by the dequantizers), A (TMEM weight stages, freed by MMA
 // completion); accumulators are freed per group by the epilogue.
+//
+// SwiGLU mode (kSwiGLU): the DiT block's MLP is a SwiGLU of three Linears (jimmysue
+// "Ideogram 4" notes, sec. 2.1 and 2.8); this mode fuses the gate and up
+// projections and the gating.  A tile's two row groups are the same 128 rows of
+// the gate weight (group 0) and of the up weight (group 1), loaded as two
+// 128-row code boxes from two tensor maps, with their (scale, bias) pairs
+// interleaved the same way by the parameter prepass.  The two accumulators then
+// hold g and u for the same 128 intermediate columns and 192 tokens, and each of
+// the 8 epilogue warps reads both for its lane quarter and half of the tokens and
+// writes h = silu(g) * u = g / (1 + e^-g) * u in fp32, rounded once.
 #pragma once
 
 #include "ql_ptx.cuh"
@@ -115,11 +125,14 @@ __device__ __forceinline__ void ring_pos(uint32_t i, int& stage, uint32_t& phase
     phase = (i / N) & 1u;
 }
 
-template <bool kBf16Out, class C>
+// map_codes2: the up weight's codes in SwiGLU mode (128-row boxes, like map_codes there); unused otherwise.
+template <bool kBf16Out, class C, bool kSwiGLU = false>
 __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
     const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
-    const __grid_constant__ CUtensorMap map_params, const __grid_constant__ CUtensorMap map_y, const Params p) {
+    const __grid_constant__ CUtensorMap map_codes2, const __grid_constant__ CUtensorMap map_params,
+    const __grid_constant__ CUtensorMap map_y, const Params p) {
     constexpr int NX = C::kNX, NC = C::kNC;
+    static_assert(!kSwiGLU || C::kBits == 4, "the SwiGLU pair is built for 4-bit codes");
     constexpr int kCodeWords = BK * C::kBits / 32;      // 32-bit code words of one row per K-step
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -151,7 +164,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         for (int i = 0; i < NA; ++i) { ptx::mbar_init(&a_full[i], kDequantWarps); ptx::mbar_init(&a_empty[i], NG); }
         ptx::mbar_init(&acc_full[0], NG);
         static_assert(kWarpEpi0 % 4 == 0, "epilogue warp w must own TMEM lane quarter w % 4");
-        for (int g = 0; g < NG; ++g) ptx::mbar_init(&acc_empty[g], 4);
+        // an accumulator is drained by its group's 4 epilogue warps, or in SwiGLU mode by all 8
+        for (int g = 0; g < NG; ++g) ptx::mbar_init(&acc_empty[g], kSwiGLU ? kEpiWarps : 4);
         for (int g = 0; g < NG; ++g) ptx::mbar_init(drain + g, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -160,6 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
     if (warp == kWarpEpi0 && lane == 0) ptx::prefetch_tensormap(&map_y);
     if (warp == kWarpTmaC && lane == 0) {
         ptx::prefetch_tensormap(&map_codes);
+        if constexpr (kSwiGLU) ptx::prefetch_tensormap(&map_codes2);
         ptx::prefetch_tensormap(&map_params);
     }
     if (warp == kWarpMma) {
@@ -251,6 +266,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             const uint32_t first_steps = static_cast<uint32_t>(p.G) * static_cast<uint32_t>(
                 (num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x));
             const uint32_t early = is_x ? 0u : min(static_cast<uint32_t>(NC), first_steps);
+            // one K-step of a tile's codes: 256 rows of one weight, or in SwiGLU mode 128 gate rows
+            // followed by the same 128 rows of the up weight
+            auto load_codes = [&](uint8_t* dst, uint64_t* bar, int kb, int w_blk) {
+                if constexpr (kSwiGLU) {
+                    ptx::tma_load_2d(dst, &map_codes, bar, kb * kCodeWords, w_blk * BWG);
+                    ptx::tma_load_2d(dst + C::kCBytes / 2, &map_codes2, bar, kb * kCodeWords, w_blk * BWG);
+                } else {
+                    ptx::tma_load_2d(dst, &map_codes, bar, kb * kCodeWords, w_blk * BW);
+                }
+            };
             auto step_coords = [&](uint32_t step, int& kb, int& w_blk, int& t_blk) {
                 const int t = static_cast<int>(blockIdx.x) + static_cast<int>(step / p.G) * static_cast<int>(gridDim.x);
                 kb = static_cast<int>(step % p.G);
@@ -260,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                 int kb, w_blk, t_blk;
                 step_coords(e, kb, w_blk, t_blk);
                 ptx::mbar_arrive_expect_tx(&full[e], C::kCBytes + kPBytes);
-                ptx::tma_load_2d(smem + C::kOffC + e * C::kCBytes, &map_codes, &full[e], kb * kCodeWords, w_blk * BW);
+                load_codes(smem + C::kOffC + e * C::kCBytes, &full[e], kb, w_blk);
             }
             ptx::grid_dependency_wait();
             for (uint32_t e = 0; e < early; ++e) {
@@ -281,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                         ptx::tma_load_2d(smem + C::kOffX + s * kXBytes, &map_x, &full[s], kb * BK, t_blk * BT);
                     } else {
                         ptx::mbar_arrive_expect_tx(&full[s], C::kCBytes + kPBytes);
-                        ptx::tma_load_2d(smem + C::kOffC + s * C::kCBytes, &map_codes, &full[s], kb * kCodeWords, w_blk * BW);
+                        load_codes(smem + C::kOffC + s * C::kCBytes, &full[s], kb, w_blk);
                         ptx::tma_load_2d(smem + C::kOffP + s * kPBytes, &map_params, &full[s], w_blk * BW, kb);
                     }
                 }
@@ -337,6 +362,71 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             ptx::mma_commit(drain + gsel);
             ptx::mbar_wait(drain + gsel, 0, nullptr);
         }
+    } else if (kSwiGLU && warp >= kWarpEpi0) {
+        // ---------------------------------------------------------------- SwiGLU epilogue
+        // Warp (quarter, half) reads the gate and up accumulators of TMEM lanes 32*quarter .. +31 (its
+        // 32 intermediate columns) for the token chunks kHalfChunks*half .. +kHalfChunks-1.
+        constexpr int kHalfChunks = BT / 32 / 2;
+        const int quarter = warp & 3;
+        const int half = (warp - kWarpEpi0) >> 2;
+        uint8_t* epi_stage = smem + C::kOffEpi + (warp - kWarpEpi0) * 2 * kStageBytes;
+        uint32_t nstore = 0;
+        int j = 0;
+        ptx::grid_dependency_wait();               // the row scales come from the kernels before this one
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++j) {
+            int t_blk, w_blk;
+            tile_coords(t, p.num_w, t_blk, w_blk);
+            // rs[c] belongs to token t_blk*BT + 32*(kHalfChunks*half + c) + lane
+            float rs[kHalfChunks];
+#pragma unroll
+            for (int c = 0; c < kHalfChunks; ++c) {
+                const int m = t_blk * BT + 32 * (kHalfChunks * half + c) + lane;
+                rs[c] = (m < p.M) ? p.rowscale[m] : 0.0f;
+            }
+            const bool got = ptx::mbar_wait(&acc_full[0], j & 1, abort_flag);
+            if (!__all_sync(0xFFFFFFFFu, got)) break;
+            ptx::tc_fence_after_sync();
+            const int n_base = w_blk * BWG + quarter * 32;      // this warp's 32 intermediate columns
+            const uint32_t tgate = tmem_base + kAccCol + (static_cast<uint32_t>(quarter * 32) << 16);
+            const uint32_t tup = tgate + static_cast<uint32_t>(BT);
+#pragma unroll 1
+            for (int c = 0; c < kHalfChunks; ++c) {
+                const int chunk = kHalfChunks * half + c;
+                uint32_t rg[32], ru[32];
+                ptx::tmem_ld_32x32b_x32(tgate + chunk * 32, rg);
+                ptx::tmem_ld_32x32b_x32(tup + chunk * 32, ru);
+                ptx::tmem_wait_ld();
+                uint8_t* stage = epi_stage + (nstore & 1) * kStageBytes;
+                if (lane == 0) ptx::bulk_wait_group_read<1>();   // the store that used this buffer has read it
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const float sc = __shfl_sync(0xFFFFFFFFu, rs[c], k);
+                    const float gv = __uint_as_float(rg[k]) * sc;
+                    const float uv = __uint_as_float(ru[k]) * sc;
+                    const float h = gv / (1.0f + expf(-gv)) * uv;
+                    if constexpr (kBf16Out) {
+                        reinterpret_cast<__nv_bfloat16*>(stage)[k * 32 + lane] = __float2bfloat16_rn(h);
+                    } else {
+                        reinterpret_cast<float*>(stage)[k * 32 + lane] = h;
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::tma_store_2d(&map_y, stage, n_base, t_blk * BT + chunk * 32);
+                    ptx::bulk_commit_group();
+                }
+                ++nstore;
+            }
+            ptx::tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(&acc_empty[0]);
+                ptx::mbar_arrive(&acc_empty[1]);
+            }
+        }
+        if (lane == 0) ptx::bulk_wait_group_all();   // every store has completed before the CTA exits
     } else if (warp >= kWarpEpi0) {
         // ---------------------------------------------------------------- epilogue
         const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31

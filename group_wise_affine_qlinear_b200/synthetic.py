@@ -151,6 +151,10 @@ class Workload:
             return weights8(self.seed, self.widx, self.N, self.K)
         return weights(self.seed, self.widx, self.N, self.K)
 
+    def w_pair(self):
+        """Gate and up weights of a SwiGLU pair, [N][K] each: weight indices widx and widx + 1."""
+        return weights(self.seed, self.widx, self.N, self.K), weights(self.seed, self.widx + 1, self.N, self.K)
+
 
 WORKLOADS = {
     w.name: w for w in [
@@ -161,6 +165,8 @@ WORKLOADS = {
                  note="DiT SwiGLU up/gate pair (2 x 18432), first 4608 rows imatrix-fitted"),
         Workload("mlp_down", 4608, 18432, 4608, seed=2, widx=1, xidx=1,
                  note="DiT SwiGLU down projection"),
+        Workload("mlp_gate_up_12288", 4608, 4608, 12288, seed=2, widx=2, xidx=0,
+                 note="SwiGLU gate and up projections at the pages' intermediate size 12288 (N = I per weight)"),
         Workload("text_proj", 512, 53248, 4608, seed=3, block_means=True,
                  note="llm_cond_proj 53248->4608; M swept over 1, 8, 32, 512 (leading rows)"),
         Workload("text_proj_w8", 512, 53248, 4608, seed=3, widx=1, block_means=True, bits=8,

@@ -240,6 +240,33 @@ QL_API ql_status qlinear8_dequant(const uint32_t* codes, const void* scales, con
 QL_API ql_status qlinear8_pack(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group,
                                uint32_t* codes, void* scales, void* biases, cudaStream_t stream);
 
+/*
+ * SwiGLU up/gate pair in one call: h = silu(x . W_gate^T) * (x . W_up^T) elementwise, with
+ * silu(z) = z / (1 + e^-z) (the DiT block's MLP is a SwiGLU of three Linears, jimmysue "Ideogram 4"
+ * notes, sec. 2.1 and 2.8; this call covers the first two and the gating, the third is an ordinary
+ * qlinear_forward of h).
+ *
+ *   x                                   bf16 [M][K]
+ *   gate_codes / up_codes               uint32 [I][K/8], 4-bit codes as above
+ *   gate_scales, gate_biases, up_...    f16 [I][K/64]
+ *   h                                   [M][I], bf16 (QL_BF16) or fp32 (QL_F32, for numerical tests)
+ *
+ * Arithmetic of the tcgen05 path (QL_PATH_TC_FUSED): g and u accumulate in fp32 from f16 operands
+ * (weights RN_f16(s * q + b), activations scaled per row by a power of two), then
+ * h = g / (1 + expf(-g)) * u in fp32, rounded once to the output type.  One GEMM computes both: each
+ * tile holds 128 rows of the gate weight and the same 128 rows of the up weight, so g and u of an
+ * output element meet in the epilogue and never travel through memory.
+ * Preconditions as for qlinear_forward with N = I (I % 8 == 0), all eight tensors 16-byte aligned,
+ * h overlapping no input and the workspace overlapping nothing; `workspace` must hold
+ * qlinear_swiglu_workspace_size(M, K, I, group) bytes (QL_ERR_WORKSPACE otherwise).
+ */
+QL_API size_t qlinear_swiglu_workspace_size(int64_t M, int64_t K, int64_t I, int32_t group);
+QL_API ql_status qlinear_swiglu_forward(const void* x, const uint32_t* gate_codes, const void* gate_scales,
+                                        const void* gate_biases, const uint32_t* up_codes,
+                                        const void* up_scales, const void* up_biases, void* h,
+                                        ql_dtype out_dtype, int64_t M, int64_t K, int64_t I, int32_t group,
+                                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Static, human-readable name of a status code. */
 QL_API const char* qlinear_status_string(ql_status status);
 

@@ -155,3 +155,32 @@ def test_workspace_size8_values(L):
     assert ql.workspace_size8(M, K, N, ql.PATH_TC_FUSED) == M * K * 2 + M * 4 + (K // 64) * N * 4
     assert ql.workspace_size8(2, 4096, 64, ql.PATH_GEMV, 4) == 4 * 2 * 64 * 4
     assert L.qlinear8_workspace_size(16, 100, 256, 64) == ctypes.c_size_t(-1).value
+
+
+# ---------------------------------------------------------------- SwiGLU pair
+
+def _sw(L, x=FAKE, gc=FAKE + (1 << 24), gs=FAKE + (2 << 24), gb=FAKE + (3 << 24), uc=FAKE + (5 << 24),
+        us=FAKE + (6 << 24), ub=FAKE + (7 << 24), h=FAKE + (4 << 24), dt=1, M=16, K=256, I=256, group=64,
+        ws=FAKE + (8 << 24), ws_bytes=1 << 24):
+    return L.qlinear_swiglu_forward(x, gc, gs, gb, uc, us, ub, h, dt, M, K, I, group, ws, ws_bytes, None)
+
+
+def test_swiglu_rejects_bad_arguments(L):
+    assert _sw(L, group=32) == 3
+    assert _sw(L, K=100) == 1
+    assert _sw(L, I=12) == 1
+    assert _sw(L, M=0) == 1
+    assert _sw(L, uc=0) == 1
+    assert _sw(L, dt=7) == 1
+    assert _sw(L, ub=FAKE + (7 << 24) + 2) == 2
+    assert _sw(L, h=FAKE + (5 << 24) + 64) == 1          # h inside the up codes
+    assert _sw(L, ws=None, ws_bytes=0) == 4
+    assert _sw(L, ws_bytes=100) == 4
+    assert _sw(L, ws=FAKE + (4 << 24)) == 1              # workspace over h
+
+
+def test_swiglu_workspace_size(L):
+    M, K, I = 4608, 4608, 12288
+    # f16 activations, row scales, and (scale, bias) pairs of 256 interleaved rows per 128-column tile
+    assert ql.swiglu_workspace_size(M, K, I) == M * K * 2 + M * 4 + (K // 64) * ((I + 127) // 128) * 256 * 4
+    assert L.qlinear_swiglu_workspace_size(16, 100, 256, 64) == ctypes.c_size_t(-1).value
