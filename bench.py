@@ -51,8 +51,8 @@ def parse():
     ap.add_argument("--no-pack", action="store_true", help="skip the quantizer (qlinear_pack) measurement")
     ap.add_argument("--swiglu", action="store_true",
                     help="also measure the fused SwiGLU pair on the MLP at the pages' width (I = 12288)")
-    ap.add_argument("--w8", action="store_true",
-                    help="also measure the 8-bit conditioning projection (text_proj_w8) at M = 1, 8, 32")
+    ap.add_argument("--no-w8", action="store_true",
+                    help="skip the 8-bit conditioning projection (text_proj_w8) at M = 1, 8, 32")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     return ap.parse_args()
 
@@ -473,7 +473,7 @@ def main():
         return out
 
     small = [] if a.no_small_m else small_m("text_proj")
-    small_w8 = small_m("text_proj_w8") if a.w8 else []
+    small_w8 = [] if a.no_w8 else small_m("text_proj_w8")
 
     # ---- the quantizer: importance-weighted fit and RTN pack of a DiT-shaped weight
     pack = None if a.no_pack else pack_measure(ql, torch, dev, flush)
