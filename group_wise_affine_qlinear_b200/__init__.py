@@ -38,6 +38,7 @@ from ._lib import (  # noqa: F401
     library_path,
     pack,
     pack8,
+    reduce_partials,
     set_profile_events,
     swiglu,
     swiglu_workspace_size,

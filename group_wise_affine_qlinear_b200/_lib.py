@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.qlinear8_dequant.restype = ctypes.c_int
         L.qlinear8_pack.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp, vp]
         L.qlinear8_pack.restype = ctypes.c_int
+        L.qlinear_reduce_partials.argtypes = [vp, i32, i64, vp, ctypes.c_int, vp]
+        L.qlinear_reduce_partials.restype = ctypes.c_int
         L.qlinear_swiglu_workspace_size.argtypes = [i64, i64, i64, i32]
         L.qlinear_swiglu_workspace_size.restype = sz
         L.qlinear_swiglu_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i32, vp, sz, vp]
@@ -289,6 +291,24 @@ def swiglu(x: torch.Tensor, gate, up, out: torch.Tensor | None = None, workspace
                                     _BF16 if out_dtype == torch.bfloat16 else _F32, M, K, I, GROUP,
                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                     _stream_handle(stream)), "qlinear_swiglu_forward")
+    return out
+
+
+def reduce_partials(partials: torch.Tensor, out: torch.Tensor | None = None, out_dtype=torch.bfloat16,
+                    stream=None) -> torch.Tensor:
+    """Sum fp32 partials [S][...] over S in order, rounded once (qlinear_reduce_partials) -> [...]."""
+    L = lib()
+    if not isinstance(partials, torch.Tensor) or partials.dim() < 2:
+        raise ValueError("partials must be a tensor [S][...]")
+    _need_cuda(partials, "partials", torch.float32)
+    S = partials.shape[0]
+    shape = tuple(partials.shape[1:])
+    if out is None:
+        out = torch.empty(shape, dtype=out_dtype, device=partials.device)
+    _need_cuda(out, "out", out_dtype, shape)
+    _check(L.qlinear_reduce_partials(partials.data_ptr(), S, out.numel(), out.data_ptr(),
+                                     _BF16 if out_dtype == torch.bfloat16 else _F32, _stream_handle(stream)),
+           "qlinear_reduce_partials")
     return out
 
 

@@ -696,6 +696,24 @@ ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t 
     return pack_impl(w, imatrix, K, N, group, codes, scales, biases, stream, 4);
 }
 
+ql_status qlinear_reduce_partials(const float* partials, int32_t S, int64_t count, void* y, ql_dtype out_dtype,
+                                  cudaStream_t stream) {
+    if (!partials || !y || S < 1 || count < 4 || count % 4 != 0) return QL_ERR_INVALID_ARG;
+    if (out_dtype != QL_BF16 && out_dtype != QL_F32) return QL_ERR_INVALID_ARG;
+    if (!aligned16(partials) || !aligned16(y)) return QL_ERR_ALIGNMENT;
+    const size_t yb = static_cast<size_t>(count) * (out_dtype == QL_BF16 ? 2 : 4);
+    if (overlap(y, yb, partials, static_cast<size_t>(S) * count * 4)) return QL_ERR_INVALID_ARG;
+    DeviceInfo* dev = nullptr;
+    ql_status s;
+    if ((s = device_info(&dev)) != QL_OK) return s;
+    const int blocks = static_cast<int>(std::min<int64_t>((count / 4 + 255) / 256, 8 * dev->sm_count));
+    if (out_dtype == QL_BF16)
+        splitk_reduce_kernel<true><<<blocks, 256, 0, stream>>>(partials, y, count, S);
+    else
+        splitk_reduce_kernel<false><<<blocks, 256, 0, stream>>>(partials, y, count, S);
+    return launch_status();
+}
+
 size_t qlinear_swiglu_workspace_size(int64_t M, int64_t K, int64_t I, int32_t group) {
     if (check_shape(M, K, I, group) != QL_OK) return static_cast<size_t>(-1);
     return swiglu_plan(M, K, I).workspace;

@@ -267,6 +267,17 @@ QL_API ql_status qlinear_swiglu_forward(const void* x, const uint32_t* gate_code
                                         ql_dtype out_dtype, int64_t M, int64_t K, int64_t I, int32_t group,
                                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * y[i] = sum_{z=0}^{S-1} partials[z][i], summed in z order in fp32 and rounded once to out_dtype.
+ * partials is fp32 [S][count] (device, read only), y is [count] of out_dtype; count % 4 == 0.
+ * This is the combination step of a K-sharded (row-parallel) layer: the ranks' fp32 partial
+ * outputs (qlinear_forward_config with QL_F32), gathered in rank order, reduce to the same bytes on
+ * every rank.  Errors: QL_ERR_INVALID_ARG (null pointer, S < 1, count not a positive multiple of 4,
+ * y overlapping partials, bad out_dtype), QL_ERR_ALIGNMENT (a pointer not 16-byte aligned).
+ */
+QL_API ql_status qlinear_reduce_partials(const float* partials, int32_t S, int64_t count, void* y,
+                                         ql_dtype out_dtype, cudaStream_t stream);
+
 /* Static, human-readable name of a status code. */
 QL_API const char* qlinear_status_string(ql_status status);
 

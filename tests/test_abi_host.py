@@ -184,3 +184,12 @@ def test_swiglu_workspace_size(L):
     # f16 activations, row scales, and (scale, bias) pairs of 256 interleaved rows per 128-column tile
     assert ql.swiglu_workspace_size(M, K, I) == M * K * 2 + M * 4 + (K // 64) * ((I + 127) // 128) * 256 * 4
     assert L.qlinear_swiglu_workspace_size(16, 100, 256, 64) == ctypes.c_size_t(-1).value
+
+
+def test_reduce_partials_validation(L):
+    assert L.qlinear_reduce_partials(None, 2, 64, FAKE, 1, None) == 1
+    assert L.qlinear_reduce_partials(FAKE, 0, 64, FAKE + (1 << 24), 1, None) == 1
+    assert L.qlinear_reduce_partials(FAKE, 2, 66, FAKE + (1 << 24), 1, None) == 1     # not a multiple of 4
+    assert L.qlinear_reduce_partials(FAKE, 2, 64, FAKE + (1 << 24), 5, None) == 1
+    assert L.qlinear_reduce_partials(FAKE + 4, 2, 64, FAKE + (1 << 24), 1, None) == 2
+    assert L.qlinear_reduce_partials(FAKE, 2, 64, FAKE + 256, 1, None) == 1           # y inside the partials
