@@ -336,7 +336,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                     if (!ptx::mbar_wait(&a_full[as], aph, abort_flag)) { ok = false; break; }
                     ptx::tc_fence_after_sync();
                     const uint32_t x_addr = ptx::smem_addr(smem + C::kOffX + xs * kXBytes);
-#pragma unroll
                     {
                         const int g = gsel;
                         if (kb == 0) {
