@@ -4,6 +4,9 @@ h = silu(x . W_gate^T) * (x . W_up^T) from one call that runs both projections i
 GEMM and gates in its epilogue.  Small ragged shapes against the full oracle, one-hot rows that pin
 the pairing of gate and up rows to one bf16 ulp, and sampled rows of the pages' MLP width
 (K = 4608, I = 12288, M = 4608).
+
+The file sorts after the other GPU parity files, so that a run stopping at its first failure has
+already checked every older path.
 """
 import numpy as np
 import pytest
