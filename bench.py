@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-pack", action="store_true", help="skip the quantizer (qlinear_pack) measurement")
     ap.add_argument("--swiglu", action="store_true",
                     help="also measure the fused SwiGLU pair on the MLP at the pages' width (I = 12288)")
+    ap.add_argument("--no-comparators", action="store_true",
+                    help="skip the cuBLAS context measurements (dense bf16 and dequant-then-matmul)")
     ap.add_argument("--no-w8", action="store_true",
                     help="skip the 8-bit conditioning projection (text_proj_w8) at M = 1, 8, 32")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -168,6 +170,54 @@ def swiglu_measure(ql, torch, dev, flush, peak_tf, steps=10):
     return {"workload": f"{w.name} M={w.M} K={w.K} I={w.N} (gate + up)", "dispatch": dispatch,
             "step_ms": call, "kernel_ms": main, "TFLOPs": flops / (call * 1e-3) / 1e12,
             "kernel_TFLOPs": flops / (main * 1e-3) / 1e12, "kernel_frac": flops / (main * 1e-3) / 1e12 / peak_tf}
+
+
+def comparators(ql, torch, dev, flush, steps=10):
+    """Context, not targets: the same layers through cuBLAS (torch.matmul) on this machine.
+
+    dense: a bf16 copy of W (made once by qlinear_dequant) times x, the unquantized layer's GEMM;
+    dequant_then_matmul: qlinear_dequant to bf16 every step, then the same GEMM, the way a packed
+    layer runs when it only has a library GEMM.  L2 is flushed before every step.
+    """
+    out = {}
+    for name, Ms in (("qkv", None), ("text_proj", 32)):
+        w = S.WORKLOADS[name]
+        M = Ms or w.M
+        x = torch.from_numpy(w.x(M).view(np.int16)).view(torch.bfloat16).to(dev)
+        c, s, b = w.w()
+        cd = torch.from_numpy(c.view(np.int32)).to(dev)
+        sd, bd = torch.from_numpy(s).to(dev), torch.from_numpy(b).to(dev)
+        wb = ql.dequant(cd, sd, bd, out_dtype=torch.bfloat16)
+        wtmp = torch.empty_like(wb)
+        y = torch.empty((M, w.N), dtype=torch.bfloat16, device=dev)
+
+        def dense():
+            torch.matmul(x, wb.t(), out=y)
+
+        def deq_mm():
+            torch.matmul(x, ql.dequant(cd, sd, bd, out_dtype=torch.bfloat16, out=wtmp).t(), out=y)
+
+        res = {}
+        for key, fn in (("dense_bf16_matmul", dense), ("dequant_then_matmul", deq_mm)):
+            for _ in range(3):
+                flush.fill_(1)
+                fn()
+            torch.cuda.synchronize()
+            ms = []
+            for i in range(steps):
+                flush.fill_(i & 0xFF)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                ms.append(e0.elapsed_time(e1))
+            mean = sum(ms) / steps
+            res[key] = {"ms": mean, "TFLOPs": 2.0 * M * w.K * w.N / (mean * 1e-3) / 1e12}
+        out[f"{name} M={M} K={w.K} N={w.N}"] = res
+        del wb, wtmp, x, y, cd, sd, bd
+        torch.cuda.empty_cache()
+    return out
 
 
 def oracle_fit_rate(rows=4):
@@ -478,6 +528,12 @@ def main():
     # ---- the quantizer: importance-weighted fit and RTN pack of a DiT-shaped weight
     pack = None if a.no_pack else pack_measure(ql, torch, dev, flush)
     swiglu = swiglu_measure(ql, torch, dev, flush, peaks()[0]) if a.swiglu else None
+    comp = None
+    if not a.no_comparators:
+        try:                            # context only: never let it cost the measured line
+            comp = comparators(ql, torch, dev, flush)
+        except Exception as exc:        # noqa: BLE001
+            comp = {"error": f"{type(exc).__name__}: {exc}"[:200]}
 
     mean_step, mean_main, mean_e2e = max_over_ranks([mean_step, mean_main, mean_e2e], dev)
 
@@ -521,6 +577,8 @@ def main():
         line["small_m_w8"] = small_w8
     if swiglu is not None:
         line["swiglu"] = swiglu
+    if comp is not None:
+        line["comparators"] = comp
     if pack is not None:
         line["pack"] = pack
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
