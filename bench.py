@@ -565,6 +565,7 @@ def main():
         "ms_per_step": mean_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16 MMA, fp32 accumulate (bf16 in/out)", "data": "synthetic",
         "config": {"workload": f"{w.name} M={M} K={K} N={N}", "seed": w.seed,
+                   "inputs_sha256": S.digest(case.x_np, case.codes_np, case.s_np, case.b_np),
                    "l2": "flushed between steps (512 MiB write)", "parallelism": f"replicas x{world}",
                    "dispatch": dispatch, "weight_GBps": w.weight_bytes / (mean_step * 1e-3) / 1e9},
         "roofline": roof,
