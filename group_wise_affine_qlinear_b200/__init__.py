@@ -39,6 +39,7 @@ from ._lib import (  # noqa: F401
     pack,
     pack8,
     reduce_partials,
+    selftest_bounded_wait,
     set_profile_events,
     swiglu,
     swiglu_workspace_size,

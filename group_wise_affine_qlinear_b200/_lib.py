@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.qlinear8_dequant.restype = ctypes.c_int
         L.qlinear8_pack.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp, vp]
         L.qlinear8_pack.restype = ctypes.c_int
+        L.qlinear_selftest_bounded_wait.argtypes = [vp]
+        L.qlinear_selftest_bounded_wait.restype = ctypes.c_int
         L.qlinear_reduce_partials.argtypes = [vp, i32, i64, vp, ctypes.c_int, vp]
         L.qlinear_reduce_partials.restype = ctypes.c_int
         L.qlinear_swiglu_workspace_size.argtypes = [i64, i64, i64, i32]
@@ -310,6 +312,11 @@ def reduce_partials(partials: torch.Tensor, out: torch.Tensor | None = None, out
                                      _BF16 if out_dtype == torch.bfloat16 else _F32, _stream_handle(stream)),
            "qlinear_reduce_partials")
     return out
+
+
+def selftest_bounded_wait(stream=None) -> None:
+    """Enqueue the bounded-wait self-test (qlinear_selftest_bounded_wait); device_status() then reads 6."""
+    _check(lib().qlinear_selftest_bounded_wait(_stream_handle(stream)), "qlinear_selftest_bounded_wait")
 
 
 def device_status(stream=None) -> int:

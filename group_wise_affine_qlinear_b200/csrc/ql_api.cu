@@ -20,6 +20,24 @@
 #include "ql_tc_skinny.cuh"
 
 namespace ql {
+
+// Self-test of the bounded waits every pipeline role uses: one CTA, two waiting threads (lane 0 of
+// warps 0 and 1) on an mbarrier that nothing arrives on.  One of them gives up after the wait limit,
+// records QL_ERR_DEVICE_TIMEOUT and raises the shared abort flag; the other returns on that flag
+// (or on its own limit).  The kernel ends about one wait limit after it starts.
+__global__ void __launch_bounds__(64) wait_selftest_kernel() {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bar, 1);
+        abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) ptx::mbar_wait(&bar, 0, &abort_flag);   // phase 0 never completes
+    __syncthreads();
+}
+
 namespace {
 
 constexpr int32_t kVersion = 100;   // 0.1.0
@@ -694,6 +712,11 @@ ql_status qlinear_dequant(const uint32_t* codes, const void* scales, const void*
 ql_status qlinear_pack(const float* w, const float* imatrix, int64_t K, int64_t N, int32_t group, uint32_t* codes,
                        void* scales, void* biases, cudaStream_t stream) {
     return pack_impl(w, imatrix, K, N, group, codes, scales, biases, stream, 4);
+}
+
+ql_status qlinear_selftest_bounded_wait(cudaStream_t stream) {
+    wait_selftest_kernel<<<1, 64, 0, stream>>>();
+    return launch_status();
 }
 
 ql_status qlinear_reduce_partials(const float* partials, int32_t S, int64_t count, void* y, ql_dtype out_dtype,

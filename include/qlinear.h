@@ -278,6 +278,15 @@ QL_API ql_status qlinear_swiglu_forward(const void* x, const uint32_t* gate_code
 QL_API ql_status qlinear_reduce_partials(const float* partials, int32_t S, int64_t count, void* y,
                                          ql_dtype out_dtype, cudaStream_t stream);
 
+/*
+ * Self-test of the bounded waits inside the library's kernels.  Enqueues one small kernel that waits
+ * on a barrier nothing ever completes, with the same bounded wait every pipeline role uses: it gives
+ * up after the library's wait limit (about one second), records QL_ERR_DEVICE_TIMEOUT in the device
+ * status word and returns, leaving the context usable.  A following qlinear_get_device_status()
+ * therefore returns QL_ERR_DEVICE_TIMEOUT.  Returns QL_ERR_CUDA if the launch fails.
+ */
+QL_API ql_status qlinear_selftest_bounded_wait(cudaStream_t stream);
+
 /* Static, human-readable name of a status code. */
 QL_API const char* qlinear_status_string(ql_status status);
 

@@ -52,3 +52,24 @@ def _rank_main(rank, world, port):
 
 def test_row_parallel_gather_two_ranks():
     mp.spawn(_rank_main, args=(2, _free_port()), nprocs=2, join=True)
+
+
+def _rank_leaves(rank, world, port, result_dir):
+    from datetime import timedelta
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=timedelta(seconds=10))
+    if rank == 1:
+        return                                  # leaves between steps: never joins the gather
+    outcome = "returned"
+    try:
+        tp.gather_partials(torch.zeros(4, 8))
+    except Exception as exc:                    # noqa: BLE001
+        outcome = "raised " + type(exc).__name__
+    with open(os.path.join(result_dir, "rank0"), "w") as f:
+        f.write(outcome)
+
+
+def test_row_parallel_gather_fails_when_a_rank_leaves(tmp_path):
+    """A rank that leaves before the exchange ends the other rank's gather with an error (no hang)."""
+    mp.spawn(_rank_leaves, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True)
+    assert (tmp_path / "rank0").read_text().startswith("raised ")
