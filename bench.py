@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--M", type=int, default=0, help="override the token count (0 = the workload's)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", type=int, default=0, help="force a kernel path (0 = dispatcher's choice)")
+    ap.add_argument("--split", type=int, default=0, help="force the split-K factor (0 = dispatcher's choice)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-m", action="store_true", help="skip the small-M weight-streaming measurements")
     ap.add_argument("--no-pack", action="store_true", help="skip the quantizer (qlinear_pack) measurement")
@@ -363,9 +364,10 @@ def whole_job_rate(work_per_rank: float, slowest_ms: float, world: int) -> float
 class Case:
     """Device-resident inputs of one workload and timed qlinear_forward steps on them."""
 
-    def __init__(self, ql, torch, w, M, path, dev, flush):
+    def __init__(self, ql, torch, w, M, path, dev, flush, split=0):
         import numpy as np
         self.ql, self.torch, self.w, self.M, self.path, self.flush = ql, torch, w, M, path, flush
+        self.split = split
         self.K, self.N = w.K, w.N
         self.x_np = w.x(M)
         self.codes_np, self.s_np, self.b_np = w.w()
@@ -374,12 +376,13 @@ class Case:
         self.sc = torch.from_numpy(self.s_np).to(dev)
         self.bi = torch.from_numpy(self.b_np).to(dev)
         self.y = torch.empty((M, self.N), dtype=torch.bfloat16, device=dev)
-        ws_bytes = ql.workspace_size(M, self.K, self.N, path, bits=w.bits)
+        ws_bytes = ql.workspace_size(M, self.K, self.N, path, split, bits=w.bits)
         self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
         self.fwd = ql.forward8 if w.bits == 8 else ql.forward
 
     def step(self):
-        self.fwd(self.x, self.codes, self.sc, self.bi, out=self.y, workspace=self.ws, path=self.path)
+        self.fwd(self.x, self.codes, self.sc, self.bi, out=self.y, workspace=self.ws, path=self.path,
+                 split_k=self.split)
 
     def warm(self, n):
         for _ in range(n):
@@ -451,7 +454,7 @@ def main():
     w = S.WORKLOADS[a.workload]
     M = a.M or w.M
     K, N = w.K, w.N
-    case = Case(ql, torch, w, M, a.path, dev, flush)
+    case = Case(ql, torch, w, M, a.path, dev, flush, a.split)
     case.warm(a.warmup)
 
     # ---- device-timed steps (inputs resident; L2 flushed between steps)
@@ -496,7 +499,8 @@ def main():
         if i >= 2:
             s_c.wait_event(out_done[i - 2])             # step i-2's y buffer has been copied out
         flush.fill_(i & 0xFF)
-        case.fwd(xb[b], case.codes, case.sc, case.bi, out=yb[b], workspace=case.ws, path=case.path)
+        case.fwd(xb[b], case.codes, case.sc, case.bi, out=yb[b], workspace=case.ws, path=case.path,
+                 split_k=case.split)
         comp_done[i].record(s_c)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[i])

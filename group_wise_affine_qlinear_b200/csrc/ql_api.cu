@@ -97,7 +97,12 @@ ql_status device_info(DeviceInfo** out) {
     }
     if (!d.fused_attr_set) {
         if (fused_smem_attr<fused::DefaultCfg>() != cudaSuccess || fused_smem_attr<fused::Q8Cfg>() != cudaSuccess ||
-            fused_smem_attr<fused::DefaultCfg, true>() != cudaSuccess)
+            fused_smem_attr<fused::DefaultCfg, true>() != cudaSuccess ||
+            cudaFuncSetAttribute(fused::fused_gemm_kernel<false, fused::DefaultCfg, false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 fused::DefaultCfg::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(fused::fused_gemm_kernel<false, fused::Q8Cfg, false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, fused::Q8Cfg::kSmemBytes) != cudaSuccess)
             return QL_ERR_CUDA;
         d.fused_attr_set = true;
     }
@@ -142,6 +147,21 @@ ql_status encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, 
     return r == CUDA_SUCCESS ? QL_OK : QL_ERR_CUDA;
 }
 
+// 3-D row-major tensor map: extents (cols, rows, planes) in elements, row and plane pitches in bytes.
+ql_status encode_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t cols, uint64_t rows,
+                    uint64_t planes, uint64_t row_pitch, uint64_t plane_pitch, uint32_t box_cols, uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    if (get_encoder(&enc) != QL_OK) return QL_ERR_CUDA;
+    const cuuint64_t dims[3] = {cols, rows, planes};
+    const cuuint64_t strides[2] = {row_pitch, plane_pitch};
+    const cuuint32_t box[3] = {box_cols, box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? QL_OK : QL_ERR_CUDA;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool overlap(const void* a, size_t na, const void* b, size_t nb) {
@@ -176,8 +196,8 @@ struct Plan {
     int ctas = 0, segmax = 0, nt = 0;
     int64_t units = 0;
     size_t workspace = 0;
-    // fused path workspace carve-up
-    size_t off_xh = 0, off_rs = 0, off_sb = 0;
+    // fused path workspace carve-up (off_part: fp32 partials [split_k][M][N] when the K-steps are split)
+    size_t off_xh = 0, off_rs = 0, off_sb = 0, off_part = 0;
     // skinny path workspace carve-up: partials, scaled f16 activations, row exponents, per-slice row maxima
     size_t off_xp = 0, off_re = 0, off_pm = 0;
     int slices = 0;
@@ -213,12 +233,14 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         return QL_OK;
     }
     if (path == QL_PATH_TC_FUSED) {
-        if (split_k > 1) return QL_ERR_UNSUPPORTED;
-        plan->split_k = 1;
+        if (split_k > G || split_k > 1024) return QL_ERR_INVALID_ARG;
+        plan->split_k = split_k > 1 ? split_k : 1;
         plan->off_xh = 0;
         plan->off_rs = round_up(static_cast<size_t>(M) * K * 2, 256);
         plan->off_sb = plan->off_rs + round_up(static_cast<size_t>(M) * 4, 256);
-        plan->workspace = plan->off_sb + round_up(static_cast<size_t>(G) * N * 4, 256);
+        plan->off_part = plan->off_sb + round_up(static_cast<size_t>(G) * N * 4, 256);
+        plan->workspace = plan->off_part;
+        if (plan->split_k > 1) plan->workspace += round_up(static_cast<size_t>(plan->split_k) * M * N * 4, 256);
         return QL_OK;
     }
     return QL_ERR_UNSUPPORTED;
@@ -303,9 +325,17 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
                        CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
         return s;
     CUtensorMap my;
-    if ((s = encode_2d(&my, bf16_out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, y, N, M,
-                       N * (bf16_out ? 2 : 4), 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+    const bool split = pl.split_k > 1;
+    float* part = reinterpret_cast<float*>(base + pl.off_part);
+    if (split) {
+        // fp32 partials [split_k][M][N]: 32 x 32 blocks, clipped at M and N within every slice
+        if ((s = encode_3d(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, part, N, M, pl.split_k, N * 4,
+                           static_cast<uint64_t>(M) * N * 4, 32, 32)) != QL_OK)
+            return s;
+    } else if ((s = encode_2d(&my, bf16_out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, y, N,
+                              M, N * (bf16_out ? 2 : 4), 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK) {
         return s;
+    }
 
     if (bits == 4)
         convert_x_kernel<4><<<static_cast<unsigned>(M), kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), xh,
@@ -328,10 +358,31 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     p.G = static_cast<int>(G);
     p.num_t = static_cast<int>((M + fused::BT - 1) / fused::BT);
     p.num_w = static_cast<int>((N + fused::BW - 1) / fused::BW);
+    p.splits = pl.split_k;
     const int tiles = p.num_t * p.num_w;
-    const int grid = std::min(tiles, sm_count);
+    const int grid = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(tiles) * pl.split_k, sm_count));
     prof_begin(st);
     const dim3 fgrid(static_cast<unsigned>(grid));
+    if (split) {
+        s = bits == 4 ? launch_dependent(fused::fused_gemm_kernel<false, fused::DefaultCfg, false, true>, fgrid,
+                                         fused::kThreads, fused::DefaultCfg::kSmemBytes, st, mx, mc, mc, mp, my, p)
+                      : launch_dependent(fused::fused_gemm_kernel<false, fused::Q8Cfg, false, true>, fgrid,
+                                         fused::kThreads, fused::Q8Cfg::kSmemBytes, st, mx, mc, mc, mp, my, p);
+        if (s != QL_OK) return s;
+        prof_end(st);
+        // ordered sum of the slices, rounded once (a plain launch: it reads what the kernel above wrote)
+        const int64_t count = M * N;
+        const int blocks = static_cast<int>(std::min<int64_t>((count / 4 + 255) / 256, 8 * sm_count));
+        if (bf16_out)
+            splitk_reduce_kernel<true><<<blocks, 256, 0, st>>>(part, y, count, pl.split_k);
+        else
+            splitk_reduce_kernel<false><<<blocks, 256, 0, st>>>(part, y, count, pl.split_k);
+        const int nc = bits == 4 ? fused::DefaultCfg::kNC : fused::Q8Cfg::kNC;
+        const int nx = bits == 4 ? fused::DefaultCfg::kNX : fused::Q8Cfg::kNX;
+        set_dispatch("path=tc_fused bits=%d tile=%dw x %dt x %dk stages=x%d/c%d/a%d ctas=%d splitk=%d launches=4",
+                     bits, fused::BW, fused::BT, fused::BK, nx, nc, fused::NA, grid, pl.split_k);
+        return launch_status();
+    }
     if (bits == 4) {
         using FC = fused::DefaultCfg;
         s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
@@ -514,6 +565,7 @@ ql_status run_swiglu(const SwigluPlan& pl, const void* x, const uint32_t* gc, co
     p.G = static_cast<int>(G);
     p.num_t = static_cast<int>((M + fused::BT - 1) / fused::BT);
     p.num_w = pl.num_w;
+    p.splits = 1;
     const int tiles = p.num_t * p.num_w;
     const int grid = std::min(tiles, sm_count);
     using FC = fused::DefaultCfg;

@@ -109,6 +109,7 @@ struct Params {
     void* y;              // [M][N] bf16 or fp32
     int M, N, G;
     int num_t, num_w;     // token tiles, weight tiles
+    int splits;           // K slices per tile (split-K instantiations; 1 otherwise)
 };
 
 __device__ __forceinline__ void tile_coords(int t, int num_w, int& t_blk, int& w_blk) {
@@ -126,13 +127,17 @@ __device__ __forceinline__ void ring_pos(uint32_t i, int& stage, uint32_t& phase
 }
 
 // map_codes2: the up weight's codes in SwiGLU mode (128-row boxes, like map_codes there); unused otherwise.
-template <bool kBf16Out, class C, bool kSwiGLU = false>
+// kSplitK: every tile's K-steps are cut into p.splits slices, each its own work unit; a unit writes the
+// fp32 partial of its slice through map_y, a 3-D map over partials [splits][M][N], and a separate
+// reduction sums the slices in order (for shapes with fewer tiles than SMs).
+template <bool kBf16Out, class C, bool kSwiGLU = false, bool kSplitK = false>
 __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
     const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
     const __grid_constant__ CUtensorMap map_codes2, const __grid_constant__ CUtensorMap map_params,
     const __grid_constant__ CUtensorMap map_y, const Params p) {
     constexpr int NX = C::kNX, NC = C::kNC;
     static_assert(!kSwiGLU || C::kBits == 4, "the SwiGLU pair is built for 4-bit codes");
+    static_assert(!kSplitK || (!kSwiGLU && !kBf16Out), "split-K units write fp32 partials of a plain layer");
     constexpr int kCodeWords = BK * C::kBits / 32;      // 32-bit code words of one row per K-step
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -152,10 +157,36 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int num_tiles = p.num_t * p.num_w;
-    // K-steps this CTA runs in total (its tiles times G); every ring position is a function of the step index.
-    const uint32_t my_tiles = blockIdx.x < static_cast<unsigned>(num_tiles)
-                                  ? (static_cast<uint32_t>(num_tiles) - 1u - blockIdx.x) / gridDim.x + 1u : 0u;
-    const uint32_t total_steps = my_tiles * static_cast<uint32_t>(p.G);
+    // Work units: a tile, or with kSplitK a (K slice, tile) pair, slice-major so that a wave of CTAs still
+    // shares activation row blocks.  Unit u covers the K-steps [kb0, kb1) of tile t.
+    const int num_units = kSplitK ? num_tiles * p.splits : num_tiles;
+    auto unit = [&](int u, int& t, int& kb0, int& kb1) {
+        if constexpr (kSplitK) {
+            const int z = u / num_tiles;
+            t = u - z * num_tiles;
+            kb0 = static_cast<int>((static_cast<int64_t>(z) * p.G) / p.splits);
+            kb1 = static_cast<int>((static_cast<int64_t>(z + 1) * p.G) / p.splits);
+        } else {
+            t = u;
+            kb0 = 0;
+            kb1 = p.G;
+        }
+    };
+    // K-steps this CTA runs in total (the sum over its units); every ring position is a function of the
+    // step index.
+    uint32_t total_steps;
+    if constexpr (kSplitK) {
+        total_steps = 0;
+        for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+            int t, kb0, kb1;
+            unit(u, t, kb0, kb1);
+            total_steps += static_cast<uint32_t>(kb1 - kb0);
+        }
+    } else {
+        const uint32_t my_tiles = blockIdx.x < static_cast<unsigned>(num_tiles)
+                                      ? (static_cast<uint32_t>(num_tiles) - 1u - blockIdx.x) / gridDim.x + 1u : 0u;
+        total_steps = my_tiles * static_cast<uint32_t>(p.G);
+    }
 
     if (threadIdx.x == 0) {
         // x and A stages are released by both MMA warps' commits
@@ -263,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             // The activations and the parameter pairs come from the kernels before this one on the
             // stream (programmatic dependent launch): the code loads of the first NC stages go out
             // at once, their parameter loads (same stage barrier) once those kernels are done.
-            const uint32_t first_steps = static_cast<uint32_t>(p.G) * static_cast<uint32_t>(
+            const uint32_t first_steps = kSplitK ? total_steps : static_cast<uint32_t>(p.G) * static_cast<uint32_t>(
                 (num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x));
             const uint32_t early = is_x ? 0u : min(static_cast<uint32_t>(NC), first_steps);
             // one K-step of a tile's codes: 256 rows of one weight, or in SwiGLU mode 128 gate rows
@@ -277,9 +308,22 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                 }
             };
             auto step_coords = [&](uint32_t step, int& kb, int& w_blk, int& t_blk) {
-                const int t = static_cast<int>(blockIdx.x) + static_cast<int>(step / p.G) * static_cast<int>(gridDim.x);
-                kb = static_cast<int>(step % p.G);
-                tile_coords(t, p.num_w, t_blk, w_blk);
+                if constexpr (kSplitK) {
+                    // walk this CTA's units to the one holding its step-th K-step
+                    int u = static_cast<int>(blockIdx.x), t, kb0, kb1;
+                    unit(u, t, kb0, kb1);
+                    while (step >= static_cast<uint32_t>(kb1 - kb0)) {
+                        step -= static_cast<uint32_t>(kb1 - kb0);
+                        u += static_cast<int>(gridDim.x);
+                        unit(u, t, kb0, kb1);
+                    }
+                    kb = kb0 + static_cast<int>(step);
+                    tile_coords(t, p.num_w, t_blk, w_blk);
+                } else {
+                    const int t = static_cast<int>(blockIdx.x) + static_cast<int>(step / p.G) * static_cast<int>(gridDim.x);
+                    kb = static_cast<int>(step % p.G);
+                    tile_coords(t, p.num_w, t_blk, w_blk);
+                }
             };
             for (uint32_t e = 0; e < early; ++e) {       // fresh stages: no empty wait
                 int kb, w_blk, t_blk;
@@ -293,10 +337,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                 step_coords(e, kb, w_blk, t_blk);
                 ptx::tma_load_2d(smem + C::kOffP + e * kPBytes, &map_params, &full[e], w_blk * BW, kb);
             }
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            for (int un = blockIdx.x; un < num_units && ok; un += gridDim.x) {
+                int t, kb0, kb1;
+                unit(un, t, kb0, kb1);
                 int t_blk, w_blk;
                 tile_coords(t, p.num_w, t_blk, w_blk);
-                for (int kb = 0; kb < p.G; ++kb, ++i) {
+                for (int kb = kb0; kb < kb1; ++kb, ++i) {
                     if (i < early) continue;
                     const int s = static_cast<int>(i % depth);
                     const uint32_t ph = (i / depth) & 1u;
@@ -326,8 +372,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             uint32_t i = 0;
             bool ok = true;
             int j = 0;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++j) {
-                for (int kb = 0; kb < p.G; ++kb, ++i) {
+            for (int un = blockIdx.x; un < num_units && ok; un += gridDim.x, ++j) {
+                int t, kb0, kb1;
+                unit(un, t, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb, ++i) {
                     int xs, as;
                     uint32_t xph, aph;
                     ring_pos<NX>(i, xs, xph);
@@ -338,8 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                     const uint32_t x_addr = ptx::smem_addr(smem + C::kOffX + xs * kXBytes);
                     {
                         const int g = gsel;
-                        if (kb == 0) {
-                            // the previous tile's group-g results must have been drained
+                        if (kb == kb0) {
+                            // the previous unit's group-g results must have been drained
                             if (!ptx::mbar_wait(&acc_empty[g], (j & 1) ^ 1, abort_flag)) { ok = false; break; }
                             ptx::tc_fence_after_sync();
                         }
@@ -348,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
 #pragma unroll
                         for (int u = 0; u < BK / UK; ++u) {
                             ptx::mma_f16_ts(d, a_tm + u * (UK / 2), ptx::sdesc_sw128(x_addr + u * UK * 2), idesc,
-                                            (kb | u) != 0);
+                                            ((kb - kb0) | u) != 0);
                         }
                     }
                     if (!ok) break;
@@ -388,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             const int n_base = w_blk * BWG + quarter * 32;      // this warp's 32 intermediate columns
             const uint32_t tgate = tmem_base + kAccCol + (static_cast<uint32_t>(quarter * 32) << 16);
             const uint32_t tup = tgate + static_cast<uint32_t>(BT);
-#pragma unroll 1
+#pragma unroll
             for (int c = 0; c < kHalfChunks; ++c) {
                 const int chunk = kHalfChunks * half + c;
                 uint32_t rg[32], ru[32];
@@ -434,7 +482,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         uint32_t nstore = 0;
         int j = 0;
         ptx::grid_dependency_wait();               // the row scales come from the kernels before this one
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++j) {
+        for (int un = blockIdx.x; un < num_units; un += gridDim.x, ++j) {
+            int t, kb0, kb1;
+            unit(un, t, kb0, kb1);
             int t_blk, w_blk;
             tile_coords(t, p.num_w, t_blk, w_blk);
             // Row scales of the tile's tokens, fetched before the accumulators are ready:
@@ -476,7 +526,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                     ptx::fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        ptx::tma_store_2d(&map_y, stage, n_base, t_blk * BT + chunk * 32);
+                        if constexpr (kSplitK) {
+                            ptx::tma_store_3d(&map_y, stage, n_base, t_blk * BT + chunk * 32, un / num_tiles);
+                        } else {
+                            ptx::tma_store_2d(&map_y, stage, n_base, t_blk * BT + chunk * 32);
+                        }
                         ptx::bulk_commit_group();
                     }
                     ++nstore;

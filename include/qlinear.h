@@ -104,6 +104,9 @@ QL_API ql_status qlinear_forward(const void* x, const uint32_t* codes, const voi
  * groups [z*G/split_k, (z+1)*G/split_k), G = K/64.
  * out_dtype: QL_BF16 = the layer's output; QL_F32 writes y as fp32 [M][N]
  * (the same arithmetic without the final rounding, for numerical tests).
+ * Split-K: QL_PATH_GEMV and QL_PATH_TC_FUSED take split_k > 1 (the fused path then writes one fp32
+ * partial per slice into the workspace and sums them in slice order, for shapes with fewer output
+ * tiles than SMs); QL_PATH_TC_SKINNY balances K itself and returns QL_ERR_UNSUPPORTED for it.
  * A path that cannot run the shape returns QL_ERR_UNSUPPORTED.
  */
 QL_API ql_status qlinear_forward_config(const void* x, const uint32_t* codes, const void* scales,

@@ -193,3 +193,11 @@ def test_reduce_partials_validation(L):
     assert L.qlinear_reduce_partials(FAKE, 2, 64, FAKE + (1 << 24), 5, None) == 1
     assert L.qlinear_reduce_partials(FAKE + 4, 2, 64, FAKE + (1 << 24), 1, None) == 2
     assert L.qlinear_reduce_partials(FAKE, 2, 64, FAKE + 256, 1, None) == 1           # y inside the partials
+
+
+def test_fused_split_k_workspace(L):
+    """The fused path's split-K adds fp32 partials [S][M][N] to its workspace; more slices than groups is an error."""
+    M, K, N = 512, 53248, 4608
+    base = ql.workspace_size(M, K, N, ql.PATH_TC_FUSED)
+    assert ql.workspace_size(M, K, N, ql.PATH_TC_FUSED, 8) == base + 8 * M * N * 4
+    assert L.qlinear_workspace_size_config(16, 256, 256, 64, ql.PATH_TC_FUSED, 5) == ctypes.c_size_t(-1).value
