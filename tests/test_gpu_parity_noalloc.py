@@ -3,9 +3,8 @@
 It serves callers that cannot allocate device memory where they run the layer
 (an engine plugin confined to someone else's memory pool, a serving loop that
 must not allocate after start-up, a runtime that supplies no workspace): its
-split-K scratch is a fixed array inside the library.  This file sorts last so
-a run that stops at the first failure has already run every other test; it
-also passes alone in a fresh process, where its first call performs the
+split-K scratch is a fixed array inside the library.  The tests pass in any
+order, and alone in a fresh process, where the first call performs the
 per-device set-up of the array's address.
 """
 import ctypes
