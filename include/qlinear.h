@@ -100,7 +100,7 @@ QL_API ql_status qlinear_forward(const void* x, const uint32_t* codes, const voi
 /*
  * qlinear_forward with the path and split-K factor forced (testing and tuning).
  * path: a ql_path; split_k: 0 = the dispatcher's choice, else the number of K
- * slices, 1 <= split_k <= K/64 (QL_ERR_INVALID_ARG otherwise); slice z covers the
+ * slices, 1 <= split_k <= K/64 (and <= 1024 on the fused path; QL_ERR_INVALID_ARG otherwise); slice z covers the
  * groups [z*G/split_k, (z+1)*G/split_k), G = K/64.
  * out_dtype: QL_BF16 = the layer's output; QL_F32 writes y as fp32 [M][N]
  * (the same arithmetic without the final rounding, for numerical tests).
@@ -162,8 +162,8 @@ QL_API ql_status qlinear_get_device_status(cudaStream_t stream);
 
 /*
  * Writes a NUL-terminated description of the calling thread's last
- * qlinear_forward dispatch, e.g. "path=tc_fused tile=128x256x64 stages=4/3 ctas=148
- * splitk=1 launches=3" (launches = kernels that call enqueued),
+ * qlinear_forward dispatch, e.g. "path=tc_fused bits=4 tile=256w x 192t x 64k stages=x4/c6/a2
+ * ctas=148 splitk=1 launches=3" (launches = kernels that call enqueued),
  * truncated to len bytes.  QL_ERR_INVALID_ARG if buf is NULL or len == 0.
  */
 QL_API ql_status qlinear_last_dispatch(char* buf, size_t len);
