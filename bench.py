@@ -50,8 +50,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-m", action="store_true", help="skip the small-M weight-streaming measurements")
     ap.add_argument("--no-pack", action="store_true", help="skip the quantizer (qlinear_pack) measurement")
-    ap.add_argument("--swiglu", action="store_true",
-                    help="also measure the fused SwiGLU pair on the MLP at the pages' width (I = 12288)")
+    ap.add_argument("--no-swiglu", action="store_true",
+                    help="skip the fused SwiGLU pair on the MLP at the pages' width (I = 12288)")
+    ap.add_argument("--no-split", action="store_true",
+                    help="skip the text projection at M = 512 on the fused path with and without split-K")
     ap.add_argument("--no-comparators", action="store_true",
                     help="skip the cuBLAS context measurements (dense bf16 and dequant-then-matmul)")
     ap.add_argument("--no-w8", action="store_true",
@@ -219,6 +221,33 @@ def comparators(ql, torch, dev, flush, steps=10):
         del wb, wtmp, x, y, cd, sd, bd
         torch.cuda.empty_cache()
     return out
+
+
+def split_measure(ql, torch, dev, flush, peak_tf, steps=10):
+    """The text projection at M = 512 (54 output tiles on 148 SMs) on the fused path, whole and split 8 ways."""
+    w = S.WORKLOADS["text_proj"]
+    M = 512
+    flops = 2.0 * M * w.K * w.N
+    out = {"workload": f"{w.name} M={M} K={w.K} N={w.N}"}
+    for split in (1, 8):
+        c = Case(ql, torch, w, M, 3, dev, flush, split)          # 3 = the fused tensor-core path
+        c.warm(3)
+        st, mn = c.timed(steps)
+        assert ql.device_status() == 0, "the fused path reported an error"
+        out[f"split{split}"] = {"dispatch": c.dispatch, "step_us": st * 1e3, "kernel_us": mn * 1e3,
+                                "TFLOPs": flops / (st * 1e-3) / 1e12,
+                                "kernel_frac": flops / (mn * 1e-3) / 1e12 / peak_tf}
+        del c
+    torch.cuda.synchronize()
+    return out
+
+
+def guarded(fn):
+    """Run an extra measurement; an error is recorded in the line instead of costing it."""
+    try:
+        return fn()
+    except Exception as exc:            # noqa: BLE001
+        return {"error": f"{type(exc).__name__}: {exc}"[:200]}
 
 
 def oracle_fit_rate(rows=4):
@@ -531,13 +560,12 @@ def main():
 
     # ---- the quantizer: importance-weighted fit and RTN pack of a DiT-shaped weight
     pack = None if a.no_pack else pack_measure(ql, torch, dev, flush)
-    swiglu = swiglu_measure(ql, torch, dev, flush, peaks()[0]) if a.swiglu else None
-    comp = None
-    if not a.no_comparators:
-        try:                            # context only: never let it cost the measured line
-            comp = comparators(ql, torch, dev, flush)
-        except Exception as exc:        # noqa: BLE001
-            comp = {"error": f"{type(exc).__name__}: {exc}"[:200]}
+    # Extras, one GPU only (their errors are recorded, never raised; with several ranks every rank would
+    # have to take the same collective steps afterwards).
+    single = world == 1
+    swiglu = guarded(lambda: swiglu_measure(ql, torch, dev, flush, peaks()[0])) if single and not a.no_swiglu else None
+    split = guarded(lambda: split_measure(ql, torch, dev, flush, peaks()[0])) if single and not a.no_split else None
+    comp = guarded(lambda: comparators(ql, torch, dev, flush)) if single and not a.no_comparators else None
 
     mean_step, mean_main, mean_e2e = max_over_ranks([mean_step, mean_main, mean_e2e], dev)
 
@@ -582,6 +610,8 @@ def main():
         line["small_m_w8"] = small_w8
     if swiglu is not None:
         line["swiglu"] = swiglu
+    if split is not None:
+        line["split_m512"] = split
     if comp is not None:
         line["comparators"] = comp
     if pack is not None:
