@@ -149,6 +149,7 @@ def swiglu_measure(ql, torch, dev, flush, peak_tf, steps=10):
         flush.fill_(1)
         step()
     torch.cuda.synchronize()
+    assert ql.device_status() == 0, "the SwiGLU pair reported an error in warm-up"
     dispatch = ql.last_dispatch()
     call_ms, main_ms = [], []
     for i in range(steps):
@@ -232,6 +233,7 @@ def split_measure(ql, torch, dev, flush, peak_tf, steps=10):
     for split in (1, 8):
         c = Case(ql, torch, w, M, 3, dev, flush, split)          # 3 = the fused tensor-core path
         c.warm(3)
+        assert ql.device_status() == 0, "the fused path reported an error in warm-up"
         st, mn = c.timed(steps)
         assert ql.device_status() == 0, "the fused path reported an error"
         out[f"split{split}"] = {"dispatch": c.dispatch, "step_us": st * 1e3, "kernel_us": mn * 1e3,
