@@ -35,7 +35,8 @@ class QLinearError(RuntimeError):
 
 
 def library_path() -> str:
-    return os.path.join(_HERE, _LIB_NAME)
+    """The in-tree libqlinear.so, or the library QL_LIBRARY names (e.g. the bounds-checked build)."""
+    return os.environ.get("QL_LIBRARY") or os.path.join(_HERE, _LIB_NAME)
 
 
 def lib() -> ctypes.CDLL:

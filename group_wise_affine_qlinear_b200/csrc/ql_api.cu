@@ -449,6 +449,7 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     p.cpt = static_cast<int>((G + cg - 1) / cg);
     p.units = pl.units;
     p.segmax = pl.segmax;
+    p.partial_elems = static_cast<int64_t>(pl.ctas) * pl.segmax * M * skinny::BW;
     // row maxima, then scaled and reordered f16 activations, per-group activation sums, row exponents
     const dim3 pre_grid(static_cast<unsigned>(pl.slices), static_cast<unsigned>(M));
     skinny::skinny_rowmax_kernel<<<pre_grid, 256, 0, st>>>(static_cast<const uint4*>(x), pmax, static_cast<int>(K));
@@ -492,10 +493,10 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     const dim3 red_grid(static_cast<unsigned>(p.num_w), static_cast<unsigned>((M + 1) / 2));
     if (bf16_out)
         s = launch_dependent(skinny::skinny_reduce_kernel<true>, red_grid, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
-                             p.units, pl.ctas, pl.segmax);
+                             p.units, pl.ctas, pl.segmax, p.partial_elems);
     else
         s = launch_dependent(skinny::skinny_reduce_kernel<false>, red_grid, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
-                             p.units, pl.ctas, pl.segmax);
+                             p.units, pl.ctas, pl.segmax, p.partial_elems);
     if (s != QL_OK) return s;
     (void)sm_count;
     set_dispatch("path=tc_skinny bits=%d nt=%d ctas=%d segmax=%d units=%lld launches=4", bits, pl.nt, pl.ctas,

@@ -22,6 +22,19 @@ __device__ __forceinline__ void record_status(unsigned int code) {
     atomicCAS(&g_device_status, 0u, code);
 }
 
+// Index checks of the bounds-checked build (compiled with QL_BOUNDS_CHECK, the stand-in for a memory
+// checker): an index outside [0, n) records QL_ERR_BOUNDS and the access is skipped.  In the normal
+// build every check is the constant true.
+#ifdef QL_BOUNDS_CHECK
+__device__ __forceinline__ bool in_bounds(int64_t i, int64_t n) {
+    if (i >= 0 && i < n) return true;
+    record_status(QL_ERR_BOUNDS);
+    return false;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(int64_t, int64_t) { return true; }
+#endif
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

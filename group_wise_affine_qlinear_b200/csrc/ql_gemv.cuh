@@ -79,7 +79,8 @@ __device__ __forceinline__ void gemv_body(
                 if (m >= M) break;
                 const int64_t o = static_cast<int64_t>(m) * N + n;
                 if (partial_out) {
-                    reinterpret_cast<float*>(out)[static_cast<int64_t>(blockIdx.y) * M * N + o] = acc[i];
+                    const int64_t at = static_cast<int64_t>(blockIdx.y) * M * N + o;
+                    if (in_bounds(at, static_cast<int64_t>(gridDim.y) * M * N)) reinterpret_cast<float*>(out)[at] = acc[i];
                 } else if constexpr (kBf16Out) {
                     reinterpret_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(acc[i]);
                 } else {
@@ -163,7 +164,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv8_kernel(
                 if (m >= M) break;
                 const int64_t o = static_cast<int64_t>(m) * N + n;
                 if (partial_out) {
-                    reinterpret_cast<float*>(out)[static_cast<int64_t>(blockIdx.y) * M * N + o] = acc[i];
+                    const int64_t at = static_cast<int64_t>(blockIdx.y) * M * N + o;
+                    if (in_bounds(at, static_cast<int64_t>(gridDim.y) * M * N)) reinterpret_cast<float*>(out)[at] = acc[i];
                 } else if constexpr (kBf16Out) {
                     reinterpret_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(acc[i]);
                 } else {

@@ -108,6 +108,7 @@ struct Params {
     int cpt;                 // chunks per tile = ceil(G / CG)
     int64_t units;           // num_w * cpt chunks
     int segmax;
+    int64_t partial_elems;   // floats in partial (index checks of the bounds-checked build)
 };
 
 // First unit of CTA c's run (runs are [first(c), first(c+1))).
@@ -419,8 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int q = 2 * j + h;
-                        if (n < p.N && q < ng) {
-                            const int64_t at = static_cast<int64_t>(n) * p.G + g0 + q;
+                        const int64_t at = static_cast<int64_t>(n) * p.G + g0 + q;
+                        if (n < p.N && q < ng && in_bounds(at, static_cast<int64_t>(p.N) * p.G)) {
                             sp |= static_cast<uint32_t>(__half_as_ushort(__ldg(p.scales + at))) << (16 * h);
                             bp |= static_cast<uint32_t>(__half_as_ushort(__ldg(p.biases + at))) << (16 * h);
                         }
@@ -497,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const int tt = 16 * h16 + t;
-                    if (tt < p.M)
+                    if (tt < p.M && in_bounds((dst - p.partial) + static_cast<int64_t>(tt) * BW + r, p.partial_elems))
                         dst[static_cast<int64_t>(tt) * BW + r] = (used0 ? __uint_as_float(d0[t]) : 0.0f) +
                                                                  (used1 ? __uint_as_float(d1[t]) : 0.0f);
                 }
@@ -525,7 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
 template <bool kBf16Out>
 __global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restrict__ partial,
                                                             const int* __restrict__ rowexp, void* __restrict__ y,
-                                                            int M, int N, int cpt, int64_t units, int P, int segmax) {
+                                                            int M, int N, int cpt, int64_t units, int P, int segmax,
+                                                            int64_t partial_elems) {
     __shared__ int64_t seg_base[kMaxCtas];
     __shared__ int count;
     const int w = blockIdx.x;
@@ -554,7 +556,10 @@ __global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restr
     if (t >= M || n >= N) return;
     float acc = 0.0f;
     const int k_end = count;
-    for (int k = 0; k < k_end; ++k) acc += partial[(seg_base[k] * M + t) * BW + r];
+    for (int k = 0; k < k_end; ++k) {
+        const int64_t at = (seg_base[k] * M + t) * BW + r;
+        if (in_bounds(at, partial_elems)) acc += partial[at];
+    }
     acc = ldexpf(acc, rowexp[t]);
     const int64_t e = static_cast<int64_t>(t) * N + n;
     if constexpr (kBf16Out) {

@@ -201,3 +201,10 @@ def test_fused_split_k_workspace(L):
     base = ql.workspace_size(M, K, N, ql.PATH_TC_FUSED)
     assert ql.workspace_size(M, K, N, ql.PATH_TC_FUSED, 8) == base + 8 * M * N * 4
     assert L.qlinear_workspace_size_config(16, 256, 256, 64, ql.PATH_TC_FUSED, 5) == ctypes.c_size_t(-1).value
+
+
+def test_bounds_checked_build_exports_every_declared_symbol():
+    """The index-checked variant (QL_BOUNDS_CHECK, selected at run time by QL_LIBRARY) builds and exports the ABI."""
+    Lb = ctypes.CDLL(qb.build(bounds_check=True))
+    for n in _declared():
+        assert hasattr(Lb, n), n
