@@ -423,6 +423,18 @@ class Case:
         self.dispatch = self.ql.last_dispatch()
         self.launches = int(self.dispatch.split("launches=")[1].split()[0]) if "launches=" in self.dispatch else 1
 
+    def timed_warm(self, steps):
+        """Mean device time of back-to-back calls with no L2 flush between them (inputs may stay in L2)."""
+        torch = self.torch
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        self.step()
+        e0.record()
+        for _ in range(steps):
+            self.step()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
     def timed(self, steps):
         """Per-step device time of the whole call and of its main kernel (L2 flushed before every step).
 
@@ -497,6 +509,7 @@ def main():
     barrier()
     clk = clocks.stop()
     assert ql.device_status() == 0, "a kernel reported an error"
+    warm_ms = case.timed_warm(a.steps)     # context: the same call without the L2 flush
 
     # ---- end to end: every step copies its x from pinned host memory, runs the layer through the
     # public API and copies its y back to pinned host memory.  Steps are pipelined the way a serving
@@ -569,7 +582,7 @@ def main():
     split = guarded(lambda: split_measure(ql, torch, dev, flush, peaks()[0])) if single and not a.no_split else None
     comp = guarded(lambda: comparators(ql, torch, dev, flush)) if single and not a.no_comparators else None
 
-    mean_step, mean_main, mean_e2e = max_over_ranks([mean_step, mean_main, mean_e2e], dev)
+    mean_step, mean_main, mean_e2e, warm_ms = max_over_ranks([mean_step, mean_main, mean_e2e, warm_ms], dev)
 
     flops = 2.0 * M * K * N
     value = whole_job_rate(flops, mean_step, world) / 1e12
@@ -601,7 +614,9 @@ def main():
         "config": {"workload": f"{w.name} M={M} K={K} N={N}", "seed": w.seed,
                    "inputs_sha256": S.digest(case.x_np, case.codes_np, case.s_np, case.b_np),
                    "l2": "flushed between steps (512 MiB write)", "parallelism": f"replicas x{world}",
-                   "dispatch": dispatch, "weight_GBps": w.weight_bytes / (mean_step * 1e-3) / 1e9},
+                   "dispatch": dispatch, "weight_GBps": w.weight_bytes / (mean_step * 1e-3) / 1e9,
+                   "l2_warm": {"ms_per_step": warm_ms, "value": whole_job_rate(flops, warm_ms, world) / 1e12,
+                               "note": "same call back to back, no flush between steps (context)"}},
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
         "gpu_launches": case.launches * a.steps,
