@@ -108,7 +108,8 @@ ql_status device_info(DeviceInfo** out) {
     }
     if (!d.skinny_attr_set) {
         if (skinny_smem_attr<16, 4>() != cudaSuccess || skinny_smem_attr<32, 4>() != cudaSuccess ||
-            skinny_smem_attr<16, 8>() != cudaSuccess || skinny_smem_attr<32, 8>() != cudaSuccess)
+            skinny_smem_attr<16, 8>() != cudaSuccess || skinny_smem_attr<32, 8>() != cudaSuccess ||
+            skinny_smem_attr<64, 4>() != cudaSuccess || skinny_smem_attr<64, 8>() != cudaSuccess)
             return QL_ERR_CUDA;
         d.skinny_attr_set = true;
     }
@@ -216,8 +217,9 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         return QL_OK;
     }
     if (path == QL_PATH_TC_SKINNY) {
-        if (M > 32 || split_k > 1) return QL_ERR_UNSUPPORTED;
-        plan->nt = M <= 16 ? 16 : 32;
+        // the dispatcher picks this path for M <= 32; M up to 64 (NT = 64) runs when forced
+        if (M > 64 || split_k > 1) return QL_ERR_UNSUPPORTED;
+        plan->nt = M <= 16 ? 16 : M <= 32 ? 32 : 64;
         const int64_t cg = bits == 4 ? skinny::Layout<16, 4>::CG : skinny::Layout<16, 8>::CG;
         const int64_t cpt = (G + cg - 1) / cg;
         plan->units = ((N + skinny::BW - 1) / skinny::BW) * cpt;
@@ -477,14 +479,20 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     if (bits == 4 && pl.nt == 16)
         s = launch_dependent(skinny::skinny_kernel<16, 4>, sgrid, skinny::kThreads, skinny::Layout<16, 4>::kSmemBytes, st,
                              mc, mx, ms, mb, p);
-    else if (bits == 4)
+    else if (bits == 4 && pl.nt == 32)
         s = launch_dependent(skinny::skinny_kernel<32, 4>, sgrid, skinny::kThreads, skinny::Layout<32, 4>::kSmemBytes, st,
+                             mc, mx, ms, mb, p);
+    else if (bits == 4)
+        s = launch_dependent(skinny::skinny_kernel<64, 4>, sgrid, skinny::kThreads, skinny::Layout<64, 4>::kSmemBytes, st,
                              mc, mx, ms, mb, p);
     else if (pl.nt == 16)
         s = launch_dependent(skinny::skinny_kernel<16, 8>, sgrid, skinny::kThreads, skinny::Layout<16, 8>::kSmemBytes, st,
                              mc, mx, ms, mb, p);
-    else
+    else if (pl.nt == 32)
         s = launch_dependent(skinny::skinny_kernel<32, 8>, sgrid, skinny::kThreads, skinny::Layout<32, 8>::kSmemBytes, st,
+                             mc, mx, ms, mb, p);
+    else
+        s = launch_dependent(skinny::skinny_kernel<64, 8>, sgrid, skinny::kThreads, skinny::Layout<64, 8>::kSmemBytes, st,
                              mc, mx, ms, mb, p);
     if (s != QL_OK) return s;
     prof_end(st);

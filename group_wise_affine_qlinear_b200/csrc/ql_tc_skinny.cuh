@@ -78,8 +78,9 @@ struct Layout {
     static constexpr int kBoxGroups = 128 / (4 * kGroupWords);           // groups per code box
     static constexpr uint32_t kCBytes = kBoxBytes * (CG / kBoxGroups);   // codes per chunk
     static constexpr uint32_t kStageBytes = kCBytes + 2 * kParHalf;      // [codes | scales | biases]
-    static constexpr int NC = B == 4 ? (NT == 16 ? 4 : 3) : (NT == 16 ? 5 : 4);    // code/parameter chunk stages
-    static constexpr int NXC = B == 4 ? (NT == 16 ? 4 : 3) : (NT == 16 ? 5 : 4);   // activation chunk stages
+    // code/parameter and activation chunk stages: the activation tiles grow with NT, so the rings shrink
+    static constexpr int NC = B == 4 ? (NT == 16 ? 4 : NT == 32 ? 3 : 2) : (NT == 16 ? 5 : NT == 32 ? 4 : 3);
+    static constexpr int NXC = B == 4 ? (NT == 16 ? 4 : NT == 32 ? 3 : 2) : (NT == 16 ? 5 : NT == 32 ? 4 : 3);
     static constexpr uint32_t kXTile = NT * BK * 2;                      // one group's activation tile (f16)
     static constexpr uint32_t kXBytes = CG * kXTile;                     // one chunk's activation tiles
     static constexpr uint32_t kOffC = 0;                                  // [NC][codes | scales | biases]
@@ -91,6 +92,7 @@ struct Layout {
     static constexpr uint32_t kAccCol = 0;                                // accumulator (set e, issuer c) at (2e+c)*NT
     static constexpr uint32_t kACol = 4 * NT;                             // A stage st, half h at kACol + 32(2st+h)
     static_assert(B == 4 || B == 8, "4- or 8-bit codes");
+    static_assert(NT == 16 || NT == 32 || NT == 64, "MMA N of 16, 32 or 64 tokens");
     static_assert(CG <= 2 * kBuildCopies && CG % kBoxGroups == 0 && kParGroups % CG == 0,
                   "at most one pair of a chunk per builder copy; whole code boxes; whole chunks per parameter box");
     static_assert(kStageBytes % 1024 == 0, "swizzled code boxes need 1 KB alignment");

@@ -69,8 +69,9 @@ typedef enum { QL_F32 = 0, QL_BF16 = 1 } ql_dtype;
 typedef enum {
     QL_PATH_AUTO = 0,       /* per-shape choice of the dispatcher */
     QL_PATH_GEMV = 1,       /* CUDA-core split-K weight streaming (any M; meant for M <= 4) */
-    QL_PATH_TC_SKINNY = 2,  /* tcgen05 weight streaming for small M (M <= 32): stream-K over K,
-                               fp32 partials reduced in a fixed order */
+    QL_PATH_TC_SKINNY = 2,  /* tcgen05 weight streaming for small M: stream-K over K, fp32 partials
+                               reduced in a fixed order; the dispatcher uses it for M <= 32, forced it
+                               runs M <= 64 (QL_ERR_UNSUPPORTED above) */
     QL_PATH_TC_FUSED = 3    /* tcgen05 fused-dequant GEMM for large M */
     /* Both tcgen05 paths multiply f16 operands with fp32 accumulation in tensor memory: each
      * weight is rounded once, RN_f16(s * q + b), and each activation row is scaled by a power of

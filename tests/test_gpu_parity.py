@@ -173,7 +173,7 @@ def test_pack_imatrix_rejects_bad_importance():
 
 def test_skinny_rejects_large_m():
     rng = np.random.default_rng(12)
-    x, codes, s, b = random_layer(rng, 33, 256, 64)
+    x, codes, s, b = random_layer(rng, 65, 256, 64)
     with pytest.raises(ValueError):
         ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=ql.PATH_TC_SKINNY)
 
