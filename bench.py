@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 from group_wise_affine_qlinear_b200 import synthetic as S  # noqa: E402
 
 METRIC = "W4g64 qmatmul TFLOP/s (large-M tensor-core path)"
+SPEC_TFLOPS, SPEC_GBPS = 2250.0, 8000.0     # B200 spec sheet: dense bf16 tensor rate, HBM3e bandwidth
 FLUSH_BYTES = 512 << 20
 
 
@@ -606,6 +607,9 @@ def main():
                 "algorithmic": f"packed W ({w.bits / 8 + 0.0625:g} B/weight) + x + y bytes per launch"}
     for sm in small + small_w8:
         sm["frac_hbm_weight"] = sm["weight_GBps"] / peak_gbs
+        sm["frac_hbm_weight_spec"] = sm["weight_GBps"] / SPEC_GBPS
+    roof["spec_peak"] = SPEC_TFLOPS if roof["bound"] == "tensor" else SPEC_GBPS
+    roof["frac_of_spec"] = roof["achieved"] / roof["spec_peak"]
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
