@@ -683,3 +683,22 @@ def test_swiglu_tolerance_gates():
     t = O.swiglu_tolerance(bad, g, u, bf16_output=False)
     assert not t["ok"] and t["max_ratio"] > 1.0
     assert not O.swiglu_tolerance(h_ref * 1.01, g, u, bf16_output=False)["ok"]     # relF = 1e-2
+
+
+def test_pack_sizes_on_the_pages_fix_the_half_bit_overhead_of_both_widths():
+    """The pages' disk sizes (bf16 ~50 GB, Q4 ~14 GB, Q8 ~27 GB, each rounded to the GB) agree with
+    4 + 0.5 and 8 + 0.5 bits per weight (R1, R9): 50 GB of bf16 is 25e9 +- 0.25e9 weights, and both packed
+    sizes fall within their rounding.  Nearby overheads for the 8-bit pack (8.25 or 9 bits per weight) do not."""
+    g = json.load(open(os.path.join(GOLDEN, "format_constants.json")))
+    snap, q4, q8 = g["bf16_snapshot_gb"]["value"], g["q4_pack_gb"]["value"], g["q8_pack_gb"]["value"]
+    n_lo, n_hi = (snap - 0.5) * 1e9 / 2, (snap + 0.5) * 1e9 / 2          # weights, from bf16 bytes
+
+    def fits(bits, size_gb):
+        lo, hi = n_lo * bits / 8 / 1e9, n_hi * bits / 8 / 1e9
+        return hi >= size_gb - 0.5 and lo <= size_gb + 0.5
+
+    four = g["code_bits"]["value"] + g["overhead_bits_per_weight"]["value"]
+    eight = g["q8_code_bits"]["value"] + g["overhead_bits_per_weight"]["value"]
+    assert (four, eight) == (4.5, 8.5)
+    assert fits(four, q4) and fits(eight, q8)
+    assert not fits(8.25, q8) and not fits(9.0, q8)
