@@ -702,3 +702,16 @@ def test_pack_sizes_on_the_pages_fix_the_half_bit_overhead_of_both_widths():
     assert (four, eight) == (4.5, 8.5)
     assert fits(four, q4) and fits(eight, q8)
     assert not fits(8.25, q8) and not fits(9.0, q8)
+
+
+def test_w8_rtn_rejects_non_finite_and_out_of_range():
+    """Like the 4-bit pack: NaN, infinities and magnitudes beyond the f16 range have no scale and bias."""
+    for bad in (np.nan, np.inf, -np.inf, 70000.0):
+        w = np.zeros((2, 64), dtype=np.float32)
+        w[1, 7] = bad
+        with pytest.raises(ValueError):
+            O.pack8_rtn(w)
+    w = np.zeros((1, 64), dtype=np.float32)
+    w[0, 0] = 65504.0                            # the f16 maximum itself is packable
+    codes, s, b = O.pack8_rtn(w)
+    assert np.all(np.isfinite(O.dequant8_f32(codes, s, b)))
