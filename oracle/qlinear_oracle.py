@@ -61,9 +61,11 @@ notes of the repository):
      (two factors, each within R5's 4e-3).
 
 Parity status: the imatrix fit (pack_imatrix) is a search heuristic with no
-printed reference values; only its invariants are pinned ("never worse than
-RTN" per group, exact recovery of on-grid groups).  Everything else is pinned
-to closed forms, library conversions or brute force by the CPU tests.
+printed reference values.  Its invariants are pinned ("never worse than RTN"
+per group, exact recovery of on-grid groups), its least-squares refit is
+pinned to numpy's lstsq, and a group that only a refit can fit exactly pins
+the search to the weighted closed-form optimum.  Everything else is pinned to
+closed forms, library conversions or brute force by the CPU tests.
 """
 from __future__ import annotations
 
@@ -377,6 +379,32 @@ def _score(g64, imp_g, q, s16, b16):
     return _seq_sum(imp_g * (g64 - deq.astype(np.float64)) ** 2)
 
 
+def weighted_ls_affine(g64, imp_g, q, sw, swx):
+    """Weighted least squares of w ~ s*q + b over each group, the codes q held fixed.
+
+    The refit step of the imatrix fit (aimarketly "Ideogram-4-IQ4_M", "What IQ4
+    means here": the group parameters are a least-squares fit weighted by
+    E[x^2]).  Minimising sum_j imp_j (w_j - s q_j - b)^2 over (s, b) gives the
+    2x2 normal equations
+        [sum imp q^2   sum imp q] [s]   [sum imp q w]
+        [sum imp q     sum imp  ] [b] = [sum imp w  ]
+    solved here by Cramer's rule in float64.  sw = sum imp and swx = sum imp w
+    do not depend on q and are passed in; every moment is summed one term at a
+    time in index order.  Returns (s, b, solvable), solvable False where the
+    determinant vanishes relative to its terms (all codes equal).
+    """
+    qf = q.astype(np.float64)
+    swq = _seq_sum(imp_g * qf)
+    swqq = _seq_sum(imp_g * qf * qf)
+    swqx = _seq_sum(imp_g * qf * g64)
+    det = swqq * sw - swq * swq
+    solvable = np.abs(det) > 1e-12 * np.maximum(swqq * sw, 1e-300)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        s_ls = (swqx * sw - swq * swx) / det
+        b_ls = (swqq * swx - swq * swqx) / det
+    return s_ls, b_ls, solvable
+
+
 def _fit_rows(w, imp):
     n, K = w.shape
     G = K // GROUP
@@ -415,15 +443,8 @@ def _fit_rows(w, imp):
             consider(q, s16, b16)
             active = np.ones(s16.shape, dtype=bool)
             for _ in range(FIT_REFITS):
-                qf = q.astype(np.float64)
-                swq = _seq_sum(imp_g * qf)
-                swqq = _seq_sum(imp_g * qf * qf)
-                swqx = _seq_sum(imp_g * qf * g64)
-                det = swqq * sw - swq * swq
-                ok = active & (np.abs(det) > 1e-12 * np.maximum(swqq * sw, 1e-300))
-                with np.errstate(divide="ignore", invalid="ignore"):
-                    s_ls = (swqx * sw - swq * swx) / det
-                    b_ls = (swqq * swx - swq * swqx) / det
+                s_ls, b_ls, solvable = weighted_ls_affine(g64, imp_g, q, sw, swx)
+                ok = active & solvable
                 ok &= np.isfinite(s_ls) & np.isfinite(b_ls) & (s_ls > 0)
                 ok &= (np.abs(s_ls) <= F16_MAX) & (np.abs(b_ls) <= F16_MAX)
                 active = ok

@@ -406,6 +406,62 @@ def test_fit_on_grid_group_has_zero_error():
     assert O.group_weighted_error(w, c, s2, b2, imp).max() == 0.0
 
 
+def test_ls_refit_matches_library_least_squares():
+    """The refit step solves the E[x^2]-weighted least squares of w ~ s*q + b for fixed codes: it agrees
+    with numpy's lstsq on sqrt(imp)-scaled [q, 1] columns to float64 rounding, on random groups with
+    random codes and log-normal importances (aimarketly "Ideogram-4-IQ4_M", "What IQ4 means here")."""
+    rng = _rng(31)
+    n, G = 6, 5
+    g64 = rng.standard_normal((n, G, 64)) * 0.02
+    q = rng.integers(0, 16, size=(n, G, 64))
+    imp_g = np.exp(rng.standard_normal((1, G, 64)) * 2.0)
+    sw = (imp_g * np.ones_like(g64)).sum(-1)
+    swx = (imp_g * g64).sum(-1)
+    s_ls, b_ls, solvable = O.weighted_ls_affine(g64, imp_g, q, sw, swx)
+    assert solvable.all()
+    for i in range(n):
+        for g in range(G):
+            r = np.sqrt(imp_g[0, g])
+            A = np.stack([q[i, g] * r, r], axis=1)
+            (s_ref, b_ref), *_ = np.linalg.lstsq(A, g64[i, g] * r, rcond=None)
+            assert abs(s_ls[i, g] - s_ref) <= 1e-9 * abs(s_ref)
+            assert abs(b_ls[i, g] - b_ref) <= 1e-9 * max(abs(b_ref), abs(s_ref))
+    # all codes equal: the system is singular and flagged so
+    _, _, solvable = O.weighted_ls_affine(g64[:1, :1], imp_g[:, :1], np.full((1, 1, 64), 7), sw[:1, :1], swx[:1, :1])
+    assert not solvable.any()
+
+
+def test_fit_refit_reaches_the_weighted_optimum():
+    """A group whose heavily weighted channels lie on an f16 affine grid (s*, b*) while unweighted outliers
+    set its min and max: RTN and every range-shrink candidate miss that grid, and only a refit of the
+    candidate whose step equals s* recovers it.  The fit must land on the best triple that reproduces the
+    weighted channels exactly, i.e. the f16 closed-form optimum, reaching its error."""
+    s_star, b_star = 2.0 ** -7, -6.5 * 2.0 ** -7
+    q_imp = np.array([0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 3, 7, 1, 5, 8, 2])
+    w = np.zeros(64)
+    w[:16] = s_star * q_imp + b_star
+    w[16:] = np.linspace(b_star - 8 * s_star, b_star + 13.4286 * s_star, 48)   # range 21.4286 s*: step s* at shrink 0.3
+    imp = np.zeros(64)
+    imp[:16] = 100.0
+    w32 = w.astype(np.float32)[None, :]
+    c, s, b = O.pack_imatrix(w32, imp)
+    impr = imp + 1e-6 * imp.mean()
+    e_fit = O.group_weighted_error(w32, c, s, b, impr)[0, 0]
+    # closed form: the triples (s*, b* - k s*) reproduce the weighted channels exactly for every shift k
+    # that keeps their codes in range; the best of them is the weighted optimum up to the outliers' share
+    best = np.inf
+    for k in range(0, 16 - q_imp.max()):
+        s16 = np.array([[s_star]], dtype=np.float16)
+        b16 = np.array([[b_star - k * s_star]], dtype=np.float16)
+        qk = np.clip(np.rint((w - (b_star - k * s_star)) / s_star), 0, 15).astype(np.int64)
+        best = min(best, O.group_weighted_error(w32, O.pack_codes(qk[None, :]), s16, b16, impr)[0, 0])
+    assert float(s[0, 0]) == s_star
+    assert np.array_equal(O.dequant_f32(c, s, b)[0, :16], w32[0, :16])
+    assert e_fit <= best * (1 + 1e-12)
+    cr, sr, br = O.pack_rtn(w32)
+    assert O.group_weighted_error(w32, cr, sr, br, impr)[0, 0] > 1e4 * e_fit
+
+
 def test_imatrix_is_mean_square():
     x = np.array([[0x3F80, 0x4000], [0xBF80, 0x0000]], dtype=np.uint16)   # [[1, 2], [-1, 0]]
     assert np.array_equal(O.imatrix_from_x(x), np.array([1.0, 2.0]))
