@@ -4,8 +4,9 @@
 
 One step = one qlinear_forward call (y = x . W^T) on the workload's seeded
 synthetic inputs, which are resident in HBM when the timed region starts.
-Between timed steps a 512 MiB buffer is written to flush the 126 MB L2, so no
-step starts with its operands cached.  Each step is timed on the launching
+Between timed steps a 512 MiB buffer is written to flush the 126 MB L2 and a
+256 MiB buffer is read so the flush's dirty lines are written back first: no
+step starts with its operands cached, and none pays for the flush.  Each step is timed on the launching
 stream with CUDA events; the main kernel is timed alone through the
 library's profile-event hook.  Under torchrun every rank runs an independent
 replica (the layer needs no exchange for data-parallel tokens), the slowest
@@ -36,6 +37,29 @@ from group_wise_affine_qlinear_b200 import synthetic as S  # noqa: E402
 METRIC = "W4g64 qmatmul TFLOP/s (large-M tensor-core path)"
 SPEC_TFLOPS, SPEC_GBPS = 2250.0, 8000.0     # B200 spec sheet: dense bf16 tensor rate, HBM3e bandwidth
 FLUSH_BYTES = 512 << 20
+CLEAN_BYTES = 256 << 20
+L2_NOTE = ("flushed between steps: 512 MiB written, then 256 MiB of another buffer read, so the flush's "
+           "dirty lines are back in HBM before the step starts")
+
+
+class L2Flush:
+    """Evicts every operand from the 126 MB L2 between timed steps.
+
+    fill_() writes 512 MiB (the flush) and, unless dirty=True, then reads 256 MiB of a second buffer: the
+    read evicts the flush's own dirty lines, whose write-back would otherwise run inside the next timed
+    step and be charged to it (a memory-only streaming kernel on 123 MB measured 31 us after the write
+    alone against 27.6 us after write + read on a B200).  dirty=True keeps the write alone, for context.
+    """
+
+    def __init__(self, torch, dev, dirty: bool = False):
+        self.torch = torch
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = None if dirty else torch.ones(CLEAN_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def fill_(self, v: int):
+        self.w.fill_(v)
+        if self.r is not None:
+            self.sink = self.torch.amax(self.r)
 
 
 def parse():
@@ -59,6 +83,11 @@ def parse():
                     help="skip the cuBLAS context measurements (dense bf16 and dequant-then-matmul)")
     ap.add_argument("--no-w8", action="store_true",
                     help="skip the 8-bit conditioning projection (text_proj_w8) at M = 1, 8, 32")
+    ap.add_argument("--no-large", action="store_true",
+                    help="skip the other M >= 4608 workloads (the MLP pair, the 2048^2 canvas)")
+    ap.add_argument("--no-dispatch", action="store_true",
+                    help="skip the dispatcher-versus-forced-configurations sweep on the text projection")
+    ap.add_argument("--no-noalloc", action="store_true", help="skip the allocation-free entry's measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     return ap.parse_args()
 
@@ -245,6 +274,91 @@ def split_measure(ql, torch, dev, flush, peak_tf, steps=10):
     return out
 
 
+def fitted_weights(ql, torch, dev, w, x_bits, codes, scales, biases):
+    """Device copies of the workload's packed weight with its first w.fitted_rows rows replaced by the
+    importance-weighted fit (qlinear_pack with an imatrix, byte-identical to the oracle's fit) of dense
+    N(0, 0.02^2) floats, the importance being E[x^2] of the workload's own activations."""
+    R = w.fitted_rows
+    dense = S.dense_weight(w.seed, w.widx, R, w.K, 0.02)
+    xf = (x_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    imp = (xf * xf).mean(axis=0).astype(np.float32)
+    cf, sf, bf = ql.pack(torch.from_numpy(dense).to(dev), imatrix=torch.from_numpy(imp).to(dev))
+    codes[:R].copy_(cf)
+    scales[:R].copy_(sf)
+    biases[:R].copy_(bf)
+    torch.cuda.synchronize()
+    assert ql.device_status() == 0, "qlinear_pack reported an error"
+
+
+def large_m_measure(ql, torch, dev, flush, peak_tf, steps=5):
+    """The other M >= 4608 workloads, each through the dispatcher: the MLP pair (up/gate N = 2 x 18432 with
+    its first 4608 rows fitted, down K = 18432) and the 2048^2 canvas (M = 33792, N = 4608 and 13824)."""
+    out = {}
+    for name in ("mlp_up_gate", "mlp_down", "canvas2048_n4608", "canvas2048_n13824"):
+        w = S.WORKLOADS[name]
+        c = Case(ql, torch, w, w.M, 0, dev, flush)
+        if w.fitted_rows:
+            fitted_weights(ql, torch, dev, w, c.x_np, c.codes, c.sc, c.bi)
+        c.warm(3)
+        assert ql.device_status() == 0, f"{name}: a kernel reported an error in warm-up"
+        st, mn = c.timed(steps)
+        assert ql.device_status() == 0, f"{name}: a kernel reported an error"
+        flops = 2.0 * w.M * w.K * w.N
+        out[name] = {"workload": f"{w.name} M={w.M} K={w.K} N={w.N}" + (f" ({w.fitted_rows} rows fitted)"
+                                                                          if w.fitted_rows else ""),
+                     "dispatch": c.dispatch, "step_ms": st, "kernel_ms": mn,
+                     "TFLOPs": flops / (st * 1e-3) / 1e12, "kernel_TFLOPs": flops / (mn * 1e-3) / 1e12,
+                     "frac": flops / (st * 1e-3) / 1e12 / peak_tf,
+                     "frac_of_spec": flops / (st * 1e-3) / 1e12 / SPEC_TFLOPS,
+                     "kernel_frac": flops / (mn * 1e-3) / 1e12 / peak_tf}
+        del c
+        torch.cuda.empty_cache()
+    return out
+
+
+def dispatch_measure(ql, torch, dev, flush, steps=10):
+    """The dispatcher against every forced configuration on the text projection for 33 <= M <= 512: the
+    automatic choice's whole-call time beside the best forced one (weight streaming up to 64 tokens, the
+    fused kernel with split-K 1, 2, 4, 5, 8)."""
+    w = S.WORKLOADS["text_proj"]
+    out = []
+    base = None
+    for M in (33, 48, 64, 65, 128, 256, 512):
+        c = Case(ql, torch, w, M, 0, dev, flush, weights=base)
+        base = (c.codes, c.sc, c.bi, c.codes_np, c.s_np, c.b_np)
+        c.warm(2)
+        auto_us = c.timed(steps)[0] * 1e3
+        auto = c.dispatch
+        forced = {}
+        for path, split in ([(2, 0)] if M <= 64 else []) + [(3, 1), (3, 2), (3, 4), (3, 5), (3, 8)]:
+            c.set_config(path, split)
+            c.warm(2)
+            forced[f"path{path}_split{split}"] = c.timed(steps)[0] * 1e3
+        best = min(forced, key=forced.get)
+        out.append({"M": M, "auto_us": auto_us, "auto_dispatch": auto, "best_forced": best,
+                    "best_forced_us": forced[best], "auto_over_best": auto_us / forced[best], "forced_us": forced})
+        del c
+    torch.cuda.empty_cache()
+    return out
+
+
+def noalloc_measure(ql, torch, dev, flush, steps=10):
+    """The allocation-free entry (CUDA-core split-K path, scratch inside the library) on the text projection."""
+    w = S.WORKLOADS["text_proj"]
+    out = []
+    base = None
+    for M in (1, 8, 32, 64):
+        c = Case(ql, torch, w, M, 0, dev, flush, weights=base)
+        base = (c.codes, c.sc, c.bi, c.codes_np, c.s_np, c.b_np)
+        c.fwd = lambda x, cd, s, b, out, workspace, path, split_k: ql.forward_noalloc(x, cd, s, b, out=out)
+        c.warm(2)
+        st, _ = c.timed(steps)
+        out.append({"M": M, "step_us": st * 1e3, "weight_GBps": w.weight_bytes / (st * 1e-3) / 1e9})
+        del c
+    assert ql.device_status() == 0, "the allocation-free entry reported an error"
+    return out
+
+
 def guarded(fn):
     """Run an extra measurement; an error is recorded in the line instead of costing it."""
     try:
@@ -359,15 +473,18 @@ def run_reference(a, rank, world):
         rate, cores, rows, dt = oracle_rate(w, M, 0.0, x, weights)     # one 64-row chunk per step
         if i >= a.warmup:
             per.append((rate, rows, dt))
+    rows_per_step = per[0][1]
     rate = sum(r[1] for r in per) * 2.0 * w.K * w.N / sum(r[2] for r in per) / 1e12
-    ms = 1e3 * 2.0 * M * w.K * w.N / (rate * 1e12)
+    ms = 1e3 * sum(r[2] for r in per) / len(per)          # measured wall time of one step (its row sample)
     line = {
         "impl": "reference", "metric": METRIC, "value": rate, "unit": "TFLOP/s", "n_gpus": a.gpus,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name} M={M} K={w.K} N={w.N}", "sample": "64 rows per step"},
+        "config": {"workload": f"{w.name} M={M} K={w.K} N={w.N}", "seed": w.seed,
+                   "sample": f"each step computes {rows_per_step} of the {M} rows (rows are independent), "
+                             f"full K and N; ms_per_step is that step's measured time"},
         "cpu_baseline": {"value": rate, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"64 of {M} rows per step (rows are independent), full N and K"},
+                         "sample": f"{rows_per_step} of {M} rows per step (rows are independent), full N and K"},
         "e2e": {"value": rate, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -396,21 +513,31 @@ def whole_job_rate(work_per_rank: float, slowest_ms: float, world: int) -> float
 class Case:
     """Device-resident inputs of one workload and timed qlinear_forward steps on them."""
 
-    def __init__(self, ql, torch, w, M, path, dev, flush, split=0):
+    def __init__(self, ql, torch, w, M, path, dev, flush, split=0, weights=None):
         import numpy as np
         self.ql, self.torch, self.w, self.M, self.path, self.flush = ql, torch, w, M, path, flush
-        self.split = split
+        self.split, self.dev = split, dev
         self.K, self.N = w.K, w.N
         self.x_np = w.x(M)
-        self.codes_np, self.s_np, self.b_np = w.w()
         self.x = torch.from_numpy(self.x_np.view(np.int16)).view(torch.bfloat16).to(dev)
-        self.codes = torch.from_numpy(self.codes_np.view(np.int32)).to(dev)
-        self.sc = torch.from_numpy(self.s_np).to(dev)
-        self.bi = torch.from_numpy(self.b_np).to(dev)
+        if weights is None:
+            self.codes_np, self.s_np, self.b_np = w.w()
+            self.codes = torch.from_numpy(self.codes_np.view(np.int32)).to(dev)
+            self.sc = torch.from_numpy(self.s_np).to(dev)
+            self.bi = torch.from_numpy(self.b_np).to(dev)
+        else:                       # device weights of the same workload from another case
+            self.codes, self.sc, self.bi, self.codes_np, self.s_np, self.b_np = weights
         self.y = torch.empty((M, self.N), dtype=torch.bfloat16, device=dev)
-        ws_bytes = ql.workspace_size(M, self.K, self.N, path, split, bits=w.bits)
-        self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.ws = None
+        self.set_config(path, split)
         self.fwd = ql.forward8 if w.bits == 8 else ql.forward
+
+    def set_config(self, path, split):
+        self.path, self.split = path, split
+        ws_bytes = self.ql.workspace_size(self.M, self.K, self.N, path, split, bits=self.w.bits)
+        if self.ws is None or self.ws.numel() < ws_bytes:
+            self.ws = None
+            self.ws = self.torch.empty(max(ws_bytes, 16), dtype=self.torch.uint8, device=self.dev)
 
     def step(self):
         self.fwd(self.x, self.codes, self.sc, self.bi, out=self.y, workspace=self.ws, path=self.path,
@@ -494,7 +621,7 @@ def main():
         torch.cuda.synchronize()
 
     dev = torch.device("cuda", local)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(torch, dev)
     w = S.WORKLOADS[a.workload]
     M = a.M or w.M
     K, N = w.K, w.N
@@ -513,7 +640,8 @@ def main():
     warm_ms = case.timed_warm(a.steps)     # context: the same call without the L2 flush
 
     # ---- end to end: every step copies its x from pinned host memory, runs the layer through the
-    # public API and copies its y back to pinned host memory.  Steps are pipelined the way a serving
+    # public API and copies its y back to pinned host memory.  No L2 flush runs inside this loop: a
+    # step's x, packed W and y together exceed the 126 MB L2 for the large-M workloads.  Steps are pipelined the way a serving
     # loop would run them: copies in, compute and copies out on three streams, with device x and y
     # double-buffered, so a step's copies overlap its neighbours' work (PCIe is full duplex).  The
     # per-step figure is the device time of the whole loop divided by the number of steps.
@@ -543,7 +671,6 @@ def main():
         s_c.wait_event(in_done[i])
         if i >= 2:
             s_c.wait_event(out_done[i - 2])             # step i-2's y buffer has been copied out
-        flush.fill_(i & 0xFF)
         case.fwd(xb[b], case.codes, case.sc, case.bi, out=yb[b], workspace=case.ws, path=case.path,
                  split_k=case.split)
         comp_done[i].record(s_c)
@@ -557,6 +684,8 @@ def main():
     mean_e2e = t_begin.elapsed_time(t_end) / a.steps
 
     # ---- the small-M half of the metric: weight streaming on the 53248 -> 4608 text projection
+    dirty = L2Flush(torch, dev, dirty=True)
+
     def small_m(name):
         out = []
         tp = S.WORKLOADS[name]
@@ -564,9 +693,12 @@ def main():
             c = Case(ql, torch, tp, Ms, 0, dev, flush)
             c.warm(3)
             st, mn = c.timed(max(10, a.steps))
+            c.flush = dirty
+            st_d, _ = c.timed(max(10, a.steps))
             out.append({"M": Ms, "dispatch": c.dispatch, "step_us": st * 1e3, "kernel_us": mn * 1e3,
                         "weight_GBps": tp.weight_bytes / (st * 1e-3) / 1e9,
-                        "algorithmic_GBps": c.algorithmic_bytes() / (st * 1e-3) / 1e9})
+                        "algorithmic_GBps": c.algorithmic_bytes() / (st * 1e-3) / 1e9,
+                        "step_us_dirty_l2": st_d * 1e3})
             del c
         torch.cuda.synchronize()
         return out
@@ -576,6 +708,9 @@ def main():
 
     # ---- the quantizer: importance-weighted fit and RTN pack of a DiT-shaped weight
     pack = None if a.no_pack else pack_measure(ql, torch, dev, flush)
+    large = guarded(lambda: large_m_measure(ql, torch, dev, flush, peaks()[0])) if world == 1 and not a.no_large else None
+    disp = guarded(lambda: dispatch_measure(ql, torch, dev, flush)) if world == 1 and not a.no_dispatch else None
+    noalloc = guarded(lambda: noalloc_measure(ql, torch, dev, flush)) if world == 1 and not a.no_noalloc else None
     # Extras, one GPU only (their errors are recorded, never raised; with several ranks every rank would
     # have to take the same collective steps afterwards).
     single = world == 1
@@ -617,12 +752,14 @@ def main():
         "dtype": "f16 MMA, fp32 accumulate (bf16 in/out)", "data": "synthetic",
         "config": {"workload": f"{w.name} M={M} K={K} N={N}", "seed": w.seed,
                    "inputs_sha256": S.digest(case.x_np, case.codes_np, case.s_np, case.b_np),
-                   "l2": "flushed between steps (512 MiB write)", "parallelism": f"replicas x{world}",
+                   "l2": L2_NOTE, "parallelism": f"replicas x{world}",
                    "dispatch": dispatch, "weight_GBps": w.weight_bytes / (mean_step * 1e-3) / 1e9,
                    "l2_warm": {"ms_per_step": warm_ms, "value": whole_job_rate(flops, warm_ms, world) / 1e12,
                                "note": "same call back to back, no flush between steps (context)"}},
         "roofline": roof,
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+                "l2": "no flush inside the loop; per-step x + packed W + y bytes: "
+                      f"{(M * K * 2 + w.weight_bytes + M * N * 2) / 1e6:.1f} MB"},
         "gpu_launches": case.launches * a.steps,
         "clocks": clk,
         "small_m": small,
@@ -637,6 +774,12 @@ def main():
         line["comparators"] = comp
     if pack is not None:
         line["pack"] = pack
+    if large is not None:
+        line["large_m"] = large
+    if disp is not None:
+        line["dispatch"] = disp
+    if noalloc is not None:
+        line["noalloc"] = noalloc
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         rate, cores, rows, dt = oracle_rate(w, M, a.cpu_seconds, case.x_np[: min(M, 512)],
                                             (case.codes_np, case.s_np, case.b_np))

@@ -36,6 +36,7 @@ from ._lib import (  # noqa: F401
     last_dispatch,
     lib,
     library_path,
+    load_library,
     pack,
     pack8,
     reduce_partials,

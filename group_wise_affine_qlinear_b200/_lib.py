@@ -45,58 +45,64 @@ def lib() -> ctypes.CDLL:
     with _lock:
         if _lib is not None:
             return _lib
-        path = library_path()
-        if not os.path.exists(path):
-            raise RuntimeError(f"{path} is missing: build it with `python -m group_wise_affine_qlinear_b200.build`")
-        L = ctypes.CDLL(path)
-        vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
-        L.qlinear_workspace_size.argtypes = [i64, i64, i64, i32]
-        L.qlinear_workspace_size.restype = sz
-        L.qlinear_workspace_size_config.argtypes = [i64, i64, i64, i32, i32, i32]
-        L.qlinear_workspace_size_config.restype = sz
-        L.qlinear_forward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, sz, vp]
-        L.qlinear_forward.restype = ctypes.c_int
-        L.qlinear_forward_config.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i32, i32, i32, vp, sz, vp]
-        L.qlinear_forward_config.restype = ctypes.c_int
-        L.qlinear_dequant.argtypes = [vp, vp, vp, i64, i64, i32, vp, ctypes.c_int, vp]
-        L.qlinear_dequant.restype = ctypes.c_int
-        L.qlinear_pack.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp, vp]
-        L.qlinear_pack.restype = ctypes.c_int
-        L.qlinear_get_device_status.argtypes = [vp]
-        L.qlinear_get_device_status.restype = ctypes.c_int
-        L.qlinear_last_dispatch.argtypes = [ctypes.c_char_p, sz]
-        L.qlinear_last_dispatch.restype = ctypes.c_int
-        L.qlinear_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp]
-        L.qlinear_forward_noalloc.restype = ctypes.c_int
-        L.qlinear_set_profile_events.argtypes = [vp, vp]
-        L.qlinear_set_profile_events.restype = ctypes.c_int
-        L.qlinear_status_string.argtypes = [ctypes.c_int]
-        L.qlinear_status_string.restype = ctypes.c_char_p
-        L.qlinear_version.argtypes = []
-        L.qlinear_version.restype = ctypes.c_int32
-        L.qlinear8_workspace_size.argtypes = [i64, i64, i64, i32]
-        L.qlinear8_workspace_size.restype = sz
-        L.qlinear8_workspace_size_config.argtypes = [i64, i64, i64, i32, i32, i32]
-        L.qlinear8_workspace_size_config.restype = sz
-        L.qlinear8_forward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, sz, vp]
-        L.qlinear8_forward.restype = ctypes.c_int
-        L.qlinear8_forward_config.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i32, i32, i32, vp, sz,
-                                              vp]
-        L.qlinear8_forward_config.restype = ctypes.c_int
-        L.qlinear8_dequant.argtypes = [vp, vp, vp, i64, i64, i32, vp, ctypes.c_int, vp]
-        L.qlinear8_dequant.restype = ctypes.c_int
-        L.qlinear8_pack.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp, vp]
-        L.qlinear8_pack.restype = ctypes.c_int
-        L.qlinear_selftest_bounded_wait.argtypes = [vp]
-        L.qlinear_selftest_bounded_wait.restype = ctypes.c_int
-        L.qlinear_reduce_partials.argtypes = [vp, i32, i64, vp, ctypes.c_int, vp]
-        L.qlinear_reduce_partials.restype = ctypes.c_int
-        L.qlinear_swiglu_workspace_size.argtypes = [i64, i64, i64, i32]
-        L.qlinear_swiglu_workspace_size.restype = sz
-        L.qlinear_swiglu_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i32, vp, sz, vp]
-        L.qlinear_swiglu_forward.restype = ctypes.c_int
-        _lib = L
-        return L
+        _lib = load_library(library_path())
+        return _lib
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    """A CDLL of a qlinear library at `path` with every entry point's argument and result types set."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m group_wise_affine_qlinear_b200.build`")
+    L = ctypes.CDLL(path)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    L.qlinear_workspace_size.argtypes = [i64, i64, i64, i32]
+    L.qlinear_workspace_size.restype = sz
+    L.qlinear_workspace_size_config.argtypes = [i64, i64, i64, i32, i32, i32]
+    L.qlinear_workspace_size_config.restype = sz
+    L.qlinear_forward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, sz, vp]
+    L.qlinear_forward.restype = ctypes.c_int
+    L.qlinear_forward_config.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i32, i32, i32, vp, sz, vp]
+    L.qlinear_forward_config.restype = ctypes.c_int
+    L.qlinear_dequant.argtypes = [vp, vp, vp, i64, i64, i32, vp, ctypes.c_int, vp]
+    L.qlinear_dequant.restype = ctypes.c_int
+    L.qlinear_pack.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp, vp]
+    L.qlinear_pack.restype = ctypes.c_int
+    L.qlinear_get_device_status.argtypes = [vp]
+    L.qlinear_get_device_status.restype = ctypes.c_int
+    L.qlinear_last_dispatch.argtypes = [ctypes.c_char_p, sz]
+    L.qlinear_last_dispatch.restype = ctypes.c_int
+    L.qlinear_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp]
+    L.qlinear_forward_noalloc.restype = ctypes.c_int
+    L.qlinear_set_profile_events.argtypes = [vp, vp]
+    L.qlinear_set_profile_events.restype = ctypes.c_int
+    L.qlinear_status_string.argtypes = [ctypes.c_int]
+    L.qlinear_status_string.restype = ctypes.c_char_p
+    L.qlinear_version.argtypes = []
+    L.qlinear_version.restype = ctypes.c_int32
+    L.qlinear8_workspace_size.argtypes = [i64, i64, i64, i32]
+    L.qlinear8_workspace_size.restype = sz
+    L.qlinear8_workspace_size_config.argtypes = [i64, i64, i64, i32, i32, i32]
+    L.qlinear8_workspace_size_config.restype = sz
+    L.qlinear8_forward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, vp, sz, vp]
+    L.qlinear8_forward.restype = ctypes.c_int
+    L.qlinear8_forward_config.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i32, i32, i32, vp, sz,
+                                          vp]
+    L.qlinear8_forward_config.restype = ctypes.c_int
+    L.qlinear8_dequant.argtypes = [vp, vp, vp, i64, i64, i32, vp, ctypes.c_int, vp]
+    L.qlinear8_dequant.restype = ctypes.c_int
+    L.qlinear8_pack.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp, vp]
+    L.qlinear8_pack.restype = ctypes.c_int
+    L.qlinear_selftest_bounded_wait.argtypes = [vp]
+    L.qlinear_selftest_bounded_wait.restype = ctypes.c_int
+    L.qlinear_reduce_partials.argtypes = [vp, i32, i64, vp, ctypes.c_int, vp]
+    L.qlinear_reduce_partials.restype = ctypes.c_int
+    L.qlinear_swiglu_workspace_size.argtypes = [i64, i64, i64, i32]
+    L.qlinear_swiglu_workspace_size.restype = sz
+    L.qlinear_swiglu_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i32, vp, sz, vp]
+    L.qlinear_swiglu_forward.restype = ctypes.c_int
+    L.qlinear_test_stall.argtypes = [i32, ctypes.c_uint64]
+    L.qlinear_test_stall.restype = ctypes.c_int
+    return L
 
 
 def _stream_handle(stream) -> int:

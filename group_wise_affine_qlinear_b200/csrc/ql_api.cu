@@ -70,7 +70,11 @@ struct DeviceInfo {
 
 template <int NT, int B>
 cudaError_t skinny_smem_attr() {
-    return cudaFuncSetAttribute(skinny::skinny_kernel<NT, B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const cudaError_t e = cudaFuncSetAttribute(skinny::skinny_kernel<NT, B, true>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               skinny::Layout<NT, B>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(skinny::skinny_kernel<NT, B, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 skinny::Layout<NT, B>::kSmemBytes);
 }
 
@@ -193,20 +197,57 @@ struct Plan {
     int bits = 4;         // code width: 4 (W4 g64) or 8 (W8 g64)
     int path = QL_PATH_GEMV;
     int split_k = 1;
+    char why[64] = "forced";      // the dispatcher's reason, reported by qlinear_last_dispatch
     // skinny path: stream-K runs
     int ctas = 0, segmax = 0, nt = 0;
     int64_t units = 0;
     size_t workspace = 0;
     // fused path workspace carve-up (off_part: fp32 partials [split_k][M][N] when the K-steps are split)
     size_t off_xh = 0, off_rs = 0, off_sb = 0, off_part = 0;
-    // skinny path workspace carve-up: partials, scaled f16 activations, row exponents, per-slice row maxima
-    size_t off_xp = 0, off_re = 0, off_pm = 0;
+    // skinny path workspace carve-up: partials, scaled f16 activations, row exponents, per-tile arrival
+    // counts, per-slice row maxima (`slices` prepass blocks per row)
+    size_t off_xp = 0, off_re = 0, off_tc = 0, off_pm = 0;
     int slices = 0;
 };
 
+// Split factor of the fused tensor-core path when the caller leaves it to the dispatcher.  Every K-step
+// of a 256 x 192 tile costs about the same (0.56-0.66 us measured on a B200 across the text projection,
+// the QKV and the MLP down projection), so a launch of `tiles` tiles cut into S slices takes about
+// ceil(tiles * S / SMs) waves of ceil(G / S) K-steps.  Splitting also writes and reads back S fp32
+// partials of y and adds the ordered-sum launch.  The S with the lowest estimate wins; a larger S must
+// beat the best smaller one by 3%; a slice keeps at least 8 K-steps.  On the measured shapes (text projection M = 96..512,
+// QKV M = 64..1024, MLP down M = 64..512) this picks the fastest forced split or one within 5% of it.
+int fused_auto_split(int64_t M, int64_t N, int64_t G, int sm_count) {
+    constexpr double kStepNs = 600.0;           // one K-step of one tile
+    constexpr double kSplitFixedNs = 5000.0;    // the extra launch and the reduction's start
+    constexpr double kBytesPerNs = 6000.0;      // HBM rate of the partials' write and read-back
+    const int64_t tiles = ((M + fused::BT - 1) / fused::BT) * ((N + fused::BW - 1) / fused::BW);
+    const int64_t smax = std::max<int64_t>(1, std::min<int64_t>(16, G / 8));
+    int best_s = 1;
+    double best = 0.0;
+    for (int64_t sk = 1; sk <= smax; ++sk) {
+        const double waves = static_cast<double>((tiles * sk + sm_count - 1) / sm_count);
+        double t = waves * static_cast<double>((G + sk - 1) / sk) * kStepNs;
+        if (sk > 1) t += kSplitFixedNs + 8.0 * static_cast<double>(sk) * M * N / kBytesPerNs;
+        if (sk == 1 || t < 0.97 * best) {     // a larger split must win by more than the model's noise
+            best = t;
+            best_s = static_cast<int>(sk);
+        }
+    }
+    return best_s;
+}
+
+// Per-shape choice of QL_PATH_AUTO: the weight-streaming tensor-core kernel up to 64 tokens (its MMA
+// N of 16, 32 or 64 tokens covers them; measured on the text projection it takes 50-60 us for
+// M = 1..64, where the fused path needs 97 us split 8 ways and 467 us unsplit), the fused kernel above,
+// with the split of fused_auto_split.
 ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int sm_count, int bits, Plan* plan) {
     const int64_t G = K / kGroup;
-    if (path == QL_PATH_AUTO) path = (M <= 32) ? QL_PATH_TC_SKINNY : QL_PATH_TC_FUSED;
+    const bool automatic = path == QL_PATH_AUTO;
+    if (automatic) {
+        path = (M <= 64) ? QL_PATH_TC_SKINNY : QL_PATH_TC_FUSED;
+        std::snprintf(plan->why, sizeof(plan->why), "%s", M <= 64 ? "auto:M<=64" : "auto:M>64");
+    }
     plan->path = path;
     plan->bits = bits;
     if (path == QL_PATH_GEMV) {
@@ -217,7 +258,7 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         return QL_OK;
     }
     if (path == QL_PATH_TC_SKINNY) {
-        // the dispatcher picks this path for M <= 32; M up to 64 (NT = 64) runs when forced
+        // the dispatcher picks this path for M <= 64 (MMA N of 16, 32 or 64 tokens)
         if (M > 64 || split_k > 1) return QL_ERR_UNSUPPORTED;
         plan->nt = M <= 16 ? 16 : M <= 32 ? 32 : 64;
         const int64_t cg = bits == 4 ? skinny::Layout<16, 4>::CG : skinny::Layout<16, 8>::CG;
@@ -229,14 +270,23 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         plan->split_k = 1;
         plan->off_xp = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * M * skinny::BW * sizeof(float), 256);
         plan->off_re = plan->off_xp + round_up(static_cast<size_t>(M) * K * 2, 256);
-        plan->slices = static_cast<int>((K / 8 + 255) / 256);
-        plan->off_pm = plan->off_re + round_up(static_cast<size_t>(plan->nt) * sizeof(int), 256);
+        plan->off_tc = plan->off_re + round_up(static_cast<size_t>(plan->nt) * sizeof(int), 256);
+        plan->off_pm = plan->off_tc + round_up(static_cast<size_t>((N + skinny::BW - 1) / skinny::BW) * sizeof(int), 256);
+        // about one prepass block per SM in all, each slice at least one 16-byte load per thread
+        plan->slices = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sm_count / M, K / 8 / skinny::kPrepThreads)));
         plan->workspace = plan->off_pm + round_up(static_cast<size_t>(M) * plan->slices * sizeof(float), 256);
         return QL_OK;
     }
     if (path == QL_PATH_TC_FUSED) {
         if (split_k > G || split_k > 1024) return QL_ERR_INVALID_ARG;
-        plan->split_k = split_k > 1 ? split_k : 1;
+        plan->split_k = split_k > 0 ? split_k : fused_auto_split(M, N, G, sm_count);
+        if (split_k == 0) {
+            const int64_t tiles = ((M + fused::BT - 1) / fused::BT) * ((N + fused::BW - 1) / fused::BW);
+            const int sk = plan->split_k;
+            std::snprintf(plan->why, sizeof(plan->why), "%s,split:%lldx%lld", automatic ? "auto:M>64" : "forced",
+                          static_cast<long long>((tiles * sk + sm_count - 1) / sm_count),
+                          static_cast<long long>((G + sk - 1) / sk));
+        }
         plan->off_xh = 0;
         plan->off_rs = round_up(static_cast<size_t>(M) * K * 2, 256);
         plan->off_sb = plan->off_rs + round_up(static_cast<size_t>(M) * 4, 256);
@@ -262,25 +312,26 @@ ql_status run_gemv(const Plan& pl, const void* x, const uint32_t* codes, const v
     prof_begin(st);
     if (pl.bits == 8) {
         if (bf16_out)
-            gemv8_kernel<true><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
+            cc_stream8_kernel<true><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
         else
-            gemv8_kernel<false><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
+            cc_stream8_kernel<false><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
     } else {
         if (bf16_out)
-            gemv_kernel<true><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
+            cc_stream_kernel<true><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
         else
-            gemv_kernel<false><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
+            cc_stream_kernel<false><<<grid, kGemvWarps * 32, 0, st>>>(xb, codes, sc, bi, out, (int)M, (int)K, (int)N, partial);
     }
     prof_end(st);
     if (partial) {
         const int64_t count = M * N;
         const int blocks = static_cast<int>(std::min<int64_t>((count / 4 + 255) / 256, 8 * sm_count));
         if (bf16_out)
-            splitk_reduce_kernel<true><<<blocks, 256, 0, st>>>(static_cast<const float*>(ws), y, count, pl.split_k);
+            ordered_sum_kernel<true><<<blocks, 256, 0, st>>>(static_cast<const float*>(ws), y, count, pl.split_k);
         else
-            splitk_reduce_kernel<false><<<blocks, 256, 0, st>>>(static_cast<const float*>(ws), y, count, pl.split_k);
+            ordered_sum_kernel<false><<<blocks, 256, 0, st>>>(static_cast<const float*>(ws), y, count, pl.split_k);
     }
-    set_dispatch("path=gemv bits=%d warps=%d splitk=%d launches=%d", pl.bits, kGemvWarps, pl.split_k, partial ? 2 : 1);
+    set_dispatch("path=gemv bits=%d warps=%d splitk=%d launches=%d why=%s", pl.bits, kGemvWarps, pl.split_k,
+                 partial ? 2 : 1, pl.why);
     return launch_status();
 }
 
@@ -376,13 +427,13 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
         const int64_t count = M * N;
         const int blocks = static_cast<int>(std::min<int64_t>((count / 4 + 255) / 256, 8 * sm_count));
         if (bf16_out)
-            splitk_reduce_kernel<true><<<blocks, 256, 0, st>>>(part, y, count, pl.split_k);
+            ordered_sum_kernel<true><<<blocks, 256, 0, st>>>(part, y, count, pl.split_k);
         else
-            splitk_reduce_kernel<false><<<blocks, 256, 0, st>>>(part, y, count, pl.split_k);
+            ordered_sum_kernel<false><<<blocks, 256, 0, st>>>(part, y, count, pl.split_k);
         const int nc = bits == 4 ? fused::DefaultCfg::kNC : fused::Q8Cfg::kNC;
         const int nx = bits == 4 ? fused::DefaultCfg::kNX : fused::Q8Cfg::kNX;
-        set_dispatch("path=tc_fused bits=%d tile=%dw x %dt x %dk stages=x%d/c%d/a%d ctas=%d splitk=%d launches=4",
-                     bits, fused::BW, fused::BT, fused::BK, nx, nc, fused::NA, grid, pl.split_k);
+        set_dispatch("path=tc_fused bits=%d tile=%dw x %dt x %dk stages=x%d/c%d/a%d ctas=%d splitk=%d launches=4 why=%s",
+                     bits, fused::BW, fused::BT, fused::BK, nx, nc, fused::NA, grid, pl.split_k, pl.why);
         return launch_status();
     }
     if (bits == 4) {
@@ -402,10 +453,19 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     prof_end(st);
     const int nc = bits == 4 ? fused::DefaultCfg::kNC : fused::Q8Cfg::kNC;
     const int nx = bits == 4 ? fused::DefaultCfg::kNX : fused::Q8Cfg::kNX;
-    set_dispatch("path=tc_fused bits=%d tile=%dw x %dt x %dk stages=x%d/c%d/a%d ctas=%d splitk=1 launches=3", bits,
-                 fused::BW, fused::BT, fused::BK, nx, nc, fused::NA, grid);
+    set_dispatch("path=tc_fused bits=%d tile=%dw x %dt x %dk stages=x%d/c%d/a%d ctas=%d splitk=1 launches=3 why=%s",
+                 bits, fused::BW, fused::BT, fused::BK, nx, nc, fused::NA, grid, pl.why);
     (void)codes;
     return launch_status();
+}
+
+template <int NT, int B>
+ql_status launch_skinny(bool bf16_out, const CUtensorMap& mc, const CUtensorMap& mx, const CUtensorMap& ms,
+                        const CUtensorMap& mb, const skinny::Params& p, int ctas, cudaStream_t st) {
+    const dim3 grid(static_cast<unsigned>(ctas));
+    constexpr uint32_t smem = skinny::Layout<NT, B>::kSmemBytes;
+    return bf16_out ? launch_dependent(skinny::skinny_kernel<NT, B, true>, grid, skinny::kThreads, smem, st, mc, mx, ms, mb, p)
+                    : launch_dependent(skinny::skinny_kernel<NT, B, false>, grid, skinny::kThreads, smem, st, mc, mx, ms, mb, p);
 }
 
 ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const void* scales, const void* biases,
@@ -415,6 +475,7 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     void* xp = wsb + pl.off_xp;
     int* rowexp = reinterpret_cast<int*>(wsb + pl.off_re);
+    int* tile_count = reinterpret_cast<int*>(wsb + pl.off_tc);
     float* pmax = reinterpret_cast<float*>(wsb + pl.off_pm);
     CUtensorMap mc, mx;
     ql_status s;
@@ -441,6 +502,9 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     skinny::Params p;
     p.param_tma = param_tma ? 1 : 0;
     p.partial = reinterpret_cast<float*>(wsb);
+    p.tile_count = tile_count;
+    p.rowexp = rowexp;
+    p.y = y;
     p.scales = static_cast<const __half*>(scales);
     p.biases = static_cast<const __half*>(biases);
     p.M = static_cast<int>(M);
@@ -452,63 +516,34 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     p.units = pl.units;
     p.segmax = pl.segmax;
     p.partial_elems = static_cast<int64_t>(pl.ctas) * pl.segmax * M * skinny::BW;
-    // row maxima, then scaled and reordered f16 activations, per-group activation sums, row exponents
+    // per-slice row maxima and zeroed arrival counts (a plain launch: it reads x and rewrites the workspace,
+    // so it waits for everything before it), then the scaled and reordered f16 activations and row
+    // exponents under programmatic dependent launch
     const dim3 pre_grid(static_cast<unsigned>(pl.slices), static_cast<unsigned>(M));
-    skinny::skinny_rowmax_kernel<<<pre_grid, 256, 0, st>>>(static_cast<const uint4*>(x), pmax, static_cast<int>(K));
+    skinny::skinny_rowmax_kernel<<<pre_grid, skinny::kPrepThreads, 0, st>>>(static_cast<const uint4*>(x), pmax,
+                                                                           tile_count, p.num_w, static_cast<int>(K));
     if ((s = launch_status()) != QL_OK) return s;
-    {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = pre_grid;
-        cfg.blockDim = dim3(256);
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const float* pm = pmax;
-        const cudaError_t e =
-            bits == 4 ? cudaLaunchKernelEx(&cfg, skinny::skinny_prepass_kernel<4>, static_cast<const uint4*>(x), pm,
-                                           static_cast<uint4*>(xp), rowexp, static_cast<int>(K))
-                      : cudaLaunchKernelEx(&cfg, skinny::skinny_prepass_kernel<8>, static_cast<const uint4*>(x), pm,
-                                           static_cast<uint4*>(xp), rowexp, static_cast<int>(K));
-        if (e != cudaSuccess) return QL_ERR_CUDA;
-    }
+    s = bits == 4 ? launch_dependent(skinny::skinny_prepass_kernel<4>, pre_grid, skinny::kPrepThreads, 0, st,
+                                     static_cast<const uint4*>(x), static_cast<const float*>(pmax),
+                                     static_cast<uint4*>(xp), rowexp, static_cast<int>(K))
+                  : launch_dependent(skinny::skinny_prepass_kernel<8>, pre_grid, skinny::kPrepThreads, 0, st,
+                                     static_cast<const uint4*>(x), static_cast<const float*>(pmax),
+                                     static_cast<uint4*>(xp), rowexp, static_cast<int>(K));
+    if (s != QL_OK) return s;
     prof_begin(st);
-    const dim3 sgrid(static_cast<unsigned>(pl.ctas));
-    if (bits == 4 && pl.nt == 16)
-        s = launch_dependent(skinny::skinny_kernel<16, 4>, sgrid, skinny::kThreads, skinny::Layout<16, 4>::kSmemBytes, st,
-                             mc, mx, ms, mb, p);
-    else if (bits == 4 && pl.nt == 32)
-        s = launch_dependent(skinny::skinny_kernel<32, 4>, sgrid, skinny::kThreads, skinny::Layout<32, 4>::kSmemBytes, st,
-                             mc, mx, ms, mb, p);
-    else if (bits == 4)
-        s = launch_dependent(skinny::skinny_kernel<64, 4>, sgrid, skinny::kThreads, skinny::Layout<64, 4>::kSmemBytes, st,
-                             mc, mx, ms, mb, p);
-    else if (pl.nt == 16)
-        s = launch_dependent(skinny::skinny_kernel<16, 8>, sgrid, skinny::kThreads, skinny::Layout<16, 8>::kSmemBytes, st,
-                             mc, mx, ms, mb, p);
-    else if (pl.nt == 32)
-        s = launch_dependent(skinny::skinny_kernel<32, 8>, sgrid, skinny::kThreads, skinny::Layout<32, 8>::kSmemBytes, st,
-                             mc, mx, ms, mb, p);
+    if (bits == 4)
+        s = pl.nt == 16 ? launch_skinny<16, 4>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st)
+          : pl.nt == 32 ? launch_skinny<32, 4>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st)
+                        : launch_skinny<64, 4>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st);
     else
-        s = launch_dependent(skinny::skinny_kernel<64, 8>, sgrid, skinny::kThreads, skinny::Layout<64, 8>::kSmemBytes, st,
-                             mc, mx, ms, mb, p);
+        s = pl.nt == 16 ? launch_skinny<16, 8>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st)
+          : pl.nt == 32 ? launch_skinny<32, 8>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st)
+                        : launch_skinny<64, 8>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st);
     if (s != QL_OK) return s;
     prof_end(st);
-    const float* part = p.partial;
-    const int* rexp = rowexp;
-    const dim3 red_grid(static_cast<unsigned>(p.num_w), static_cast<unsigned>((M + 1) / 2));
-    if (bf16_out)
-        s = launch_dependent(skinny::skinny_reduce_kernel<true>, red_grid, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
-                             p.units, pl.ctas, pl.segmax, p.partial_elems);
-    else
-        s = launch_dependent(skinny::skinny_reduce_kernel<false>, red_grid, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
-                             p.units, pl.ctas, pl.segmax, p.partial_elems);
-    if (s != QL_OK) return s;
     (void)sm_count;
-    set_dispatch("path=tc_skinny bits=%d nt=%d ctas=%d segmax=%d units=%lld launches=4", bits, pl.nt, pl.ctas,
-                 pl.segmax, static_cast<long long>(pl.units));
+    set_dispatch("path=tc_skinny bits=%d nt=%d ctas=%d segmax=%d units=%lld launches=3 why=%s", bits, pl.nt, pl.ctas,
+                 pl.segmax, static_cast<long long>(pl.units), pl.why);
     return launch_status();
 }
 
@@ -780,6 +815,21 @@ ql_status qlinear_selftest_bounded_wait(cudaStream_t stream) {
     return launch_status();
 }
 
+ql_status qlinear_test_stall(int32_t kernel_mask, uint64_t wait_limit_ns) {
+#ifdef QL_BOUNDS_CHECK
+    if (kernel_mask < 0 || kernel_mask > (kStallFused | kStallSkinny) || wait_limit_ns == 0) return QL_ERR_INVALID_ARG;
+    const unsigned long long limit = wait_limit_ns;
+    if (cudaMemcpyToSymbol(g_stall_mask, &kernel_mask, sizeof(kernel_mask)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_wait_limit_ns, &limit, sizeof(limit)) != cudaSuccess)
+        return QL_ERR_CUDA;
+    return QL_OK;
+#else
+    (void)kernel_mask;
+    (void)wait_limit_ns;
+    return QL_ERR_UNSUPPORTED;
+#endif
+}
+
 ql_status qlinear_reduce_partials(const float* partials, int32_t S, int64_t count, void* y, ql_dtype out_dtype,
                                   cudaStream_t stream) {
     if (!partials || !y || S < 1 || count < 4 || count % 4 != 0) return QL_ERR_INVALID_ARG;
@@ -792,9 +842,9 @@ ql_status qlinear_reduce_partials(const float* partials, int32_t S, int64_t coun
     if ((s = device_info(&dev)) != QL_OK) return s;
     const int blocks = static_cast<int>(std::min<int64_t>((count / 4 + 255) / 256, 8 * dev->sm_count));
     if (out_dtype == QL_BF16)
-        splitk_reduce_kernel<true><<<blocks, 256, 0, stream>>>(partials, y, count, S);
+        ordered_sum_kernel<true><<<blocks, 256, 0, stream>>>(partials, y, count, S);
     else
-        splitk_reduce_kernel<false><<<blocks, 256, 0, stream>>>(partials, y, count, S);
+        ordered_sum_kernel<false><<<blocks, 256, 0, stream>>>(partials, y, count, S);
     return launch_status();
 }
 

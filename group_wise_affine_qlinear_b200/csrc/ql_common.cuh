@@ -45,6 +45,23 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // records QL_ERR_DEVICE_TIMEOUT and lets the kernel unwind.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;   // 1 s
 
+// Kernels whose code producer the checked build can hold back (qlinear_test_stall).
+constexpr int kStallFused = 1, kStallSkinny = 2;
+
+#ifdef QL_BOUNDS_CHECK
+// Test hooks of the checked build (the index-checked variant): the host can shorten the wait limit and
+// hold back the code producer of the kernels in a mask, so that a real pipeline's waits expire with no
+// copy or MMA in flight and its unwinding can be tested.  The shipped build has neither: its limit is
+// the constant above and nothing is held back.
+static __device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+static __device__ int g_stall_mask;
+__device__ __forceinline__ uint64_t wait_limit_ns() { return g_wait_limit_ns; }
+__device__ __forceinline__ bool stalled(int kernel_bit) { return (g_stall_mask & kernel_bit) != 0; }
+#else
+__device__ __forceinline__ constexpr uint64_t wait_limit_ns() { return kWaitLimitNs; }
+__device__ __forceinline__ constexpr bool stalled(int) { return false; }
+#endif
+
 __device__ __forceinline__ uint32_t bits_of(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 half2_of(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 

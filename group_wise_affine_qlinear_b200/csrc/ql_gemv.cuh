@@ -92,7 +92,7 @@ __device__ __forceinline__ void gemv_body(
 }
 
 template <bool kBf16Out>
-__global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(
+__global__ void __launch_bounds__(kGemvWarps * 32) cc_stream_kernel(
     const __nv_bfloat16* __restrict__ x, const uint32_t* __restrict__ codes,
     const __half* __restrict__ scales, const __half* __restrict__ biases,
     void* __restrict__ out, int M, int K, int N, bool partial_out) {
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(
 // The same split-K GEMV for 8-bit codes (codes uint32 [N][K/4], low byte first): each lane step
 // streams a quarter group (16 codes, one 128-bit load) and the 16 matching activations.
 template <bool kBf16Out>
-__global__ void __launch_bounds__(kGemvWarps * 32) gemv8_kernel(
+__global__ void __launch_bounds__(kGemvWarps * 32) cc_stream8_kernel(
     const __nv_bfloat16* __restrict__ x, const uint32_t* __restrict__ codes,
     const __half* __restrict__ scales, const __half* __restrict__ biases,
     void* __restrict__ out, int M, int K, int N, bool partial_out) {
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv8_kernel(
 // y[i] = sum_{z=0}^{S-1} partial[z][i] in that fixed order (deterministic), four
 // elements per thread.  count = M*N is a multiple of 8.
 template <bool kBf16Out>
-__device__ __forceinline__ void splitk_reduce_body(const float* __restrict__ partial, void* __restrict__ y,
+__device__ __forceinline__ void ordered_sum_body(const float* __restrict__ partial, void* __restrict__ y,
                                                    int64_t count, int S) {
     const int64_t n4 = count / 4;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -201,9 +201,9 @@ __device__ __forceinline__ void splitk_reduce_body(const float* __restrict__ par
 }
 
 template <bool kBf16Out>
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ partial,
+__global__ void __launch_bounds__(256) ordered_sum_kernel(const float* __restrict__ partial,
                                                             void* __restrict__ y, int64_t count, int S) {
-    splitk_reduce_body<kBf16Out>(partial, y, count, S);
+    ordered_sum_body<kBf16Out>(partial, y, count, S);
 }
 
 // Split factor of the weight-streaming path: double it while the grid has fewer

@@ -17,6 +17,16 @@
 // calls that overlap on the GPU (different streams, or several host threads)
 // race on it and must be serialized by the caller.  Nothing in it needs to
 // start at zero -- each call writes every partial it later reads.
+//
+// The cached address belongs to the device's context as it was at the first
+// call: after cudaDeviceReset on that device the cached address is stale, so
+// this entry point must not be used across a device reset.
+//
+// Size bound: the split factor keeps S * N / 8 below 8 * SMs (it stops
+// doubling once the grid has four waves of 8-row CTAs), so the partials of a
+// call need S * M * N * 4 < 256 * SMs * M bytes: 2.4 MB at M = 64 on the 148
+// SMs of a B200.  Parts with more than 256 SMs could exceed the array; such a
+// shape is refused with QL_ERR_WORKSPACE before anything is launched.
 #include <algorithm>
 #include <mutex>
 
@@ -27,6 +37,8 @@ namespace {
 
 constexpr size_t kScratchBytes = QL_NOALLOC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
+static_assert(kScratchBytes >= size_t(256) * 148 * QL_NOALLOC_MAX_M,
+              "the scratch array holds the largest partials of a B200 (148 SMs) at the maximum M");
 
 static __device__ __align__(256) float g_noalloc_scratch[kScratchBytes / sizeof(float)];
 
@@ -49,7 +61,7 @@ ql_status scratch_address(float** out, int* sm_count) {
 }
 
 template <bool kBf16Out>
-__global__ void __launch_bounds__(ql::kGemvWarps * 32) noalloc_gemv_kernel(
+__global__ void __launch_bounds__(ql::kGemvWarps * 32) noalloc_stream_kernel(
     const __nv_bfloat16* __restrict__ x, const uint32_t* __restrict__ codes, const __half* __restrict__ scales,
     const __half* __restrict__ biases, void* __restrict__ out, int M, int K, int N, bool partial_out) {
     ql::gemv_body<kBf16Out>(x, codes, scales, biases, out, M, K, N, partial_out);
@@ -58,7 +70,7 @@ __global__ void __launch_bounds__(ql::kGemvWarps * 32) noalloc_gemv_kernel(
 template <bool kBf16Out>
 __global__ void __launch_bounds__(256) noalloc_reduce_kernel(const float* __restrict__ partial, void* __restrict__ y,
                                                              int64_t count, int S) {
-    ql::splitk_reduce_body<kBf16Out>(partial, y, count, S);
+    ql::ordered_sum_body<kBf16Out>(partial, y, count, S);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -87,6 +99,10 @@ QL_API ql_status qlinear_forward_noalloc(const void* x, const uint32_t* codes, c
     if (overlap(y, yb, x, xb) || overlap(y, yb, codes, cb) || overlap(y, yb, scales, pb) || overlap(y, yb, biases, pb))
         return QL_ERR_INVALID_ARG;
 
+    // An error left pending by some earlier launch is not this call's: report it without launching
+    // (and without clearing it), so that the error read after the launches below is this call's own.
+    if (cudaPeekAtLastError() != cudaSuccess) return QL_ERR_CUDA;
+
     float* scratch = nullptr;
     int sms = 0;
     ql_status s = scratch_address(&scratch, &sms);
@@ -99,7 +115,7 @@ QL_API ql_status qlinear_forward_noalloc(const void* x, const uint32_t* codes, c
     auto sp = static_cast<const __half*>(scales);
     auto bp = static_cast<const __half*>(biases);
     const dim3 grid(static_cast<unsigned>(N / ql::kGemvWarps), static_cast<unsigned>(S));
-    noalloc_gemv_kernel<true><<<grid, ql::kGemvWarps * 32, 0, stream>>>(xp, codes, sp, bp, S > 1 ? scratch : y,
+    noalloc_stream_kernel<true><<<grid, ql::kGemvWarps * 32, 0, stream>>>(xp, codes, sp, bp, S > 1 ? scratch : y,
                                                                         (int)M, (int)K, (int)N, S > 1);
     if (S > 1) {
         const int64_t count = M * N;

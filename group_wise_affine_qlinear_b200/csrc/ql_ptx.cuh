@@ -56,7 +56,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     while (true) {
         if (mbar_test(a, parity)) return true;
         if (abort != nullptr && *abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > wait_limit_ns()) {
             record_status(QL_ERR_DEVICE_TIMEOUT);
             if (abort != nullptr) *abort = 1;
             return false;

@@ -284,7 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         }
     } else if (warp == kWarpTmaX || warp == kWarpTmaC) {
         // ---------------------------------------------------------------- TMA producers
-        if (lane == 0) {
+        // (the checked build's stall hook holds the code producer back: no code or parameter load)
+        if (lane == 0 && !(warp == kWarpTmaC && stalled(kStallFused))) {
             const bool is_x = warp == kWarpTmaX;
             const int depth = is_x ? NX : NC;
             uint64_t* full = is_x ? x_full : c_full;

@@ -170,6 +170,19 @@ QL_API ql_status qlinear_get_device_status(cudaStream_t stream);
 QL_API ql_status qlinear_last_dispatch(char* buf, size_t len);
 
 /*
+ * Test hook of the checked build (libqlinear_bounds.so, compiled with QL_BOUNDS_CHECK); the pages have no
+ * counterpart.  kernel_mask bit 0 holds back the code producer of the fused tensor-core kernel
+ * (QL_PATH_TC_FUSED), bit 1 that of the weight-streaming kernel (QL_PATH_TC_SKINNY): they issue no code
+ * or parameter load, so the kernel's other roles wait until the limit, record QL_ERR_DEVICE_TIMEOUT and
+ * unwind (nothing of theirs in flight, tensor memory freed).  wait_limit_ns replaces the one-second
+ * limit of every bounded wait in the library's kernels (> 0); call with kernel_mask 0 and 1000000000
+ * to restore the defaults.  Synchronous (two small host-to-device copies on the legacy stream).
+ * The shipped library returns QL_ERR_UNSUPPORTED and changes nothing; QL_ERR_INVALID_ARG for an
+ * unknown bit or a zero limit.
+ */
+QL_API ql_status qlinear_test_stall(int32_t kernel_mask, uint64_t wait_limit_ns);
+
+/*
  * Allocation-free forward for small M.  The pages have no counterpart of this
  * call; it exists for callers that cannot allocate device memory where they
  * run the layer (a plugin living inside another engine's fixed memory pool, a
@@ -187,7 +200,12 @@ QL_API ql_status qlinear_last_dispatch(char* buf, size_t len);
  * All calls share the one array and it keeps the last call's contents: calls
  * that overlap on the GPU (other streams or host threads) race and must be
  * serialized by the caller.  No cudaMalloc, cudaFree or allocating library
- * routine is called.
+ * routine is called.  The cached address is that of the context current at
+ * the first call: do not use this entry point across cudaDeviceReset.  A
+ * launch error already pending on the calling thread when the call is made
+ * returns QL_ERR_CUDA before anything is launched and is left pending.
+ * It runs the CUDA-core split-K path (QL_PATH_GEMV), whose cost grows with M
+ * (each 4-row block of activations streams the weights again).
  */
 #define QL_NOALLOC_SCRATCH_BYTES (4u << 20)
 #define QL_NOALLOC_MAX_M 64

@@ -111,6 +111,35 @@ def test_workspace_size_values(L):
     assert L.qlinear_workspace_size(16, 100, 256, 64) == ctypes.c_size_t(-1).value
 
 
+# The dispatcher's choice, read through the workspace it asks for (the library assumes a B200's 148
+# SMs when no GPU is present).  Expected choices are the fastest forced configurations measured on a
+# B200 for these shapes (or within 5% of it): the weight-streaming kernel up to 64 tokens, then the
+# fused kernel split so that ceil(tiles * S / SMs) waves of ceil(G / S) K-steps are fewest.
+DISPATCH_TABLE = [
+    # (M, K, N, path, split) -- text projection 53248 -> 4608, QKV 4608 -> 13824, MLP down 18432 -> 4608
+    (1, 53248, 4608, ql.PATH_TC_SKINNY, 0), (32, 53248, 4608, ql.PATH_TC_SKINNY, 0),
+    (33, 53248, 4608, ql.PATH_TC_SKINNY, 0), (64, 53248, 4608, ql.PATH_TC_SKINNY, 0),
+    (65, 53248, 4608, ql.PATH_TC_FUSED, 8), (128, 53248, 4608, ql.PATH_TC_FUSED, 8),
+    (192, 53248, 4608, ql.PATH_TC_FUSED, 8), (256, 53248, 4608, ql.PATH_TC_FUSED, 4),
+    (384, 53248, 4608, ql.PATH_TC_FUSED, 4), (512, 53248, 4608, ql.PATH_TC_FUSED, 5),
+    (128, 4608, 13824, ql.PATH_TC_FUSED, 2), (256, 4608, 13824, ql.PATH_TC_FUSED, 1),
+    (512, 4608, 13824, ql.PATH_TC_FUSED, 1), (1024, 4608, 13824, ql.PATH_TC_FUSED, 1),
+    (4608, 4608, 13824, ql.PATH_TC_FUSED, 1),
+    (128, 18432, 4608, ql.PATH_TC_FUSED, 8), (512, 18432, 4608, ql.PATH_TC_FUSED, 5),
+    (4608, 18432, 4608, ql.PATH_TC_FUSED, 1),
+]
+
+
+@pytest.mark.parametrize("M,K,N,path,split", DISPATCH_TABLE)
+def test_dispatcher_table(L, M, K, N, path, split):
+    auto = ql.workspace_size(M, K, N)
+    assert auto == ql.workspace_size(M, K, N, path, split)
+    if path == ql.PATH_TC_FUSED:
+        for other in (1, 2, 4, 8, 12, 16):
+            if other != split:
+                assert ql.workspace_size(M, K, N, path, other) != auto
+
+
 def test_profile_events_pairing(L):
     assert L.qlinear_set_profile_events(FAKE, None) == 1
     assert L.qlinear_set_profile_events(None, None) == 0
@@ -198,7 +227,7 @@ def test_reduce_partials_validation(L):
 def test_fused_split_k_workspace(L):
     """The fused path's split-K adds fp32 partials [S][M][N] to its workspace; more slices than groups is an error."""
     M, K, N = 512, 53248, 4608
-    base = ql.workspace_size(M, K, N, ql.PATH_TC_FUSED)
+    base = ql.workspace_size(M, K, N, ql.PATH_TC_FUSED, 1)
     assert ql.workspace_size(M, K, N, ql.PATH_TC_FUSED, 8) == base + 8 * M * N * 4
     assert L.qlinear_workspace_size_config(16, 256, 256, 64, ql.PATH_TC_FUSED, 5) == ctypes.c_size_t(-1).value
 
