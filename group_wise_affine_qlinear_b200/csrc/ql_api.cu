@@ -70,11 +70,7 @@ struct DeviceInfo {
 
 template <int NT, int B>
 cudaError_t skinny_smem_attr() {
-    const cudaError_t e = cudaFuncSetAttribute(skinny::skinny_kernel<NT, B, true>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               skinny::Layout<NT, B>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(skinny::skinny_kernel<NT, B, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(skinny::skinny_kernel<NT, B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 skinny::Layout<NT, B>::kSmemBytes);
 }
 
@@ -204,9 +200,8 @@ struct Plan {
     size_t workspace = 0;
     // fused path workspace carve-up (off_part: fp32 partials [split_k][M][N] when the K-steps are split)
     size_t off_xh = 0, off_rs = 0, off_sb = 0, off_part = 0;
-    // skinny path workspace carve-up: partials, scaled f16 activations, row exponents, per-tile arrival
-    // counts, per-slice row maxima (`slices` prepass blocks per row)
-    size_t off_xp = 0, off_re = 0, off_tc = 0, off_pm = 0;
+    // skinny path workspace carve-up: partials, scaled f16 activations, row exponents, per-slice row maxima
+    size_t off_xp = 0, off_re = 0, off_pm = 0;
     int slices = 0;
 };
 
@@ -270,10 +265,8 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         plan->split_k = 1;
         plan->off_xp = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * M * skinny::BW * sizeof(float), 256);
         plan->off_re = plan->off_xp + round_up(static_cast<size_t>(M) * K * 2, 256);
-        plan->off_tc = plan->off_re + round_up(static_cast<size_t>(plan->nt) * sizeof(int), 256);
-        plan->off_pm = plan->off_tc + round_up(static_cast<size_t>((N + skinny::BW - 1) / skinny::BW) * sizeof(int), 256);
-        // about one prepass block per SM in all, each slice at least one 16-byte load per thread
-        plan->slices = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sm_count / M, K / 8 / skinny::kPrepThreads)));
+        plan->slices = static_cast<int>((K / 8 + 255) / 256);
+        plan->off_pm = plan->off_re + round_up(static_cast<size_t>(plan->nt) * sizeof(int), 256);
         plan->workspace = plan->off_pm + round_up(static_cast<size_t>(M) * plan->slices * sizeof(float), 256);
         return QL_OK;
     }
@@ -459,15 +452,6 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     return launch_status();
 }
 
-template <int NT, int B>
-ql_status launch_skinny(bool bf16_out, const CUtensorMap& mc, const CUtensorMap& mx, const CUtensorMap& ms,
-                        const CUtensorMap& mb, const skinny::Params& p, int ctas, cudaStream_t st) {
-    const dim3 grid(static_cast<unsigned>(ctas));
-    constexpr uint32_t smem = skinny::Layout<NT, B>::kSmemBytes;
-    return bf16_out ? launch_dependent(skinny::skinny_kernel<NT, B, true>, grid, skinny::kThreads, smem, st, mc, mx, ms, mb, p)
-                    : launch_dependent(skinny::skinny_kernel<NT, B, false>, grid, skinny::kThreads, smem, st, mc, mx, ms, mb, p);
-}
-
 ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const void* scales, const void* biases,
                      void* y, bool bf16_out, int64_t M, int64_t K, int64_t N, void* ws, cudaStream_t st,
                      int sm_count) {
@@ -475,7 +459,6 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     void* xp = wsb + pl.off_xp;
     int* rowexp = reinterpret_cast<int*>(wsb + pl.off_re);
-    int* tile_count = reinterpret_cast<int*>(wsb + pl.off_tc);
     float* pmax = reinterpret_cast<float*>(wsb + pl.off_pm);
     CUtensorMap mc, mx;
     ql_status s;
@@ -502,9 +485,6 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     skinny::Params p;
     p.param_tma = param_tma ? 1 : 0;
     p.partial = reinterpret_cast<float*>(wsb);
-    p.tile_count = tile_count;
-    p.rowexp = rowexp;
-    p.y = y;
     p.scales = static_cast<const __half*>(scales);
     p.biases = static_cast<const __half*>(biases);
     p.M = static_cast<int>(M);
@@ -516,33 +496,62 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     p.units = pl.units;
     p.segmax = pl.segmax;
     p.partial_elems = static_cast<int64_t>(pl.ctas) * pl.segmax * M * skinny::BW;
-    // per-slice row maxima and zeroed arrival counts (a plain launch: it reads x and rewrites the workspace,
-    // so it waits for everything before it), then the scaled and reordered f16 activations and row
-    // exponents under programmatic dependent launch
+    // row maxima, then scaled and reordered f16 activations, per-group activation sums, row exponents
     const dim3 pre_grid(static_cast<unsigned>(pl.slices), static_cast<unsigned>(M));
-    skinny::skinny_rowmax_kernel<<<pre_grid, skinny::kPrepThreads, 0, st>>>(static_cast<const uint4*>(x), pmax,
-                                                                           tile_count, p.num_w, static_cast<int>(K));
+    skinny::skinny_rowmax_kernel<<<pre_grid, 256, 0, st>>>(static_cast<const uint4*>(x), pmax, static_cast<int>(K));
     if ((s = launch_status()) != QL_OK) return s;
-    s = bits == 4 ? launch_dependent(skinny::skinny_prepass_kernel<4>, pre_grid, skinny::kPrepThreads, 0, st,
-                                     static_cast<const uint4*>(x), static_cast<const float*>(pmax),
-                                     static_cast<uint4*>(xp), rowexp, static_cast<int>(K))
-                  : launch_dependent(skinny::skinny_prepass_kernel<8>, pre_grid, skinny::kPrepThreads, 0, st,
-                                     static_cast<const uint4*>(x), static_cast<const float*>(pmax),
-                                     static_cast<uint4*>(xp), rowexp, static_cast<int>(K));
-    if (s != QL_OK) return s;
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = pre_grid;
+        cfg.blockDim = dim3(256);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const float* pm = pmax;
+        const cudaError_t e =
+            bits == 4 ? cudaLaunchKernelEx(&cfg, skinny::skinny_prepass_kernel<4>, static_cast<const uint4*>(x), pm,
+                                           static_cast<uint4*>(xp), rowexp, static_cast<int>(K))
+                      : cudaLaunchKernelEx(&cfg, skinny::skinny_prepass_kernel<8>, static_cast<const uint4*>(x), pm,
+                                           static_cast<uint4*>(xp), rowexp, static_cast<int>(K));
+        if (e != cudaSuccess) return QL_ERR_CUDA;
+    }
     prof_begin(st);
-    if (bits == 4)
-        s = pl.nt == 16 ? launch_skinny<16, 4>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st)
-          : pl.nt == 32 ? launch_skinny<32, 4>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st)
-                        : launch_skinny<64, 4>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st);
+    const dim3 sgrid(static_cast<unsigned>(pl.ctas));
+    if (bits == 4 && pl.nt == 16)
+        s = launch_dependent(skinny::skinny_kernel<16, 4>, sgrid, skinny::kThreads, skinny::Layout<16, 4>::kSmemBytes, st,
+                             mc, mx, ms, mb, p);
+    else if (bits == 4 && pl.nt == 32)
+        s = launch_dependent(skinny::skinny_kernel<32, 4>, sgrid, skinny::kThreads, skinny::Layout<32, 4>::kSmemBytes, st,
+                             mc, mx, ms, mb, p);
+    else if (bits == 4)
+        s = launch_dependent(skinny::skinny_kernel<64, 4>, sgrid, skinny::kThreads, skinny::Layout<64, 4>::kSmemBytes, st,
+                             mc, mx, ms, mb, p);
+    else if (pl.nt == 16)
+        s = launch_dependent(skinny::skinny_kernel<16, 8>, sgrid, skinny::kThreads, skinny::Layout<16, 8>::kSmemBytes, st,
+                             mc, mx, ms, mb, p);
+    else if (pl.nt == 32)
+        s = launch_dependent(skinny::skinny_kernel<32, 8>, sgrid, skinny::kThreads, skinny::Layout<32, 8>::kSmemBytes, st,
+                             mc, mx, ms, mb, p);
     else
-        s = pl.nt == 16 ? launch_skinny<16, 8>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st)
-          : pl.nt == 32 ? launch_skinny<32, 8>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st)
-                        : launch_skinny<64, 8>(bf16_out, mc, mx, ms, mb, p, pl.ctas, st);
+        s = launch_dependent(skinny::skinny_kernel<64, 8>, sgrid, skinny::kThreads, skinny::Layout<64, 8>::kSmemBytes, st,
+                             mc, mx, ms, mb, p);
     if (s != QL_OK) return s;
     prof_end(st);
+    const float* part = p.partial;
+    const int* rexp = rowexp;
+    const dim3 red_grid(static_cast<unsigned>(p.num_w), static_cast<unsigned>((M + 1) / 2));
+    if (bf16_out)
+        s = launch_dependent(skinny::skinny_reduce_kernel<true>, red_grid, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
+                             p.units, pl.ctas, pl.segmax, p.partial_elems);
+    else
+        s = launch_dependent(skinny::skinny_reduce_kernel<false>, red_grid, 256, 0, st, part, rexp, y, p.M, p.N, p.cpt,
+                             p.units, pl.ctas, pl.segmax, p.partial_elems);
+    if (s != QL_OK) return s;
     (void)sm_count;
-    set_dispatch("path=tc_skinny bits=%d nt=%d ctas=%d segmax=%d units=%lld launches=3 why=%s", bits, pl.nt, pl.ctas,
+    set_dispatch("path=tc_skinny bits=%d nt=%d ctas=%d segmax=%d units=%lld launches=4 why=%s", bits, pl.nt, pl.ctas,
                  pl.segmax, static_cast<long long>(pl.units), pl.why);
     return launch_status();
 }

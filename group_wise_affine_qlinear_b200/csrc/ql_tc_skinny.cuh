@@ -14,26 +14,20 @@
 // kernel's arithmetic (one f16 rounding of each weight, activations scaled per
 // row by a power of two into f16, fp32 accumulation) in a layout for few tokens.
 //
-// The activations come from a prepass pair of about one small block per SM each:
+// The activations come from a prepass pair under programmatic dependent launch:
 // per-slice row maxima, then x' = f16(x * 2^e_t) with e_t putting the row maximum
 // in [2^14, 2^15), in the order the dequantizer emits its pairs in (0,4,1,5,2,6,3,7
-// of every 8-block for 4-bit codes, 0,2,1,3,4,6,5,7 for 8-bit codes).  Their
-// blocks are small enough (128 threads, 32 registers) to share an SM with a
-// streaming CTA, so the main kernel, launched behind them under programmatic
-// dependent launch, gets every SM at once: it starts streaming codes and
-// parameters immediately and waits for the prepass only before its first
-// activation load and its first reduction.
+// of every 8-block for 4-bit codes, 0,2,1,3,4,6,5,7 for 8-bit codes).  The main kernel starts streaming codes and parameters at
+// once and waits for the prepass only before its first activation load.
 //
 // Stream-K schedule: the work is cut into chunks of CG consecutive groups of one
 // 128-row tile (CG = 8 for 4-bit codes, 4 for the 8-bit codes of the Q8 pack,
 // huggingface "SceneWorks/ideogram-4-mlx", Versions; either way 32 KB of codes; a
 // tile has ceil(G/CG) chunks; a tile's last chunk may be partial).  The chunks, tile-major, are split into one equal contiguous run per
 // CTA; each tile segment a run covers leaves one fp32 partial [tokens][128]
-// (scaled by 2^e_t) in the workspace.  The CTA that publishes the last partial of
-// a tile (a per-tile arrival count, zeroed by the prepass) sums the partials of the
-// CTAs that covered the tile in CTA order -- the same order whichever CTA comes
-// last, so the result is deterministic -- scales back by 2^-e_t and writes y.  A
-// call is three launches: the two prepass kernels and this kernel.
+// (scaled by 2^e_t) in the workspace, and the reduce kernel sums, per output, the
+// partials of the CTAs that covered its tile in CTA order (deterministic) and
+// scales back by 2^-e_t.
 //
 // Roles step over pairs of consecutive groups of a chunk (pair j = groups 2j,
 // 2j+1), numbered pc along the run: four builder copies (pc % 4) and two MMA
@@ -50,8 +44,7 @@
 //                 loads from L2 take about a microsecond, so they run several chunks ahead
 //   warps 2, 3    MMA issuers for even / odd pairs (warp 2 also allocates TMEM)
 //   warps 4-19    A builders, copies 0-3 of 4 warps: one weight row per thread
-//   warps 20-23   drain: one weight row per thread, at the end of each tile segment; the
-//                 tile's reduction when this CTA completes it
+//   warps 20-23   drain: one weight row per thread, at the end of each tile segment
 #pragma once
 
 #include "ql_ptx.cuh"
@@ -71,9 +64,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBoxBytes = BW * 128;                     // 16 KB: one code box, 128 bytes of each row
 constexpr int kParGroups = 8;                                // groups per scale (bias) box: 16-byte rows
 constexpr uint32_t kParHalf = BW * kParGroups * 2;           // one box of scales (or biases): [128][8] f16
-constexpr int kMaxCtas = 256;                // the planner launches at most this many CTAs
-constexpr int kPrepThreads = 128;            // prepass block: 128 threads at <= 32 registers fit beside a
-                                             // streaming CTA (768 threads x 80 registers) on one SM
+constexpr int kMaxCtas = 256;                // the planner launches at most this many CTAs, so every
+                                             // tile's covering CTAs fit the reduce kernel's list
 static_assert(NA % kBuildCopies == 0 && NA % kMmaCopies == 0, "every A stage serves one copy of each role");
 
 // NT tokens, B-bit codes.  A chunk is CG groups: 8 for 4-bit codes (four pairs, one per builder copy),
@@ -94,10 +86,9 @@ struct Layout {
     static constexpr uint32_t kOffC = 0;                                  // [NC][codes | scales | biases]
     static constexpr uint32_t kOffX = kOffC + NC * kStageBytes;          // [NXC][CG][x tile], 1 KB aligned
     static constexpr uint32_t kOffBar = kOffX + NXC * kXBytes;
-    static constexpr uint32_t kNumBars = 2 * NC + 2 * NXC + 2 * NA + 4 + kMmaCopies + 2;
-    static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;                     // TMEM base, abort flag, flags
-    static constexpr uint32_t kOffCover = kOffMisc + 16;                             // [kMaxCtas] partial offsets
-    static constexpr uint32_t kSmemBytes = kOffCover + kMaxCtas * 8 + 1024;
+    static constexpr uint32_t kNumBars = 2 * NC + 2 * NXC + 2 * NA + 4 + kMmaCopies;
+    static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
     static constexpr uint32_t kAccCol = 0;                                // accumulator (set e, issuer c) at (2e+c)*NT
     static constexpr uint32_t kACol = 4 * NT;                             // A stage st, half h at kACol + 32(2st+h)
     static_assert(B == 4 || B == 8, "4- or 8-bit codes");
@@ -112,9 +103,6 @@ struct Layout {
 
 struct Params {
     float* partial;          // [P][segmax][M][128] fp32, scaled by 2^e_t
-    int* tile_count;         // [num_w] partials published per tile (zeroed by the prepass)
-    const int* rowexp;       // [M] -e_t (from the prepass)
-    void* y;                 // [M][N] bf16 or fp32
     const __half* scales;    // [N][G]
     const __half* biases;    // [N][G]
     int param_tma;           // 1: scales/biases arrive as TMA tiles (needs G % 8 == 0); 0: direct loads
@@ -130,61 +118,44 @@ __host__ __device__ __forceinline__ int64_t run_first(int64_t units, int P, int 
     return units * c / P;
 }
 
-// Activation prepass, two kernels over a grid of (slice, row) sized to about one block per SM, each
-// block 128 threads at <= 32 registers so that it fits on an SM beside a streaming CTA: the main kernel,
-// launched behind the second under programmatic dependent launch, then gets every SM at once.  Each
-// thread keeps kPrepUnroll 16-byte loads in flight.
-constexpr int kPrepUnroll = 4;
+// Activation prepass, two kernels over a grid of (slice, row): one thread per 8-block of k, 256 per
+// CTA, so every 8-block of a row is read in parallel.
 
-// pmax[t][slice] = max |x[t][k]| over the slice's 8-blocks.  Block (0, 0) also zeroes the per-tile
-// arrival counts of the main kernel's reduction.
-__global__ void __launch_bounds__(kPrepThreads, 16) skinny_rowmax_kernel(const uint4* __restrict__ x,
-                                                                        float* __restrict__ pmax,
-                                                                        int* __restrict__ tile_count, int num_w,
-                                                                        int K) {
+// pmax[t][slice] = max |x[t][k]| over the slice's 8-blocks.
+__global__ void __launch_bounds__(256) skinny_rowmax_kernel(const uint4* __restrict__ x, float* __restrict__ pmax,
+                                                            int K) {
     ptx::launch_dependents();
-    __shared__ float red[kPrepThreads / 32];
-    const int t = blockIdx.y, kb = K / 8, S = gridDim.x;
-    const int c0 = static_cast<int>((static_cast<int64_t>(blockIdx.x) * kb) / S);
-    const int c1 = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * kb) / S);
-    const uint4* row = x + static_cast<int64_t>(t) * kb;
+    __shared__ float red[8];
+    const int t = blockIdx.y, kb = K / 8;
+    const int c = blockIdx.x * 256 + threadIdx.x;
     float m = 0.0f;
-    for (int c = c0 + threadIdx.x; c < c1; c += kPrepUnroll * kPrepThreads) {
-        uint4 v[kPrepUnroll];
-#pragma unroll
-        for (int u = 0; u < kPrepUnroll; ++u)
-            if (c + u * kPrepThreads < c1) v[u] = row[c + u * kPrepThreads];
-#pragma unroll
-        for (int u = 0; u < kPrepUnroll; ++u)
-            if (c + u * kPrepThreads < c1)
-                m = fmaxf(m, fmaxf(fmaxf(fmaxf(fabsf(bf16_lo(v[u].x)), fabsf(bf16_hi(v[u].x))),
-                                         fmaxf(fabsf(bf16_lo(v[u].y)), fabsf(bf16_hi(v[u].y)))),
-                                   fmaxf(fmaxf(fabsf(bf16_lo(v[u].z)), fabsf(bf16_hi(v[u].z))),
-                                         fmaxf(fabsf(bf16_lo(v[u].w)), fabsf(bf16_hi(v[u].w))))));
+    if (c < kb) {
+        const uint4 v = x[static_cast<int64_t>(t) * kb + c];
+        m = fmaxf(fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))),
+                  fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-    if (blockIdx.x == 0 && t == 0)
-        for (int i = threadIdx.x; i < num_w; i += kPrepThreads) tile_count[i] = 0;
     __syncthreads();
-    if (threadIdx.x == 0)
-        pmax[static_cast<int64_t>(t) * S + blockIdx.x] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    if (threadIdx.x == 0) {
+        for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
+        pmax[static_cast<int64_t>(t) * gridDim.x + blockIdx.x] = fmaxf(m, red[0]);
+    }
 }
 
 // For row t: e_t puts max_k |x[t][k]| in [2^14, 2^15) (0 for a zero or non-finite row);
 // xp[t][k] = f16(x * 2^e_t) in the order the dequantizer of kBits-bit codes emits its pairs in
 // (0,4,1,5,2,6,3,7 of each 8-block for 4-bit codes, 0,2,1,3,4,6,5,7 for 8-bit codes); rowexp[t] = -e_t.
 template <int kBits>
-__global__ void __launch_bounds__(kPrepThreads, 16) skinny_prepass_kernel(const uint4* __restrict__ x,
-                                                                         const float* __restrict__ pmax,
-                                                                         uint4* __restrict__ xp,
-                                                                         int* __restrict__ rowexp, int K) {
+__global__ void __launch_bounds__(256) skinny_prepass_kernel(const uint4* __restrict__ x, const float* __restrict__ pmax,
+                                                             uint4* __restrict__ xp, int* __restrict__ rowexp, int K) {
     ptx::launch_dependents();
     ptx::grid_dependency_wait();                               // pmax comes from the kernel before
-    const int t = blockIdx.y, kb = K / 8, S = gridDim.x;
+    const int t = blockIdx.y, kb = K / 8;
+    const int c = blockIdx.x * 256 + threadIdx.x;
     float m = 0.0f;
-    for (int i = 0; i < S; ++i) m = fmaxf(m, pmax[static_cast<int64_t>(t) * S + i]);
+    for (int i = 0; i < static_cast<int>(gridDim.x); ++i) m = fmaxf(m, pmax[static_cast<int64_t>(t) * gridDim.x + i]);
     int ex = 0;
     if (m > 0.0f && m <= 3.4028235e38f) {
         int E;
@@ -192,97 +163,24 @@ __global__ void __launch_bounds__(kPrepThreads, 16) skinny_prepass_kernel(const 
         ex = 15 - E;
     }
     if (blockIdx.x == 0 && threadIdx.x == 0) rowexp[t] = -ex;
-    const int c0 = static_cast<int>((static_cast<int64_t>(blockIdx.x) * kb) / S);
-    const int c1 = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * kb) / S);
-    const uint4* row = x + static_cast<int64_t>(t) * kb;
-    uint4* out = xp + static_cast<int64_t>(t) * kb;
-    for (int c = c0 + threadIdx.x; c < c1; c += kPrepUnroll * kPrepThreads) {
-        uint4 v[kPrepUnroll];
+    if (c < kb) {
+        const uint4 v = x[static_cast<int64_t>(t) * kb + c];
+        const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                            bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+        uint32_t o[4];
 #pragma unroll
-        for (int u = 0; u < kPrepUnroll; ++u)
-            if (c + u * kPrepThreads < c1) v[u] = row[c + u * kPrepThreads];
-#pragma unroll
-        for (int u = 0; u < kPrepUnroll; ++u) {
-            if (c + u * kPrepThreads >= c1) continue;
-            const float f[8] = {bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y),
-                                bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w)};
-            uint32_t o[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                // 4-bit: slot pairs (k0, k4) (k1, k5) (k2, k6) (k3, k7); 8-bit: (k0, k2) (k1, k3) (k4, k6) (k5, k7)
-                const int lo = kBits == 4 ? j : 2 * (j & 2) + (j & 1);
-                const int hi = kBits == 4 ? j + 4 : lo + 2;
-                const __half2 h = __halves2half2(__float2half_rn(ldexpf(f[lo], ex)), __float2half_rn(ldexpf(f[hi], ex)));
-                o[j] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            out[c + u * kPrepThreads] = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int j = 0; j < 4; ++j) {
+            // 4-bit: slot pairs (k0, k4) (k1, k5) (k2, k6) (k3, k7); 8-bit: (k0, k2) (k1, k3) (k4, k6) (k5, k7)
+            const int lo = kBits == 4 ? j : 2 * (j & 2) + (j & 1);
+            const int hi = kBits == 4 ? j + 4 : lo + 2;
+            const __half2 h = __halves2half2(__float2half_rn(ldexpf(f[lo], ex)), __float2half_rn(ldexpf(f[hi], ex)));
+            o[j] = *reinterpret_cast<const uint32_t*>(&h);
         }
+        xp[static_cast<int64_t>(t) * kb + c] = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
 
-// Code producer: chunk ci (chunk cq of tile w) into its stage of the code ring: the chunk's code boxes and
-// the parameter box holding it, all completing on the stage's full barrier.
-template <class L>
-__device__ __forceinline__ void load_chunk(uint8_t* smem, uint64_t* c_full, uint32_t ci, int w, int cq, bool param_tma,
-                                           const CUtensorMap* map_codes, const CUtensorMap* map_scales,
-                                           const CUtensorMap* map_biases) {
-    const int g0 = cq * L::CG;
-    const int s = static_cast<int>(ci % L::NC);
-    uint8_t* st = smem + L::kOffC + s * L::kStageBytes;
-    ptx::mbar_arrive_expect_tx(&c_full[s], L::kCBytes + (param_tma ? 2 * kParHalf : 0u));
-#pragma unroll
-    for (int bx = 0; bx < L::CG / L::kBoxGroups; ++bx)   // consecutive boxes: long contiguous row segments
-        ptx::tma_load_2d(st + bx * kBoxBytes, map_codes, &c_full[s], (g0 + bx * L::kBoxGroups) * L::kGroupWords, w * BW);
-    if (param_tma) {
-        // the 8-group box holding the chunk (a chunk of 4 groups uses half of it)
-        const int gp = g0 - g0 % kParGroups;
-        ptx::tma_load_2d(st + L::kCBytes, map_scales, &c_full[s], gp, w * BW);
-        ptx::tma_load_2d(st + L::kCBytes + kParHalf, map_biases, &c_full[s], gp, w * BW);
-    }
-}
-
-// The ordered reduction of one finished tile w by the CTA that completed it: thread r (weight row r of the
-// tile) sums, for every token, the covering CTAs' partials in CTA order (offsets in cover[0..k_end)),
-// scales back by 2^-e_t and writes y.  Tokens go in batches with every load of a batch in flight.  Kept
-// out of line so that its registers do not weigh on the streaming roles of the kernel.
-template <bool kBf16Out>
-__device__ __forceinline__ void reduce_tile(const Params& p, const int64_t* cover, int k_end, int w, int r) {
-    __threadfence();                              // the other CTAs' partials after their counts
-    const int n = w * BW + r;
-    constexpr int kRedBatch = 4;
-    for (int t0 = 0; t0 < p.M && n < p.N; t0 += kRedBatch) {
-        float acc[kRedBatch];
-        int ex[kRedBatch];
-#pragma unroll
-        for (int b = 0; b < kRedBatch; ++b) {
-            acc[b] = 0.0f;
-            ex[b] = t0 + b < p.M ? p.rowexp[t0 + b] : 0;
-        }
-        for (int k = 0; k < k_end; ++k) {          // covering CTAs in CTA order
-            float v[kRedBatch];
-#pragma unroll
-            for (int b = 0; b < kRedBatch; ++b) {
-                const int64_t at = cover[k] + static_cast<int64_t>(t0 + b) * BW + r;
-                v[b] = (t0 + b < p.M && in_bounds(at, p.partial_elems)) ? __ldcg(p.partial + at) : 0.0f;
-            }
-#pragma unroll
-            for (int b = 0; b < kRedBatch; ++b) acc[b] += v[b];
-        }
-#pragma unroll
-        for (int b = 0; b < kRedBatch; ++b) {
-            if (t0 + b >= p.M) break;
-            const float val = ldexpf(acc[b], ex[b]);
-            const int64_t e = static_cast<int64_t>(t0 + b) * p.N + n;
-            if constexpr (kBf16Out) {
-                reinterpret_cast<__nv_bfloat16*>(p.y)[e] = __float2bfloat16_rn(val);
-            } else {
-                reinterpret_cast<float*>(p.y)[e] = val;
-            }
-        }
-    }
-}
-
-template <int NT, int B, bool kBf16Out>
+template <int NT, int B>
 __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_constant__ CUtensorMap map_codes,
                                                             const __grid_constant__ CUtensorMap map_x,
                                                             const __grid_constant__ CUtensorMap map_scales,
@@ -307,8 +205,6 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     uint64_t* acc_full = a_empty + NA;          // two: one per accumulator set
     uint64_t* acc_empty = acc_full + 2;         // two
     uint64_t* drain = acc_empty + 2;            // one per MMA issuer
-    uint64_t* pub = drain + kMmaCopies;         // the four drain warps have published a partial
-    uint64_t* verdict = pub + 1;                // the tile's arrival count has been taken
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
 
@@ -319,36 +215,23 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
     const int64_t u1 = run_first(p.units, P, blockIdx.x + 1);
     const uint32_t nchunks = static_cast<uint32_t>(u1 - u0);
 
-    // Thread 0 is the code producer's lane: it initializes the barriers and puts the first stages' loads
-    // in flight (fresh stages need no empty wait) before the block-wide sync and the TMEM allocation.
-    // (the checked build's stall hook holds the code producer back: no code or parameter load at all)
-    const bool held = stalled(kStallSkinny);
-    const uint32_t early = held ? 0u : min(static_cast<uint32_t>(NC), nchunks);
     if (threadIdx.x == 0) {
         for (int i = 0; i < NC; ++i) { ptx::mbar_init(&c_full[i], 1); ptx::mbar_init(&c_empty[i], 4 * kBuildCopies); }
         for (int i = 0; i < NXC; ++i) { ptx::mbar_init(&x_full[i], 1); ptx::mbar_init(&x_empty[i], kMmaCopies); }
         for (int i = 0; i < NA; ++i) { ptx::mbar_init(&a_full[i], 4); ptx::mbar_init(&a_empty[i], 1); }
         for (int i = 0; i < 2; ++i) { ptx::mbar_init(&acc_full[i], kMmaCopies); ptx::mbar_init(&acc_empty[i], 4); }
         for (int i = 0; i < kMmaCopies; ++i) ptx::mbar_init(&drain[i], 1);
-        ptx::mbar_init(pub, 4);
-        ptx::mbar_init(verdict, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
+    }
+    if (warp == kWarpTmaX && lane == 0) ptx::prefetch_tensormap(&map_x);
+    if (warp == kWarpTmaC && lane == 0) {
         ptx::prefetch_tensormap(&map_codes);
         if (p.param_tma) {
             ptx::prefetch_tensormap(&map_scales);
             ptx::prefetch_tensormap(&map_biases);
         }
-        int w = static_cast<int>(u0 / p.cpt), cq = static_cast<int>(u0 % p.cpt);
-        for (uint32_t ci = 0; ci < early; ++ci) {
-            load_chunk<L>(smem, c_full, ci, w, cq, p.param_tma != 0, &map_codes, &map_scales, &map_biases);
-            if (++cq == p.cpt) {
-                cq = 0;
-                ++w;
-            }
-        }
     }
-    if (warp == kWarpTmaX && lane == 0) ptx::prefetch_tensormap(&map_x);
     if (warp == kWarpMma0) {
         ptx::tmem_alloc(tmem_slot, kTmemCols);
         ptx::tmem_relinquish();
@@ -386,15 +269,28 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
 
     if (warp == kWarpTmaC) {
         // ---------------------------------------------------------------- code + parameter producer
-        // (codes and parameters do not depend on the prepass: no dependency wait)
-        if (lane == 0 && !held) {
-            uint32_t ci = early;
+        // (codes and parameters do not depend on the prepass: no dependency wait; the checked build's
+        // stall hook holds this producer back: no code or parameter load at all)
+        if (lane == 0 && !stalled(kStallSkinny)) {
+            uint32_t ci = 0;
             ChunkPos cp = start;
-            for (uint32_t k = 0; k < early; ++k) advance(cp);
             for (; ci < nchunks; ++ci, advance(cp)) {
+                int w, g0, ng;
+                chunk_groups(cp, w, g0, ng);
                 const int s = static_cast<int>(ci % NC);
                 if (!ptx::mbar_wait(&c_empty[s], ((ci / NC) & 1u) ^ 1u, abort_flag)) break;
-                load_chunk<L>(smem, c_full, ci, cp.w, cp.cq, p.param_tma != 0, &map_codes, &map_scales, &map_biases);
+                uint8_t* st = smem + L::kOffC + s * kStageBytes;
+                ptx::mbar_arrive_expect_tx(&c_full[s], kCBytes + (p.param_tma ? 2 * kParHalf : 0u));
+#pragma unroll
+                for (int bx = 0; bx < CG / kBoxGroups; ++bx)   // consecutive boxes: long contiguous row segments
+                    ptx::tma_load_2d(st + bx * kBoxBytes, &map_codes, &c_full[s], (g0 + bx * kBoxGroups) * L::kGroupWords,
+                                     w * BW);
+                if (p.param_tma) {
+                    // the 8-group box holding the chunk (a chunk of 4 groups uses half of it)
+                    const int gp = g0 - g0 % kParGroups;
+                    ptx::tma_load_2d(st + kCBytes, &map_scales, &c_full[s], gp, w * BW);
+                    ptx::tma_load_2d(st + kCBytes + kParHalf, &map_biases, &c_full[s], gp, w * BW);
+                }
             }
             // never leave the CTA with bulk copies still landing in its shared memory
             for (uint32_t j = (ci > static_cast<uint32_t>(NC) ? ci - NC : 0u); j < ci; ++j)
@@ -581,10 +477,6 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
         const int r = quarter * 32 + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         const int w_first = start.w;
-        volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);   // this CTA reduces the tile
-        volatile int* n_cover = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 12);
-        int64_t* cover = reinterpret_cast<int64_t*>(smem + L::kOffCover);   // covering partials' offsets
-        ptx::grid_dependency_wait();     // row exponents and zeroed arrival counts come from the prepass
         uint32_t pb = 0, seg = 0, seg_pb = 0;    // pairs so far; segments drained; first pair of the segment
         ChunkPos cp = start;
         for (uint32_t i = 0; i < nchunks; ++i, advance(cp)) {
@@ -619,37 +511,6 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
             if (lane == 0) ptx::mbar_arrive(&acc_empty[set]);
             ++seg;
             seg_pb = pb;
-
-            // Publish the partial of tile cp.w.  Each drain warp fences its stores and arrives on `pub`;
-            // thread r = 0 lists the tile's covering CTAs, takes the tile's arrival count and posts the
-            // verdict; the CTA whose partial completes the tile's set sums the partials in CTA order.
-            // Every wait is bounded, so an expired wait unwinds all four warps alike.
-            const int w = cp.w;
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(pub);
-            if (r == 0) {
-                bool ok = ptx::mbar_wait(pub, (seg - 1) & 1u, abort_flag);
-                if (ok) {
-                    const int64_t lo = static_cast<int64_t>(w) * p.cpt, hi = lo + p.cpt;   // the tile's chunks
-                    int c = static_cast<int>((lo * P) / p.units);
-                    while (c > 0 && run_first(p.units, P, c) > lo) --c;
-                    while (c + 1 <= P && run_first(p.units, P, c + 1) <= lo) ++c;
-                    int k = 0;
-                    for (int64_t f0 = run_first(p.units, P, c); c < P && f0 < hi; ++c) {
-                        const int64_t f1 = run_first(p.units, P, c + 1);
-                        if (f1 > f0 && k < kMaxCtas)        // non-empty run: its segment of tile w
-                            cover[k++] = (static_cast<int64_t>(c) * p.segmax + (w - static_cast<int>(f0 / p.cpt))) * p.M * BW;
-                        f0 = f1;
-                    }
-                    *n_cover = k;
-                    *last_flag = in_bounds(w, p.num_w) ? atomicAdd(p.tile_count + w, 1) == k - 1 : 0;
-                    ptx::mbar_arrive(verdict);
-                }
-            }
-            const bool ok = ptx::mbar_wait(verdict, (seg - 1) & 1u, abort_flag);
-            if (!__all_sync(0xFFFFFFFFu, ok)) break;
-            if (*last_flag) reduce_tile<kBf16Out>(p, cover, *n_cover, w, r);
         }
     }
 
@@ -659,6 +520,55 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
         __syncwarp();
         ptx::tc_fence_after_sync();
         ptx::tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// y[t][n] = 2^rowexp[t] * (sum over the CTAs whose runs cover tile n/128, in CTA order, of their
+// partials for that tile).  One CTA per (tile, 2 tokens): thread 0 lists the covering CTAs' segment
+// bases once, the other threads only load and add.
+template <bool kBf16Out>
+__global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restrict__ partial,
+                                                            const int* __restrict__ rowexp, void* __restrict__ y,
+                                                            int M, int N, int cpt, int64_t units, int P, int segmax,
+                                                            int64_t partial_elems) {
+    __shared__ int64_t seg_base[kMaxCtas];
+    __shared__ int count;
+    const int w = blockIdx.x;
+    if (threadIdx.x == 0) {
+        // CTAs whose run of chunks [first(c), first(c+1)) meets [w*cpt, (w+1)*cpt), in CTA order
+        const int64_t lo = static_cast<int64_t>(w) * cpt, hi = lo + cpt;
+        int c = static_cast<int>((lo * P) / units);
+        while (c > 0 && run_first(units, P, c) > lo) --c;
+        while (c + 1 <= P && run_first(units, P, c + 1) <= lo) ++c;
+        int k = 0;
+        int64_t f0 = run_first(units, P, c);
+        for (; c < P && f0 < hi; ++c) {
+            const int64_t f1 = run_first(units, P, c + 1);
+            if (f1 > f0) {                                        // non-empty run
+                const int w_first = static_cast<int>(f0 / cpt);
+                seg_base[k++] = static_cast<int64_t>(c) * segmax + (w - w_first);
+            }
+            f0 = f1;
+        }
+        count = k;
+    }
+    ptx::grid_dependency_wait();                                  // partials come from the kernel before
+    __syncthreads();
+    const int t = blockIdx.y * 2 + (threadIdx.x >> 7), r = threadIdx.x & 127;
+    const int n = w * BW + r;
+    if (t >= M || n >= N) return;
+    float acc = 0.0f;
+    const int k_end = count;
+    for (int k = 0; k < k_end; ++k) {
+        const int64_t at = (seg_base[k] * M + t) * BW + r;
+        if (in_bounds(at, partial_elems)) acc += partial[at];
+    }
+    acc = ldexpf(acc, rowexp[t]);
+    const int64_t e = static_cast<int64_t>(t) * N + n;
+    if constexpr (kBf16Out) {
+        reinterpret_cast<__nv_bfloat16*>(y)[e] = __float2bfloat16_rn(acc);
+    } else {
+        reinterpret_cast<float*>(y)[e] = acc;
     }
 }
 
