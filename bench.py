@@ -101,9 +101,12 @@ def peaks():
 
 
 def kernel_source_hash() -> str:
+    """First 12 hex digits of the sha256 over every CUDA source of the library, in name order: a recorded
+    ncu traffic figure is used only while the kernels it was taken on are unchanged."""
     import hashlib
     d = os.path.join(ROOT, "group_wise_affine_qlinear_b200", "csrc")
-    src = b"".join(open(os.path.join(d, f), "rb").read() for f in ("ql_tc_fused.cuh", "ql_ptx.cuh", "ql_dequant_f16.cuh"))
+    names = sorted(f for f in os.listdir(d) if f.endswith((".cu", ".cuh", ".h")))
+    src = b"".join(f.encode() + b"\0" + open(os.path.join(d, f), "rb").read() for f in names)
     return hashlib.sha256(src).hexdigest()[:12]
 
 
@@ -203,7 +206,8 @@ def swiglu_measure(ql, torch, dev, flush, peak_tf, steps=10):
     call, main = sum(call_ms) / steps, sum(main_ms) / steps
     return {"workload": f"{w.name} M={w.M} K={w.K} I={w.N} (gate + up)", "dispatch": dispatch,
             "step_ms": call, "kernel_ms": main, "TFLOPs": flops / (call * 1e-3) / 1e12,
-            "kernel_TFLOPs": flops / (main * 1e-3) / 1e12, "kernel_frac": flops / (main * 1e-3) / 1e12 / peak_tf}
+            "kernel_TFLOPs": flops / (main * 1e-3) / 1e12, "kernel_frac": flops / (main * 1e-3) / 1e12 / peak_tf,
+            "traffic": recorded_traffic(dispatch.split()[0], f"{w.name}:M={w.M}")}
 
 
 def comparators(ql, torch, dev, flush, steps=10):
@@ -268,7 +272,8 @@ def split_measure(ql, torch, dev, flush, peak_tf, steps=10):
         assert ql.device_status() == 0, "the fused path reported an error"
         out[f"split{split}"] = {"dispatch": c.dispatch, "step_us": st * 1e3, "kernel_us": mn * 1e3,
                                 "TFLOPs": flops / (st * 1e-3) / 1e12,
-                                "kernel_frac": flops / (mn * 1e-3) / 1e12 / peak_tf}
+                                "kernel_frac": flops / (mn * 1e-3) / 1e12 / peak_tf,
+                                "traffic": recorded_traffic(c.dispatch.split()[0], f"{w.name}:M={M}:split={split}")}
         del c
     torch.cuda.synchronize()
     return out
@@ -698,7 +703,8 @@ def main():
             out.append({"M": Ms, "dispatch": c.dispatch, "step_us": st * 1e3, "kernel_us": mn * 1e3,
                         "weight_GBps": tp.weight_bytes / (st * 1e-3) / 1e9,
                         "algorithmic_GBps": c.algorithmic_bytes() / (st * 1e-3) / 1e9,
-                        "step_us_dirty_l2": st_d * 1e3})
+                        "step_us_dirty_l2": st_d * 1e3,
+                        "traffic": recorded_traffic(c.dispatch.split()[0], f"{name}:M={Ms}")})
             del c
         torch.cuda.synchronize()
         return out
