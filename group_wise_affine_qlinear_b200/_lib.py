@@ -102,6 +102,8 @@ def load_library(path: str) -> ctypes.CDLL:
     L.qlinear_swiglu_forward.restype = ctypes.c_int
     L.qlinear_test_stall.argtypes = [i32, ctypes.c_uint64]
     L.qlinear_test_stall.restype = ctypes.c_int
+    L.qlinear_test_ring_depth.argtypes = [i32]
+    L.qlinear_test_ring_depth.restype = ctypes.c_int
     return L
 
 

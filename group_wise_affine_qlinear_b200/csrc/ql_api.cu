@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -74,13 +75,15 @@ cudaError_t skinny_smem_attr() {
                                 skinny::Layout<NT, B>::kSmemBytes);
 }
 
-template <class FC, bool kSwiGLU = false>
+template <int B, bool kSwiGLU = false>
 cudaError_t fused_smem_attr() {
-    const cudaError_t e = cudaFuncSetAttribute(fused::fused_gemm_kernel<true, FC, kSwiGLU>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, FC::kSmemBytes);
+    using FB = typename fused::PickCfg<B, true>::type;
+    using FF = typename fused::PickCfg<B, false>::type;
+    const cudaError_t e = cudaFuncSetAttribute(fused::fused_gemm_kernel<true, FB, kSwiGLU>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, FB::kSmemBytes);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(fused::fused_gemm_kernel<false, FC, kSwiGLU>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, FC::kSmemBytes);
+    return cudaFuncSetAttribute(fused::fused_gemm_kernel<false, FF, kSwiGLU>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, FF::kSmemBytes);
 }
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -96,13 +99,14 @@ ql_status device_info(DeviceInfo** out) {
         d.sm_count = n;
     }
     if (!d.fused_attr_set) {
-        if (fused_smem_attr<fused::DefaultCfg>() != cudaSuccess || fused_smem_attr<fused::Q8Cfg>() != cudaSuccess ||
-            fused_smem_attr<fused::DefaultCfg, true>() != cudaSuccess ||
-            cudaFuncSetAttribute(fused::fused_gemm_kernel<false, fused::DefaultCfg, false, true>,
+        if (fused_smem_attr<4>() != cudaSuccess || fused_smem_attr<8>() != cudaSuccess ||
+            fused_smem_attr<4, true>() != cudaSuccess ||
+            cudaFuncSetAttribute(fused::fused_gemm_kernel<false, fused::PickCfg<4, false>::type, false, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 fused::DefaultCfg::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(fused::fused_gemm_kernel<false, fused::Q8Cfg, false, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, fused::Q8Cfg::kSmemBytes) != cudaSuccess)
+                                 fused::PickCfg<4, false>::type::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(fused::fused_gemm_kernel<false, fused::PickCfg<8, false>::type, false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 fused::PickCfg<8, false>::type::kSmemBytes) != cudaSuccess)
             return QL_ERR_CUDA;
         d.fused_attr_set = true;
     }
@@ -201,8 +205,7 @@ struct Plan {
     // fused path workspace carve-up (off_part: fp32 partials [split_k][M][N] when the K-steps are split)
     size_t off_xh = 0, off_rs = 0, off_sb = 0, off_part = 0;
     // skinny path workspace carve-up: partials, scaled f16 activations, row exponents, per-slice row maxima
-    size_t off_xp = 0, off_re = 0, off_pm = 0;
-    int slices = 0;
+    size_t off_xp = 0, off_re = 0;
 };
 
 // Split factor of the fused tensor-core path when the caller leaves it to the dispatcher.  Every K-step
@@ -265,9 +268,7 @@ ql_status make_plan(int64_t M, int64_t K, int64_t N, int path, int split_k, int 
         plan->split_k = 1;
         plan->off_xp = round_up(static_cast<size_t>(plan->ctas) * plan->segmax * M * skinny::BW * sizeof(float), 256);
         plan->off_re = plan->off_xp + round_up(static_cast<size_t>(M) * K * 2, 256);
-        plan->slices = static_cast<int>((K / 8 + 255) / 256);
-        plan->off_pm = plan->off_re + round_up(static_cast<size_t>(plan->nt) * sizeof(int), 256);
-        plan->workspace = plan->off_pm + round_up(static_cast<size_t>(M) * plan->slices * sizeof(float), 256);
+        plan->workspace = plan->off_re + round_up(static_cast<size_t>(plan->nt) * sizeof(int), 256);
         return QL_OK;
     }
     if (path == QL_PATH_TC_FUSED) {
@@ -346,6 +347,46 @@ ql_status launch_dependent(void (*kernel)(KArgs...), dim3 grid, int block, size_
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
+#ifdef QL_BOUNDS_CHECK
+// Ring-depth variants of the 4-bit bf16 fused kernel (the checked build's qlinear_test_ring_depth):
+// (activation stages, code stages, 4-bit codes, bf16 staging, staging blocks per warp).
+using RingV1 = fused::Cfg<2, 1, 4, 2, 1>;
+using RingV2 = fused::Cfg<3, 1, 4, 2, 2>;
+using RingV3 = fused::Cfg<2, 2, 4, 2, 2>;
+using RingV4 = fused::Cfg<4, 2, 4, 2, 1>;
+using RingV5 = fused::Cfg<6, 1, 4, 2, 2>;
+using RingV6 = fused::Cfg<3, 3, 4, 2, 2>;
+static_assert(QL_TEST_RING_VARIANTS == 7, "one configuration per variant");
+std::atomic<int> g_ring_variant{0};
+
+template <class FC>
+ql_status launch_ring(dim3 grid, cudaStream_t st, const CUtensorMap& mx, const CUtensorMap& mc, const CUtensorMap& mp,
+                      const CUtensorMap& my, const fused::Params& p) {
+    static_assert(FC::kS == fused::PickCfg<4, true>::type::kS, "the parameter boxes are sized for kS K-steps");
+    return launch_dependent(fused::fused_gemm_kernel<true, FC>, grid, fused::kThreads, FC::kSmemBytes, st, mx, mc, mc,
+                            mp, my, p);
+}
+
+ql_status launch_ring_variant(int v, dim3 grid, cudaStream_t st, const CUtensorMap& mx, const CUtensorMap& mc,
+                              const CUtensorMap& mp, const CUtensorMap& my, const fused::Params& p) {
+    switch (v) {
+        case 1: return launch_ring<RingV1>(grid, st, mx, mc, mp, my, p);
+        case 2: return launch_ring<RingV2>(grid, st, mx, mc, mp, my, p);
+        case 3: return launch_ring<RingV3>(grid, st, mx, mc, mp, my, p);
+        case 4: return launch_ring<RingV4>(grid, st, mx, mc, mp, my, p);
+        case 5: return launch_ring<RingV5>(grid, st, mx, mc, mp, my, p);
+        case 6: return launch_ring<RingV6>(grid, st, mx, mc, mp, my, p);
+        default: return QL_ERR_INVALID_ARG;
+    }
+}
+
+template <class FC>
+cudaError_t ring_smem_attr() {
+    return cudaFuncSetAttribute(fused::fused_gemm_kernel<true, FC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                FC::kSmemBytes);
+}
+#endif
+
 ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const void* scales, const void* biases,
                     void* y, bool bf16_out, int64_t M, int64_t K, int64_t N, void* ws, cudaStream_t st,
                     int sm_count) {
@@ -360,14 +401,14 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xh, K, M, K * 2, fused::BK, fused::BT,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
-    // one K-step of codes per box: 32 bytes of each of 256 rows (4-bit codes, unswizzled) or 64 bytes
-    // (8-bit codes, 64-byte swizzle, which the dequantizers undo)
+    // one code stage per box: 128 bytes of each of 256 rows (4 K-steps of 4-bit codes, 2 of 8-bit codes),
+    // 128-byte swizzle, which the dequantizers undo; the (scale, bias) pairs of the same K-steps
     const int bits = pl.bits;
+    const int cfg_steps = bits == 4 ? fused::PickCfg<4, true>::type::kS : fused::PickCfg<8, true>::type::kS;
     if ((s = encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K * bits / 32, N, K * bits / 8,
-                       fused::BK * bits / 32, fused::BW,
-                       bits == 4 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_64B)) != QL_OK)
+                       fused::kCodeRowBytes / 4, fused::BW, CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
-    if ((s = encode_2d(&mp, CU_TENSOR_MAP_DATA_TYPE_UINT32, sb, N, G, N * 4, fused::BW, 1,
+    if ((s = encode_2d(&mp, CU_TENSOR_MAP_DATA_TYPE_UINT32, sb, N, G, N * 4, fused::BW, cfg_steps,
                        CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
         return s;
     CUtensorMap my;
@@ -409,11 +450,13 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     const int grid = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(tiles) * pl.split_k, sm_count));
     prof_begin(st);
     const dim3 fgrid(static_cast<unsigned>(grid));
+    using F4 = fused::PickCfg<4, false>::type;
+    using F8 = fused::PickCfg<8, false>::type;
     if (split) {
-        s = bits == 4 ? launch_dependent(fused::fused_gemm_kernel<false, fused::DefaultCfg, false, true>, fgrid,
-                                         fused::kThreads, fused::DefaultCfg::kSmemBytes, st, mx, mc, mc, mp, my, p)
-                      : launch_dependent(fused::fused_gemm_kernel<false, fused::Q8Cfg, false, true>, fgrid,
-                                         fused::kThreads, fused::Q8Cfg::kSmemBytes, st, mx, mc, mc, mp, my, p);
+        s = bits == 4 ? launch_dependent(fused::fused_gemm_kernel<false, F4, false, true>, fgrid, fused::kThreads,
+                                         F4::kSmemBytes, st, mx, mc, mc, mp, my, p)
+                      : launch_dependent(fused::fused_gemm_kernel<false, F8, false, true>, fgrid, fused::kThreads,
+                                         F8::kSmemBytes, st, mx, mc, mc, mp, my, p);
         if (s != QL_OK) return s;
         prof_end(st);
         // ordered sum of the slices, rounded once (a plain launch: it reads what the kernel above wrote)
@@ -423,31 +466,39 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
             ordered_sum_kernel<true><<<blocks, 256, 0, st>>>(part, y, count, pl.split_k);
         else
             ordered_sum_kernel<false><<<blocks, 256, 0, st>>>(part, y, count, pl.split_k);
-        const int nc = bits == 4 ? fused::DefaultCfg::kNC : fused::Q8Cfg::kNC;
-        const int nx = bits == 4 ? fused::DefaultCfg::kNX : fused::Q8Cfg::kNX;
-        set_dispatch("path=tc_fused bits=%d tile=%dw x %dt x %dk stages=x%d/c%d/a%d ctas=%d splitk=%d launches=4 why=%s",
-                     bits, fused::BW, fused::BT, fused::BK, nx, nc, fused::NA, grid, pl.split_k, pl.why);
+        const int nc = bits == 4 ? F4::kNC : F8::kNC;
+        const int nx = bits == 4 ? F4::kNX : F8::kNX;
+        set_dispatch("path=tc_fused bits=%d tile=%dw x %dt x %dk stages=x%d/c%dx%d/a%d ctas=%d splitk=%d launches=4 why=%s",
+                     bits, fused::BW, fused::BT, fused::BK, nx, nc, cfg_steps, fused::NA, grid, pl.split_k, pl.why);
         return launch_status();
     }
+    using B4 = fused::PickCfg<4, true>::type;
+    using B8 = fused::PickCfg<8, true>::type;
+#ifdef QL_BOUNDS_CHECK
+    if (const int v = g_ring_variant.load(); v != 0 && bits == 4 && bf16_out) {
+        if ((s = launch_ring_variant(v, fgrid, st, mx, mc, mp, my, p)) != QL_OK) return s;
+        prof_end(st);
+        set_dispatch("path=tc_fused bits=4 ring_variant=%d ctas=%d splitk=1 launches=3 why=%s", v, grid, pl.why);
+        return launch_status();
+    }
+#endif
     if (bits == 4) {
-        using FC = fused::DefaultCfg;
-        s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
+        s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, B4>, fgrid, fused::kThreads, B4::kSmemBytes, st,
                                         mx, mc, mc, mp, my, p)
-                     : launch_dependent(fused::fused_gemm_kernel<false, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
+                     : launch_dependent(fused::fused_gemm_kernel<false, F4>, fgrid, fused::kThreads, F4::kSmemBytes, st,
                                         mx, mc, mc, mp, my, p);
     } else {
-        using FC = fused::Q8Cfg;
-        s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
+        s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, B8>, fgrid, fused::kThreads, B8::kSmemBytes, st,
                                         mx, mc, mc, mp, my, p)
-                     : launch_dependent(fused::fused_gemm_kernel<false, FC>, fgrid, fused::kThreads, FC::kSmemBytes, st,
+                     : launch_dependent(fused::fused_gemm_kernel<false, F8>, fgrid, fused::kThreads, F8::kSmemBytes, st,
                                         mx, mc, mc, mp, my, p);
     }
     if (s != QL_OK) return s;
     prof_end(st);
-    const int nc = bits == 4 ? fused::DefaultCfg::kNC : fused::Q8Cfg::kNC;
-    const int nx = bits == 4 ? fused::DefaultCfg::kNX : fused::Q8Cfg::kNX;
-    set_dispatch("path=tc_fused bits=%d tile=%dw x %dt x %dk stages=x%d/c%d/a%d ctas=%d splitk=1 launches=3 why=%s",
-                 bits, fused::BW, fused::BT, fused::BK, nx, nc, fused::NA, grid, pl.why);
+    const int nc = bits == 4 ? (bf16_out ? B4::kNC : F4::kNC) : (bf16_out ? B8::kNC : F8::kNC);
+    const int nx = bits == 4 ? (bf16_out ? B4::kNX : F4::kNX) : (bf16_out ? B8::kNX : F8::kNX);
+    set_dispatch("path=tc_fused bits=%d tile=%dw x %dt x %dk stages=x%d/c%dx%d/a%d ctas=%d splitk=1 launches=3 why=%s",
+                 bits, fused::BW, fused::BT, fused::BK, nx, nc, cfg_steps, fused::NA, grid, pl.why);
     (void)codes;
     return launch_status();
 }
@@ -459,7 +510,6 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     void* xp = wsb + pl.off_xp;
     int* rowexp = reinterpret_cast<int*>(wsb + pl.off_re);
-    float* pmax = reinterpret_cast<float*>(wsb + pl.off_pm);
     CUtensorMap mc, mx;
     ql_status s;
     const int bits = pl.bits;
@@ -496,28 +546,15 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
     p.units = pl.units;
     p.segmax = pl.segmax;
     p.partial_elems = static_cast<int64_t>(pl.ctas) * pl.segmax * M * skinny::BW;
-    // row maxima, then scaled and reordered f16 activations, per-group activation sums, row exponents
-    const dim3 pre_grid(static_cast<unsigned>(pl.slices), static_cast<unsigned>(M));
-    skinny::skinny_rowmax_kernel<<<pre_grid, 256, 0, st>>>(static_cast<const uint4*>(x), pmax, static_cast<int>(K));
+    // row exponents and scaled, reordered f16 activations (one cluster of CTAs per row)
+    const dim3 pre_grid(static_cast<unsigned>(skinny::kPrepCluster), static_cast<unsigned>(M));
+    if (bits == 4)
+        skinny::skinny_prepass_kernel<4><<<pre_grid, skinny::kPrepThreads, 0, st>>>(
+            static_cast<const uint4*>(x), static_cast<uint4*>(xp), rowexp, static_cast<int>(K));
+    else
+        skinny::skinny_prepass_kernel<8><<<pre_grid, skinny::kPrepThreads, 0, st>>>(
+            static_cast<const uint4*>(x), static_cast<uint4*>(xp), rowexp, static_cast<int>(K));
     if ((s = launch_status()) != QL_OK) return s;
-    {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = pre_grid;
-        cfg.blockDim = dim3(256);
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const float* pm = pmax;
-        const cudaError_t e =
-            bits == 4 ? cudaLaunchKernelEx(&cfg, skinny::skinny_prepass_kernel<4>, static_cast<const uint4*>(x), pm,
-                                           static_cast<uint4*>(xp), rowexp, static_cast<int>(K))
-                      : cudaLaunchKernelEx(&cfg, skinny::skinny_prepass_kernel<8>, static_cast<const uint4*>(x), pm,
-                                           static_cast<uint4*>(xp), rowexp, static_cast<int>(K));
-        if (e != cudaSuccess) return QL_ERR_CUDA;
-    }
     prof_begin(st);
     const dim3 sgrid(static_cast<unsigned>(pl.ctas));
     if (bits == 4 && pl.nt == 16)
@@ -551,7 +588,7 @@ ql_status run_skinny(const Plan& pl, const void* x, const uint32_t* codes, const
                              p.units, pl.ctas, pl.segmax, p.partial_elems);
     if (s != QL_OK) return s;
     (void)sm_count;
-    set_dispatch("path=tc_skinny bits=%d nt=%d ctas=%d segmax=%d units=%lld launches=4 why=%s", bits, pl.nt, pl.ctas,
+    set_dispatch("path=tc_skinny bits=%d nt=%d ctas=%d segmax=%d units=%lld launches=3 why=%s", bits, pl.nt, pl.ctas,
                  pl.segmax, static_cast<long long>(pl.units), pl.why);
     return launch_status();
 }
@@ -588,14 +625,17 @@ ql_status run_swiglu(const SwigluPlan& pl, const void* x, const uint32_t* gc, co
     if ((s = encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xh, K, M, K * 2, fused::BK, fused::BT,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
-    // 128-row code boxes: a tile's gate rows, then the same rows of the up weight
-    if ((s = encode_2d(&mcg, CU_TENSOR_MAP_DATA_TYPE_UINT32, gc, K / 8, I, K / 2, fused::BK / 8, fused::BWG,
-                       CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+    // 128-row code boxes of one code stage (128 bytes per row, 128-byte swizzle): a tile's gate rows,
+    // then the same rows of the up weight
+    using FB = fused::PickCfg<4, true>::type;
+    using FF = fused::PickCfg<4, false>::type;
+    if ((s = encode_2d(&mcg, CU_TENSOR_MAP_DATA_TYPE_UINT32, gc, K / 8, I, K / 2, fused::kCodeRowBytes / 4, fused::BWG,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
-    if ((s = encode_2d(&mcu, CU_TENSOR_MAP_DATA_TYPE_UINT32, uc, K / 8, I, K / 2, fused::BK / 8, fused::BWG,
-                       CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
+    if ((s = encode_2d(&mcu, CU_TENSOR_MAP_DATA_TYPE_UINT32, uc, K / 8, I, K / 2, fused::kCodeRowBytes / 4, fused::BWG,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != QL_OK)
         return s;
-    if ((s = encode_2d(&mp, CU_TENSOR_MAP_DATA_TYPE_UINT32, sb, pl.ncols, G, pl.ncols * 4, fused::BW, 1,
+    if ((s = encode_2d(&mp, CU_TENSOR_MAP_DATA_TYPE_UINT32, sb, pl.ncols, G, pl.ncols * 4, fused::BW, FB::kS,
                        CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
         return s;
     if ((s = encode_2d(&my, bf16_out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, h, I, M,
@@ -621,17 +661,17 @@ ql_status run_swiglu(const SwigluPlan& pl, const void* x, const uint32_t* gc, co
     p.splits = 1;
     const int tiles = p.num_t * p.num_w;
     const int grid = std::min(tiles, sm_count);
-    using FC = fused::DefaultCfg;
     const dim3 fgrid(static_cast<unsigned>(grid));
     prof_begin(st);
-    s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, FC, true>, fgrid, fused::kThreads, FC::kSmemBytes,
+    s = bf16_out ? launch_dependent(fused::fused_gemm_kernel<true, FB, true>, fgrid, fused::kThreads, FB::kSmemBytes,
                                     st, mx, mcg, mcu, mp, my, p)
-                 : launch_dependent(fused::fused_gemm_kernel<false, FC, true>, fgrid, fused::kThreads, FC::kSmemBytes,
+                 : launch_dependent(fused::fused_gemm_kernel<false, FF, true>, fgrid, fused::kThreads, FF::kSmemBytes,
                                     st, mx, mcg, mcu, mp, my, p);
     if (s != QL_OK) return s;
     prof_end(st);
-    set_dispatch("path=tc_fused_swiglu bits=4 tile=%dg+%du x %dt x %dk stages=x%d/c%d/a%d ctas=%d launches=3",
-                 fused::BWG, fused::BWG, fused::BT, fused::BK, FC::kNX, FC::kNC, fused::NA, grid);
+    set_dispatch("path=tc_fused_swiglu bits=4 tile=%dg+%du x %dt x %dk stages=x%d/c%dx%d/a%d ctas=%d launches=3",
+                 fused::BWG, fused::BWG, fused::BT, fused::BK, bf16_out ? FB::kNX : FF::kNX,
+                 bf16_out ? FB::kNC : FF::kNC, FB::kS, fused::NA, grid);
     return launch_status();
 }
 
@@ -835,6 +875,21 @@ ql_status qlinear_test_stall(int32_t kernel_mask, uint64_t wait_limit_ns) {
 #else
     (void)kernel_mask;
     (void)wait_limit_ns;
+    return QL_ERR_UNSUPPORTED;
+#endif
+}
+
+ql_status qlinear_test_ring_depth(int32_t variant) {
+#ifdef QL_BOUNDS_CHECK
+    if (variant < 0 || variant >= QL_TEST_RING_VARIANTS) return QL_ERR_INVALID_ARG;
+    if (ring_smem_attr<RingV1>() != cudaSuccess || ring_smem_attr<RingV2>() != cudaSuccess ||
+        ring_smem_attr<RingV3>() != cudaSuccess || ring_smem_attr<RingV4>() != cudaSuccess ||
+        ring_smem_attr<RingV5>() != cudaSuccess || ring_smem_attr<RingV6>() != cudaSuccess)
+        return QL_ERR_CUDA;
+    g_ring_variant.store(variant);
+    return QL_OK;
+#else
+    (void)variant;
     return QL_ERR_UNSUPPORTED;
 #endif
 }

@@ -22,7 +22,47 @@ namespace ql {
 
 constexpr int kPrepThreads = 256;
 
-// One CTA per row.  Pass 1 reads the row for max|x|, pass 2 re-reads (L2) and converts.
+// One CTA per row.  Pass 1 reads the row for max|x|, keeping up to kConvCache 8-blocks per thread in
+// registers (all of a row of K <= 8192), pass 2 converts them (re-reading, from L2, only what did not
+// fit).  All of a thread's pass-1 loads are issued before the first is used.
+constexpr int kConvCache = 4;
+
+// The f16 8-block of a bf16 8-block scaled by inv, in the k order the dequantizer of kBits-bit codes
+// emits its pairs in.
+template <int kBits>
+__device__ __forceinline__ uint4 convert8(const uint4 v, float inv) {
+    // source order 0..7 = (v.x lo, v.x hi, v.y lo, v.y hi, v.z lo, v.z hi, v.w lo, v.w hi)
+    const float f0 = bf16_lo(v.x) * inv, f1 = bf16_hi(v.x) * inv;
+    const float f2 = bf16_lo(v.y) * inv, f3 = bf16_hi(v.y) * inv;
+    const float f4 = bf16_lo(v.z) * inv, f5 = bf16_hi(v.z) * inv;
+    const float f6 = bf16_lo(v.w) * inv, f7 = bf16_hi(v.w) * inv;
+    uint4 o;
+    if constexpr (kBits == 4) {
+        o.x = bits_of(__floats2half2_rn(f0, f4));
+        o.y = bits_of(__floats2half2_rn(f1, f5));
+        o.z = bits_of(__floats2half2_rn(f2, f6));
+        o.w = bits_of(__floats2half2_rn(f3, f7));
+    } else {
+        static_assert(kBits == 8, "4- or 8-bit codes");
+        o.x = bits_of(__floats2half2_rn(f0, f2));
+        o.y = bits_of(__floats2half2_rn(f1, f3));
+        o.z = bits_of(__floats2half2_rn(f4, f6));
+        o.w = bits_of(__floats2half2_rn(f5, f7));
+    }
+    return o;
+}
+
+__device__ __forceinline__ float absmax_bf16x8(const uint4 v, float amax) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // bit-level |.|: NaN patterns compare above every finite value
+        amax = fmaxf(amax, fabsf(bf16_lo(w[j])));
+        amax = fmaxf(amax, fabsf(bf16_hi(w[j])));
+    }
+    return amax;
+}
+
 // kBits: width of the weight codes the activations will meet (4 or 8), which fixes the k order.
 template <int kBits>
 __global__ void __launch_bounds__(kPrepThreads) convert_x_kernel(const __nv_bfloat16* __restrict__ x,
@@ -36,17 +76,17 @@ __global__ void __launch_bounds__(kPrepThreads) convert_x_kernel(const __nv_bflo
     uint4* dst = reinterpret_cast<uint4*>(xh + m * K);
     const int n8 = K / 8;
 
-    float amax = 0.0f;
-    for (int i = threadIdx.x; i < n8; i += kPrepThreads) {
-        const uint4 v = __ldg(src + i);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint4 v[kConvCache];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            // bit-level |.|: NaN patterns compare above every finite value
-            amax = fmaxf(amax, fabsf(bf16_lo(w[j])));
-            amax = fmaxf(amax, fabsf(bf16_hi(w[j])));
-        }
+    for (int j = 0; j < kConvCache; ++j) {
+        const int i = threadIdx.x + j * kPrepThreads;
+        v[j] = i < n8 ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
     }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kConvCache; ++j) amax = absmax_bf16x8(v[j], amax);
+    for (int i = threadIdx.x + kConvCache * kPrepThreads; i < n8; i += kPrepThreads)
+        amax = absmax_bf16x8(__ldg(src + i), amax);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
@@ -64,28 +104,13 @@ __global__ void __launch_bounds__(kPrepThreads) convert_x_kernel(const __nv_bflo
     }
     __syncthreads();
     const float inv = __uint_as_float(static_cast<uint32_t>(127 - row_exp) << 23);   // 2^-e, exact
-    for (int i = threadIdx.x; i < n8; i += kPrepThreads) {
-        const uint4 v = __ldg(src + i);
-        // source order 0..7 = (v.x lo, v.x hi, v.y lo, v.y hi, v.z lo, v.z hi, v.w lo, v.w hi)
-        const float f0 = bf16_lo(v.x) * inv, f1 = bf16_hi(v.x) * inv;
-        const float f2 = bf16_lo(v.y) * inv, f3 = bf16_hi(v.y) * inv;
-        const float f4 = bf16_lo(v.z) * inv, f5 = bf16_hi(v.z) * inv;
-        const float f6 = bf16_lo(v.w) * inv, f7 = bf16_hi(v.w) * inv;
-        uint4 o;
-        if constexpr (kBits == 4) {
-            o.x = bits_of(__floats2half2_rn(f0, f4));
-            o.y = bits_of(__floats2half2_rn(f1, f5));
-            o.z = bits_of(__floats2half2_rn(f2, f6));
-            o.w = bits_of(__floats2half2_rn(f3, f7));
-        } else {
-            static_assert(kBits == 8, "4- or 8-bit codes");
-            o.x = bits_of(__floats2half2_rn(f0, f2));
-            o.y = bits_of(__floats2half2_rn(f1, f3));
-            o.z = bits_of(__floats2half2_rn(f4, f6));
-            o.w = bits_of(__floats2half2_rn(f5, f7));
-        }
-        dst[i] = o;
+#pragma unroll
+    for (int j = 0; j < kConvCache; ++j) {
+        const int i = threadIdx.x + j * kPrepThreads;
+        if (i < n8) dst[i] = convert8<kBits>(v[j], inv);
     }
+    for (int i = threadIdx.x + kConvCache * kPrepThreads; i < n8; i += kPrepThreads)
+        dst[i] = convert8<kBits>(__ldg(src + i), inv);
 }
 
 // sb[g][n] = (scale[n][g], bias[n][g]); 32x32 tiles through shared memory.  Launched behind

@@ -78,6 +78,29 @@ __device__ __forceinline__ bool elect_one() {
 
 // ------------------------------------------------------------------ programmatic dependent launch
 
+// ------------------------------------------------------------------ thread-block clusters
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Every thread of every CTA of the cluster arrives, then waits for all of them (the hardware cluster
+// barrier; the CTAs of a cluster are resident together, so it completes once all have arrived).
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// A float of CTA `rank`'s shared memory at the address that p has in this CTA's.
+__device__ __forceinline__ float ld_shared_cluster_f32(const void* p, uint32_t rank) {
+    uint32_t remote;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(p)), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+
 // Lets the next kernel on the stream (launched with programmatic stream
 // serialization) be scheduled before this grid finishes; it must still call
 // grid_dependency_wait before it reads anything this grid writes.

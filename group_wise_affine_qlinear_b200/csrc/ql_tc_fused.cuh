@@ -37,9 +37,10 @@
 //               32*(w%4).. of group (w-12)/4): TMEM -> registers -> rowscale ->
 //               bf16/fp32 -> a 32x32 staging block in shared memory -> TMA
 //               tensor store (which also clips the ragged edges of y)
-// Rings: X (activation tiles, freed by MMA completion), C (codes + parameters,
-// freed once read by the dequantizers), A (TMEM weight stages, freed by MMA
-// completion); accumulators are freed per group by the epilogue.
+// Rings: X (activation tiles, one K-step each, freed by MMA completion), C (codes +
+// parameters of kS consecutive K-steps, freed once the dequantizers have read the
+// last of them), A (TMEM weight stages, one K-step each, freed by MMA completion);
+// accumulators are freed per group by the epilogue.
 //
 // SwiGLU mode (kSwiGLU): the DiT block's MLP is a SwiGLU of three Linears (jimmysue
 // "Ideogram 4" notes, sec. 2.1 and 2.8); this mode fuses the gate and up
@@ -79,16 +80,22 @@ constexpr int NA = 2;                   // TMEM weight stages
 static_assert(kAStageCol + NA * NG * 32 <= kTmemCols, "tensor memory budget");
 
 constexpr uint32_t kXBytes = BT * BK * 2;   // 24 KB
-constexpr uint32_t kPBytes = BW * 4;        // 1 KB of (scale, bias)
-constexpr uint32_t kStageBytes = 32 * 32 * 4;   // one epilogue staging block (fp32 worst case)
-constexpr uint32_t kEpiBytes = kEpiWarps * 2 * kStageBytes;   // 2 buffers per epilogue warp
+constexpr uint32_t kCodeRowBytes = 128;     // code bytes of one weight row per code stage
 
-// NX activation stages, NC code stages, B-bit codes (4: 8 KB of codes per stage; 8: 16 KB, stored
-// with the 64-byte swizzle).
-template <int NX, int NC, int B = 4>
+// NX activation stages; NC code stages, each holding kS = 128 / (8 * B) consecutive K-steps of B-bit
+// codes (128 bytes of every one of the tile's 256 rows, stored with the 128-byte swizzle: 4 steps of
+// 4-bit codes, 2 of 8-bit codes) with their (scale, bias) pairs; epilogue staging blocks of 32 x 32
+// outputs of OB bytes each (2: bf16, 4: fp32), NB of them per epilogue warp.  Wide code rows keep the
+// number of rows the TMA unit fetches per K-step low (64 rows of 128 bytes instead of 256 of 32); the
+// narrower bf16 staging leaves room for a fifth activation stage.
+template <int NX, int NC, int B, int OB, int NB>
 struct Cfg {
-    static constexpr int kNX = NX, kNC = NC, kBits = B;
-    static constexpr uint32_t kCBytes = BW * BK * B / 8;
+    static constexpr int kNX = NX, kNC = NC, kBits = B, kOutBytes = OB, kNB = NB;
+    static constexpr int kS = kCodeRowBytes / (BK * B / 8);
+    static constexpr uint32_t kCBytes = BW * kCodeRowBytes;
+    static constexpr uint32_t kPBytes = BW * 4 * kS;
+    static constexpr uint32_t kStageBytes = 32 * 32 * OB;
+    static constexpr uint32_t kEpiBytes = kEpiWarps * NB * kStageBytes;
     static constexpr uint32_t kOffX = 0;
     static constexpr uint32_t kOffC = kOffX + NX * kXBytes;
     static constexpr uint32_t kOffP = kOffC + NC * kCBytes;
@@ -97,12 +104,18 @@ struct Cfg {
     static constexpr uint32_t kNumBars = 2 * NX + 2 * NC + 2 * NA + 1 + NG + NG;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
-    static_assert(kXBytes % 1024 == 0, "swizzle atoms need 1 KB alignment");
+    static_assert(kXBytes % 1024 == 0 && kCBytes % 1024 == 0, "swizzle atoms need 1 KB alignment");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-using DefaultCfg = Cfg<4, 6>;
-using Q8Cfg = Cfg<4, 3, 8>;
+// The configuration of each (code width, output type): bf16 outputs stage in half the space of fp32
+// ones (split-K partials, fp32 outputs), which keep one staging block per warp to stay in budget.
+template <int B, bool kBf16Out>
+struct PickCfg;
+template <> struct PickCfg<4, true> { using type = Cfg<5, 2, 4, 2, 2>; };
+template <> struct PickCfg<4, false> { using type = Cfg<4, 2, 4, 4, 1>; };
+template <> struct PickCfg<8, true> { using type = Cfg<5, 2, 8, 2, 2>; };
+template <> struct PickCfg<8, false> { using type = Cfg<4, 2, 8, 4, 1>; };
 
 struct Params {
     float* rowscale;      // [M] 2^e_m
@@ -138,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
     constexpr int NX = C::kNX, NC = C::kNC;
     static_assert(!kSwiGLU || C::kBits == 4, "the SwiGLU pair is built for 4-bit codes");
     static_assert(!kSplitK || (!kSwiGLU && !kBf16Out), "split-K units write fp32 partials of a plain layer");
+    static_assert(kBf16Out == (C::kOutBytes == 2), "the staging blocks are sized for the output type");
     constexpr int kCodeWords = BK * C::kBits / 32;      // 32-bit code words of one row per K-step
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -172,21 +186,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             kb1 = p.G;
         }
     };
-    // K-steps this CTA runs in total (the sum over its units); every ring position is a function of the
-    // step index.
-    uint32_t total_steps;
-    if constexpr (kSplitK) {
-        total_steps = 0;
-        for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
-            int t, kb0, kb1;
-            unit(u, t, kb0, kb1);
-            total_steps += static_cast<uint32_t>(kb1 - kb0);
-        }
-    } else {
-        const uint32_t my_tiles = blockIdx.x < static_cast<unsigned>(num_tiles)
-                                      ? (static_cast<uint32_t>(num_tiles) - 1u - blockIdx.x) / gridDim.x + 1u : 0u;
-        total_steps = my_tiles * static_cast<uint32_t>(p.G);
-    }
+    // Every role walks the same units in the same order: the X and A ring positions follow the K-step
+    // count, the C ring position the code-stage count (a unit's steps in stages of kS, the last partial).
 
     if (threadIdx.x == 0) {
         // x and A stages are released by both MMA warps' commits
@@ -222,148 +223,164 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         const int grp = warp >> 2;                 // weight-row group
         const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
         const int r = grp * BWG + quarter * 32 + lane;   // weight row within the tile
-        // Rows whose bit 2 is set read their two 16-byte halves in the opposite order,
-        // so each group of 8 lanes touches 8 distinct 16-byte bank groups.
-        const int h = (r >> 2) & 1;
+        const int sw = r & 7;                      // the 128-byte swizzle of row r's 16-byte pieces
+        const uint8_t* crow0 = smem + C::kOffC + r * kCodeRowBytes;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        for (uint32_t i = 0; i < total_steps; ++i) {
-            int cs, as;
-            uint32_t cph, aph;
-            ring_pos<NC>(i, cs, cph);
-            ring_pos<NA>(i, as, aph);
-            // Codes arrive far ahead of the tensor core: unpack them into registers first
-            // and wait for the TMEM stage only when the result is ready to be written.
-            bool got = ptx::mbar_wait(&c_full[cs], cph, abort_flag);
-            if (!__all_sync(0xFFFFFFFFu, got)) break;
-            uint32_t a[32];
-            if constexpr (C::kBits == 4) {
-                const uint4* crow = reinterpret_cast<const uint4*>(smem + C::kOffC + cs * C::kCBytes + r * 32);
-                const uint4 first = crow[h];
-                const uint4 second = crow[h ^ 1];
-                const uint32_t sb = reinterpret_cast<const uint32_t*>(smem + C::kOffP + cs * kPBytes)[r];
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&c_empty[cs]);     // codes and parameters are in registers
-                const uint4 c0 = h ? second : first;
-                const uint4 c1 = h ? first : second;
-                const __half2 sb2 = half2_of(sb);
-                const __half2 s2 = __low2half2(sb2);
-                const __half2 b2 = __high2half2(sb2);
-                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        uint32_t i = 0, ci = 0;                    // K-step and code-stage counters
+        bool ok = true;
+        for (int un = blockIdx.x; un < num_units && ok; un += gridDim.x) {
+            int t, kb0, kb1;
+            unit(un, t, kb0, kb1);
+            for (int kc = kb0; kc < kb1 && ok; kc += C::kS, ++ci) {
+                int cs;
+                uint32_t cph;
+                ring_pos<NC>(ci, cs, cph);
+                // Codes arrive far ahead of the tensor core: unpack them into registers first
+                // and wait for the TMEM stage only when the result is ready to be written.
+                if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&c_full[cs], cph, abort_flag))) { ok = false; break; }
+                const uint8_t* crow = crow0 + cs * C::kCBytes;
+                const uint32_t* sbs = reinterpret_cast<const uint32_t*>(smem + C::kOffP + cs * C::kPBytes);
+                const int nsteps = min(C::kS, kb1 - kc);
+                for (int st = 0; st < nsteps; ++st, ++i) {
+                    int as;
+                    uint32_t aph;
+                    ring_pos<NA>(i, as, aph);
+                    uint32_t a[32];
+                    const uint32_t sb = sbs[st * BW + r];
+                    const __half2 sb2 = half2_of(sb);
+                    const __half2 s2 = __low2half2(sb2);
+                    const __half2 b2 = __high2half2(sb2);
+                    if constexpr (C::kBits == 4) {
+                        // step st is pieces 2st, 2st+1 of the row (16 codes each)
+                        const uint4 c0 = *reinterpret_cast<const uint4*>(crow + (((2 * st) ^ sw) << 4));
+                        const uint4 c1 = *reinterpret_cast<const uint4*>(crow + (((2 * st + 1) ^ sw) << 4));
+                        if (st + 1 == nsteps) {            // the stage's codes and parameters are in registers
+                            __syncwarp();
+                            if (lane == 0) ptx::mbar_arrive(&c_empty[cs]);
+                        }
+                        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-                for (int c = 0; c < 8; ++c) dequant_word(words[c], s2, b2, &a[4 * c]);
-            } else {
-                // Row r's 64 code bytes are four 16-byte pieces stored with the 64-byte swizzle (piece c
-                // at c ^ ((r >> 1) & 3)), so every 8 lanes of a load touch 8 distinct bank groups.
-                const uint8_t* crow = smem + C::kOffC + cs * C::kCBytes + r * 64;
-                const int sw = (r >> 1) & 3;
-                uint4 cv[4];
+                        for (int c = 0; c < 8; ++c) dequant_word(words[c], s2, b2, &a[4 * c]);
+                    } else {
+                        // step st is pieces 4st .. 4st+3 of the row (16 byte codes each)
+                        uint4 cv[4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) cv[c] = *reinterpret_cast<const uint4*>(crow + ((c ^ sw) << 4));
-                const uint32_t sb = reinterpret_cast<const uint32_t*>(smem + C::kOffP + cs * kPBytes)[r];
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&c_empty[cs]);     // codes and parameters are in registers
-                const __half2 sb2 = half2_of(sb);
-                const __half2 s2 = __low2half2(sb2);
-                const __half2 b2 = __high2half2(sb2);
+                        for (int c = 0; c < 4; ++c)
+                            cv[c] = *reinterpret_cast<const uint4*>(crow + (((4 * st + c) ^ sw) << 4));
+                        if (st + 1 == nsteps) {
+                            __syncwarp();
+                            if (lane == 0) ptx::mbar_arrive(&c_empty[cs]);
+                        }
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    dequant_word8(cv[c].x, s2, b2, &a[8 * c + 0]);
-                    dequant_word8(cv[c].y, s2, b2, &a[8 * c + 2]);
-                    dequant_word8(cv[c].z, s2, b2, &a[8 * c + 4]);
-                    dequant_word8(cv[c].w, s2, b2, &a[8 * c + 6]);
+                        for (int c = 0; c < 4; ++c) {
+                            dequant_word8(cv[c].x, s2, b2, &a[8 * c + 0]);
+                            dequant_word8(cv[c].y, s2, b2, &a[8 * c + 2]);
+                            dequant_word8(cv[c].z, s2, b2, &a[8 * c + 4]);
+                            dequant_word8(cv[c].w, s2, b2, &a[8 * c + 6]);
+                        }
+                    }
+                    if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&a_empty[as], aph ^ 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after_sync();
+                    ptx::tmem_st_32x32b_x32(tmem_base + lane_addr + kAStageCol + 64u * as + 32u * grp, a);
+                    ptx::tmem_wait_st();
+                    ptx::tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&a_full[as]);
                 }
             }
-            got = ptx::mbar_wait(&a_empty[as], aph ^ 1, abort_flag);
-            if (!__all_sync(0xFFFFFFFFu, got)) break;
-            ptx::tc_fence_after_sync();
-            ptx::tmem_st_32x32b_x32(tmem_base + lane_addr + kAStageCol + 64u * as + 32u * grp, a);
-            ptx::tmem_wait_st();
-            ptx::tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&a_full[as]);
         }
-    } else if (warp == kWarpTmaX || warp == kWarpTmaC) {
-        // ---------------------------------------------------------------- TMA producers
-        // (the checked build's stall hook holds the code producer back: no code or parameter load)
-        if (lane == 0 && !(warp == kWarpTmaC && stalled(kStallFused))) {
-            const bool is_x = warp == kWarpTmaX;
-            const int depth = is_x ? NX : NC;
-            uint64_t* full = is_x ? x_full : c_full;
-            uint64_t* empty = is_x ? x_empty : c_empty;
+    } else if (warp == kWarpTmaX) {
+        // ---------------------------------------------------------------- TMA producer of activation tiles
+        if (lane == 0) {
             uint32_t i = 0;
             bool ok = true;
-            // The activations and the parameter pairs come from the kernels before this one on the
-            // stream (programmatic dependent launch): the code loads of the first NC stages go out
-            // at once, their parameter loads (same stage barrier) once those kernels are done.
-            const uint32_t first_steps = kSplitK ? total_steps : static_cast<uint32_t>(p.G) * static_cast<uint32_t>(
-                (num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x));
-            const uint32_t early = is_x ? 0u : min(static_cast<uint32_t>(NC), first_steps);
-            // one K-step of a tile's codes: 256 rows of one weight, or in SwiGLU mode 128 gate rows
-            // followed by the same 128 rows of the up weight
-            auto load_codes = [&](uint8_t* dst, uint64_t* bar, int kb, int w_blk) {
-                if constexpr (kSwiGLU) {
-                    ptx::tma_load_2d(dst, &map_codes, bar, kb * kCodeWords, w_blk * BWG);
-                    ptx::tma_load_2d(dst + C::kCBytes / 2, &map_codes2, bar, kb * kCodeWords, w_blk * BWG);
-                } else {
-                    ptx::tma_load_2d(dst, &map_codes, bar, kb * kCodeWords, w_blk * BW);
-                }
-            };
-            auto step_coords = [&](uint32_t step, int& kb, int& w_blk, int& t_blk) {
-                if constexpr (kSplitK) {
-                    // walk this CTA's units to the one holding its step-th K-step
-                    int u = static_cast<int>(blockIdx.x), t, kb0, kb1;
-                    unit(u, t, kb0, kb1);
-                    while (step >= static_cast<uint32_t>(kb1 - kb0)) {
-                        step -= static_cast<uint32_t>(kb1 - kb0);
-                        u += static_cast<int>(gridDim.x);
-                        unit(u, t, kb0, kb1);
-                    }
-                    kb = kb0 + static_cast<int>(step);
-                    tile_coords(t, p.num_w, t_blk, w_blk);
-                } else {
-                    const int t = static_cast<int>(blockIdx.x) + static_cast<int>(step / p.G) * static_cast<int>(gridDim.x);
-                    kb = static_cast<int>(step % p.G);
-                    tile_coords(t, p.num_w, t_blk, w_blk);
-                }
-            };
-            for (uint32_t e = 0; e < early; ++e) {       // fresh stages: no empty wait
-                int kb, w_blk, t_blk;
-                step_coords(e, kb, w_blk, t_blk);
-                ptx::mbar_arrive_expect_tx(&full[e], C::kCBytes + kPBytes);
-                load_codes(smem + C::kOffC + e * C::kCBytes, &full[e], kb, w_blk);
-            }
-            ptx::grid_dependency_wait();
-            for (uint32_t e = 0; e < early; ++e) {
-                int kb, w_blk, t_blk;
-                step_coords(e, kb, w_blk, t_blk);
-                ptx::tma_load_2d(smem + C::kOffP + e * kPBytes, &map_params, &full[e], w_blk * BW, kb);
-            }
+            ptx::grid_dependency_wait();               // the activations come from the prepass
             for (int un = blockIdx.x; un < num_units && ok; un += gridDim.x) {
                 int t, kb0, kb1;
                 unit(un, t, kb0, kb1);
                 int t_blk, w_blk;
                 tile_coords(t, p.num_w, t_blk, w_blk);
                 for (int kb = kb0; kb < kb1; ++kb, ++i) {
-                    if (i < early) continue;
-                    const int s = static_cast<int>(i % depth);
-                    const uint32_t ph = (i / depth) & 1u;
-                    if (!ptx::mbar_wait(&empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
-                    if (is_x) {
-                        ptx::mbar_arrive_expect_tx(&full[s], kXBytes);
-                        ptx::tma_load_2d(smem + C::kOffX + s * kXBytes, &map_x, &full[s], kb * BK, t_blk * BT);
-                    } else {
-                        ptx::mbar_arrive_expect_tx(&full[s], C::kCBytes + kPBytes);
-                        load_codes(smem + C::kOffC + s * C::kCBytes, &full[s], kb, w_blk);
-                        ptx::tma_load_2d(smem + C::kOffP + s * kPBytes, &map_params, &full[s], w_blk * BW, kb);
-                    }
+                    int s;
+                    uint32_t ph;
+                    ring_pos<NX>(i, s, ph);
+                    if (!ptx::mbar_wait(&x_empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(&x_full[s], kXBytes);
+                    ptx::tma_load_2d(smem + C::kOffX + s * kXBytes, &map_x, &x_full[s], kb * BK, t_blk * BT);
                 }
             }
             // Never leave the CTA with bulk copies still landing in its shared memory:
             // wait for the most recent load of every stage that received one.
-            const uint32_t issued = i;
-            for (uint32_t j = (issued > static_cast<uint32_t>(depth) ? issued - depth : 0u); j < issued; ++j) {
-                ptx::mbar_wait(&full[j % depth], (j / depth) & 1u, nullptr);
+            for (uint32_t j = (i > static_cast<uint32_t>(NX) ? i - NX : 0u); j < i; ++j)
+                ptx::mbar_wait(&x_full[j % NX], (j / NX) & 1u, nullptr);
+        }
+    } else if (warp == kWarpTmaC) {
+        // ---------------------------------------------------------------- TMA producer of codes and parameters
+        // (the checked build's stall hook holds it back: no code or parameter load)
+        if (lane == 0 && !stalled(kStallFused)) {
+            // one code stage: kS K-steps of a tile's 256 rows (in SwiGLU mode 128 gate rows, then the same
+            // 128 rows of the up weight); steps past the tensor's K are zero-filled, steps of the next
+            // split-K slice are loaded and not used
+            auto load_codes = [&](uint8_t* dst, uint64_t* bar, int kc, int w_blk) {
+                if constexpr (kSwiGLU) {
+                    ptx::tma_load_2d(dst, &map_codes, bar, kc * kCodeWords, w_blk * BWG);
+                    ptx::tma_load_2d(dst + C::kCBytes / 2, &map_codes2, bar, kc * kCodeWords, w_blk * BWG);
+                } else {
+                    ptx::tma_load_2d(dst, &map_codes, bar, kc * kCodeWords, w_blk * BW);
+                }
+            };
+            // The parameter pairs come from the kernel before this one on the stream (programmatic
+            // dependent launch): the code loads of the first NC stages go out at once, their parameter
+            // loads (same stage barrier) once that kernel is done.
+            uint32_t ci = 0;
+            bool ok = true, waited = false;
+            int first_kc[NC], first_w[NC];
+            for (int un = blockIdx.x; un < num_units && ok; un += gridDim.x) {
+                int t, kb0, kb1;
+                unit(un, t, kb0, kb1);
+                int t_blk, w_blk;
+                tile_coords(t, p.num_w, t_blk, w_blk);
+                for (int kc = kb0; kc < kb1; kc += C::kS, ++ci) {
+                    int s;
+                    uint32_t ph;
+                    ring_pos<NC>(ci, s, ph);
+                    if (ci >= static_cast<uint32_t>(NC) && !waited) {
+                        ptx::grid_dependency_wait();
+#pragma unroll
+                        for (int e = 0; e < NC; ++e)
+                            ptx::tma_load_2d(smem + C::kOffP + e * C::kPBytes, &map_params, &c_full[e],
+                                             first_w[e] * BW, first_kc[e]);
+                        waited = true;
+                    }
+                    if (!ptx::mbar_wait(&c_empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(&c_full[s], C::kCBytes + C::kPBytes);
+                    load_codes(smem + C::kOffC + s * C::kCBytes, &c_full[s], kc, w_blk);
+                    if (waited) {
+                        ptx::tma_load_2d(smem + C::kOffP + s * C::kPBytes, &map_params, &c_full[s], w_blk * BW, kc);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < NC; ++e) {     // constant indices keep the arrays in registers
+                            if (e == s) {
+                                first_kc[e] = kc;
+                                first_w[e] = w_blk;
+                            }
+                        }
+                    }
+                }
             }
+            if (!waited) {                             // fewer than NC stages in all
+                ptx::grid_dependency_wait();
+#pragma unroll
+                for (int e = 0; e < NC; ++e)
+                    if (static_cast<uint32_t>(e) < ci)
+                        ptx::tma_load_2d(smem + C::kOffP + e * C::kPBytes, &map_params, &c_full[e], first_w[e] * BW,
+                                         first_kc[e]);
+            }
+            for (uint32_t j = (ci > static_cast<uint32_t>(NC) ? ci - NC : 0u); j < ci; ++j)
+                ptx::mbar_wait(&c_full[j % NC], (j / NC) & 1u, nullptr);
         }
     } else if (warp == kWarpMma || warp == kWarpMma2) {
         // ---------------------------------------------------------------- MMA issuers, one per group
@@ -417,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         constexpr int kHalfChunks = BT / 32 / 2;
         const int quarter = warp & 3;
         const int half = (warp - kWarpEpi0) >> 2;
-        uint8_t* epi_stage = smem + C::kOffEpi + (warp - kWarpEpi0) * 2 * kStageBytes;
+        uint8_t* epi_stage = smem + C::kOffEpi + (warp - kWarpEpi0) * C::kNB * C::kStageBytes;
         uint32_t nstore = 0;
         int j = 0;
         ptx::grid_dependency_wait();               // the row scales come from the kernels before this one
@@ -444,8 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                 ptx::tmem_ld_32x32b_x32(tgate + chunk * 32, rg);
                 ptx::tmem_ld_32x32b_x32(tup + chunk * 32, ru);
                 ptx::tmem_wait_ld();
-                uint8_t* stage = epi_stage + (nstore & 1) * kStageBytes;
-                if (lane == 0) ptx::bulk_wait_group_read<1>();   // the store that used this buffer has read it
+                uint8_t* stage = epi_stage + (nstore % C::kNB) * C::kStageBytes;
+                if (lane == 0) ptx::bulk_wait_group_read<C::kNB - 1>();   // the store that used this buffer has read it
                 __syncwarp();
 #pragma unroll
                 for (int k = 0; k < 32; ++k) {
@@ -479,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         // ---------------------------------------------------------------- epilogue
         const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
         const int g = (warp - kWarpEpi0) >> 2;     // accumulator group this warp drains
-        uint8_t* epi_stage = smem + C::kOffEpi + (warp - kWarpEpi0) * 2 * kStageBytes;
+        uint8_t* epi_stage = smem + C::kOffEpi + (warp - kWarpEpi0) * C::kNB * C::kStageBytes;
         uint32_t nstore = 0;
         int j = 0;
         ptx::grid_dependency_wait();               // the row scales come from the kernels before this one
@@ -511,9 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                     ptx::tmem_wait_ld();
                     if (chunk + 1 < BT / 32) ptx::tmem_ld_32x32b_x32(taddr + (chunk + 1) * 32, r[(chunk + 1) & 1]);
                     const uint32_t* v = r[chunk & 1];
-                    // staging block [32 tokens][32 columns], double-buffered per warp
-                    uint8_t* stage = epi_stage + (nstore & 1) * kStageBytes;
-                    if (lane == 0) ptx::bulk_wait_group_read<1>();   // the store that used this buffer has read it
+                    // staging block [32 tokens][32 columns], C::kNB of them per warp
+                    uint8_t* stage = epi_stage + (nstore % C::kNB) * C::kStageBytes;
+                    if (lane == 0) ptx::bulk_wait_group_read<C::kNB - 1>();   // the store that used this buffer has read it
                     __syncwarp();
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {

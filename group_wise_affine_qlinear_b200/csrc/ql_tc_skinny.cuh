@@ -14,11 +14,13 @@
 // kernel's arithmetic (one f16 rounding of each weight, activations scaled per
 // row by a power of two into f16, fp32 accumulation) in a layout for few tokens.
 //
-// The activations come from a prepass pair under programmatic dependent launch:
-// per-slice row maxima, then x' = f16(x * 2^e_t) with e_t putting the row maximum
-// in [2^14, 2^15), in the order the dequantizer emits its pairs in (0,4,1,5,2,6,3,7
-// of every 8-block for 4-bit codes, 0,2,1,3,4,6,5,7 for 8-bit codes).  The main kernel starts streaming codes and parameters at
-// once and waits for the prepass only before its first activation load.
+// The activations come from one prepass kernel (a cluster of CTAs per row that
+// meet in distributed shared memory for the row maximum), which the main kernel
+// follows under programmatic dependent launch: x' = f16(x * 2^e_t) with e_t putting
+// the row maximum in [2^14, 2^15), in the order the dequantizer emits its pairs in
+// (0,4,1,5,2,6,3,7 of every 8-block for 4-bit codes, 0,2,1,3,4,6,5,7 for 8-bit
+// codes).  The main kernel starts streaming codes and parameters at once and waits
+// for the prepass only before its first activation load.
 //
 // Stream-K schedule: the work is cut into chunks of CG consecutive groups of one
 // 128-row tile (CG = 8 for 4-bit codes, 4 for the 8-bit codes of the Q8 pack,
@@ -121,63 +123,86 @@ __host__ __device__ __forceinline__ int64_t run_first(int64_t units, int P, int 
 // Activation prepass, two kernels over a grid of (slice, row): one thread per 8-block of k, 256 per
 // CTA, so every 8-block of a row is read in parallel.
 
-// pmax[t][slice] = max |x[t][k]| over the slice's 8-blocks.
-__global__ void __launch_bounds__(256) skinny_rowmax_kernel(const uint4* __restrict__ x, float* __restrict__ pmax,
-                                                            int K) {
-    ptx::launch_dependents();
-    __shared__ float red[8];
-    const int t = blockIdx.y, kb = K / 8;
-    const int c = blockIdx.x * 256 + threadIdx.x;
-    float m = 0.0f;
-    if (c < kb) {
-        const uint4 v = x[static_cast<int64_t>(t) * kb + c];
-        m = fmaxf(fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))),
-                  fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+// The activation prepass in one launch, one cluster of kPrepCluster CTAs per row t: each CTA takes
+// 1/kPrepCluster of the row's 8-blocks, the CTAs' maxima meet in distributed shared memory, then
+// e_t puts max_k |x[t][k]| in [2^14, 2^15) (0 for a zero or non-finite row);
+// xp[t][k] = f16(x * 2^e_t) in the order the dequantizer of kBits-bit codes emits its pairs in
+// (0,4,1,5,2,6,3,7 of each 8-block for 4-bit codes, 0,2,1,3,4,6,5,7 for 8-bit codes); rowexp[t] = -e_t.
+// Grid (kPrepCluster, M); no thread leaves before the second cluster barrier, so every CTA's shared
+// memory outlives its peers' reads of it.
+constexpr int kPrepCluster = 8;
+constexpr int kPrepThreads = 512;
+constexpr int kPrepCache = 4;                 // 8-blocks a thread keeps in registers between the passes
+
+__device__ __forceinline__ float absmax8(const uint4 v) {
+    return fmaxf(fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))), fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))),
+                 fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))), fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+}
+
+template <int kBits>
+__device__ __forceinline__ uint4 prescale8(const uint4 v, int ex) {
+    const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                        bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // 4-bit: slot pairs (k0, k4) (k1, k5) (k2, k6) (k3, k7); 8-bit: (k0, k2) (k1, k3) (k4, k6) (k5, k7)
+        const int lo = kBits == 4 ? j : 2 * (j & 2) + (j & 1);
+        const int hi = kBits == 4 ? j + 4 : lo + 2;
+        const __half2 h = __halves2half2(__float2half_rn(ldexpf(f[lo], ex)), __float2half_rn(ldexpf(f[hi], ex)));
+        o[j] = *reinterpret_cast<const uint32_t*>(&h);
     }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <int kBits>
+__global__ void __cluster_dims__(kPrepCluster, 1, 1) __launch_bounds__(kPrepThreads)
+    skinny_prepass_kernel(const uint4* __restrict__ x, uint4* __restrict__ xp, int* __restrict__ rowexp, int K) {
+    ptx::launch_dependents();
+    __shared__ float red[kPrepThreads / 32];
+    const int t = blockIdx.y, kb = K / 8;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const int per = (kb + kPrepCluster - 1) / kPrepCluster;
+    const int c0 = static_cast<int>(rank) * per, c1 = min(kb, c0 + per);
+    const uint4* xr = x + static_cast<int64_t>(t) * kb;
+    uint4 v[kPrepCache];
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kPrepCache; ++j) {
+        const int c = c0 + j * kPrepThreads + static_cast<int>(threadIdx.x);
+        v[j] = c < c1 ? xr[c] : make_uint4(0u, 0u, 0u, 0u);
+        m = fmaxf(m, absmax8(v[j]));
+    }
+    for (int c = c0 + kPrepCache * kPrepThreads + static_cast<int>(threadIdx.x); c < c1; c += kPrepThreads)
+        m = fmaxf(m, absmax8(xr[c]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     __syncthreads();
     if (threadIdx.x == 0) {
-        for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
-        pmax[static_cast<int64_t>(t) * gridDim.x + blockIdx.x] = fmaxf(m, red[0]);
+        for (int i = 1; i < kPrepThreads / 32; ++i) m = fmaxf(m, red[i]);
+        red[0] = m;                                   // this CTA's slice maximum
     }
-}
-
-// For row t: e_t puts max_k |x[t][k]| in [2^14, 2^15) (0 for a zero or non-finite row);
-// xp[t][k] = f16(x * 2^e_t) in the order the dequantizer of kBits-bit codes emits its pairs in
-// (0,4,1,5,2,6,3,7 of each 8-block for 4-bit codes, 0,2,1,3,4,6,5,7 for 8-bit codes); rowexp[t] = -e_t.
-template <int kBits>
-__global__ void __launch_bounds__(256) skinny_prepass_kernel(const uint4* __restrict__ x, const float* __restrict__ pmax,
-                                                             uint4* __restrict__ xp, int* __restrict__ rowexp, int K) {
-    ptx::launch_dependents();
-    ptx::grid_dependency_wait();                               // pmax comes from the kernel before
-    const int t = blockIdx.y, kb = K / 8;
-    const int c = blockIdx.x * 256 + threadIdx.x;
-    float m = 0.0f;
-    for (int i = 0; i < static_cast<int>(gridDim.x); ++i) m = fmaxf(m, pmax[static_cast<int64_t>(t) * gridDim.x + i]);
+    ptx::cluster_sync();                              // every CTA's red[0] is written
+    m = 0.0f;
+#pragma unroll
+    for (int r = 0; r < kPrepCluster; ++r) m = fmaxf(m, ptx::ld_shared_cluster_f32(&red[0], static_cast<uint32_t>(r)));
+    ptx::cluster_sync();                              // every peer has read this CTA's red[0]
     int ex = 0;
     if (m > 0.0f && m <= 3.4028235e38f) {
         int E;
-        frexpf(m, &E);                                         // m = f 2^E, f in [0.5, 1)
+        frexpf(m, &E);                                // m = f 2^E, f in [0.5, 1)
         ex = 15 - E;
     }
-    if (blockIdx.x == 0 && threadIdx.x == 0) rowexp[t] = -ex;
-    if (c < kb) {
-        const uint4 v = x[static_cast<int64_t>(t) * kb + c];
-        const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                            bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-        uint32_t o[4];
+    if (rank == 0 && threadIdx.x == 0) rowexp[t] = -ex;
+    uint4* xo = xp + static_cast<int64_t>(t) * kb;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            // 4-bit: slot pairs (k0, k4) (k1, k5) (k2, k6) (k3, k7); 8-bit: (k0, k2) (k1, k3) (k4, k6) (k5, k7)
-            const int lo = kBits == 4 ? j : 2 * (j & 2) + (j & 1);
-            const int hi = kBits == 4 ? j + 4 : lo + 2;
-            const __half2 h = __halves2half2(__float2half_rn(ldexpf(f[lo], ex)), __float2half_rn(ldexpf(f[hi], ex)));
-            o[j] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        xp[static_cast<int64_t>(t) * kb + c] = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int j = 0; j < kPrepCache; ++j) {
+        const int c = c0 + j * kPrepThreads + static_cast<int>(threadIdx.x);
+        if (c < c1) xo[c] = prescale8<kBits>(v[j], ex);
     }
+    for (int c = c0 + kPrepCache * kPrepThreads + static_cast<int>(threadIdx.x); c < c1; c += kPrepThreads)
+        xo[c] = prescale8<kBits>(xr[c], ex);
 }
 
 template <int NT, int B>

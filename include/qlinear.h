@@ -163,8 +163,10 @@ QL_API ql_status qlinear_get_device_status(cudaStream_t stream);
 
 /*
  * Writes a NUL-terminated description of the calling thread's last
- * qlinear_forward dispatch, e.g. "path=tc_fused bits=4 tile=256w x 192t x 64k stages=x4/c6/a2
- * ctas=148 splitk=1 launches=3" (launches = kernels that call enqueued),
+ * qlinear_forward dispatch, e.g. "path=tc_fused bits=4 tile=256w x 192t x 64k stages=x5/c2x4/a2
+ * ctas=148 splitk=1 launches=3 why=auto:M>64,split:9x72" (stages: activation, code x K-steps per
+ * code stage, tensor-memory weight stages; launches = kernels that call enqueued; why = the rule or
+ * the caller's forced path behind the choice),
  * truncated to len bytes.  QL_ERR_INVALID_ARG if buf is NULL or len == 0.
  */
 QL_API ql_status qlinear_last_dispatch(char* buf, size_t len);
@@ -181,6 +183,19 @@ QL_API ql_status qlinear_last_dispatch(char* buf, size_t len);
  * unknown bit or a zero limit.
  */
 QL_API ql_status qlinear_test_stall(int32_t kernel_mask, uint64_t wait_limit_ns);
+
+/*
+ * Test hook of the checked build (libqlinear_bounds.so); the pages have no counterpart.  Selects the ring
+ * depths of the fused tensor-core kernel that later 4-bit, bf16-output, unsplit qlinear_forward calls
+ * (QL_PATH_TC_FUSED or the dispatcher's choice of it) launch on this process: variant 0 is the shipped
+ * configuration, variants 1 .. QL_TEST_RING_VARIANTS-1 other (activation stages, code stages, epilogue
+ * staging blocks per warp) triples.  Every ring position is a function of the step count alone, so the
+ * output must be the same bytes for every variant.  The shipped library returns QL_ERR_UNSUPPORTED;
+ * QL_ERR_INVALID_ARG for a variant out of range; QL_ERR_CUDA if the variant's shared-memory size
+ * cannot be set on the current device.
+ */
+#define QL_TEST_RING_VARIANTS 7
+QL_API ql_status qlinear_test_ring_depth(int32_t variant);
 
 /*
  * Allocation-free forward for small M.  The pages have no counterpart of this

@@ -237,3 +237,10 @@ def test_bounds_checked_build_exports_every_declared_symbol():
     Lb = ctypes.CDLL(qb.build(bounds_check=True))
     for n in _declared():
         assert hasattr(Lb, n), n
+
+
+def test_test_hooks_are_inert_in_the_shipped_library(L):
+    """The checked build's hooks (held-back producers, ring depths) change nothing in the shipped library."""
+    assert L.qlinear_test_stall(1, 20_000_000) == 3              # QL_ERR_UNSUPPORTED
+    assert L.qlinear_test_ring_depth(1) == 3
+    assert L.qlinear_test_ring_depth(0) == 3
