@@ -33,10 +33,10 @@
 //   warps 9, 11 single-thread MMA issuers for groups 0 / 1 (warp 9 also allocates TMEM);
 //               issuing from two threads doubles the tcgen05.mma issue rate
 //   warp 10     TMA producer of code and parameter tiles
-//   warps 12-19 epilogue, one set of four per group (warp w drains TMEM lanes
-//               32*(w%4).. of group (w-12)/4): TMEM -> registers -> rowscale ->
-//               bf16/fp32 -> a 32x32 staging block in shared memory -> TMA
-//               tensor store (which also clips the ragged edges of y)
+//   warps 12-19 epilogue: all eight drain group 0, then group 1 (warp w takes TMEM
+//               lanes 32*(w%4).. and half of the tokens): TMEM -> registers ->
+//               rowscale -> bf16/fp32 -> a 32x32 staging block in shared memory ->
+//               TMA tensor store (which also clips the ragged edges of y)
 // Rings: X (activation tiles, one K-step each, freed by MMA completion), C (codes +
 // parameters of kS consecutive K-steps, freed once the dequantizers have read the
 // last of them), A (TMEM weight stages, one K-step each); accumulators are freed per
@@ -201,8 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         for (int i = 0; i < NA; ++i) ptx::mbar_init(&a_full[i], kDequantWarps);
         ptx::mbar_init(&acc_full[0], NG);
         static_assert(kWarpEpi0 % 4 == 0, "epilogue warp w must own TMEM lane quarter w % 4");
-        // an accumulator is drained by its group's 4 epilogue warps, or in SwiGLU mode by all 8
-        for (int g = 0; g < NG; ++g) ptx::mbar_init(&acc_empty[g], kSwiGLU ? kEpiWarps : 4);
+        // an accumulator is drained by all 8 epilogue warps (a lane quarter and half of the tokens each)
+        for (int g = 0; g < NG; ++g) ptx::mbar_init(&acc_empty[g], kEpiWarps);
         for (int g = 0; g < NG; ++g) ptx::mbar_init(drain + g, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -503,8 +503,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         if (lane == 0) ptx::bulk_wait_group_all();   // every store has completed before the CTA exits
     } else if (warp >= kWarpEpi0) {
         // ---------------------------------------------------------------- epilogue
+        // All 8 warps drain group 0's accumulator first, then group 1's: warp (quarter, half) takes TMEM
+        // lanes 32*quarter .. +31 and the token chunks kHalf*half .. +kHalf-1 of each group, so group 0 is
+        // released after half a drain and its MMAs of the next unit run while group 1 is drained.
+        constexpr int kHalf = BT / 32 / 2;         // token chunks of 32 per warp and group
         const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
-        const int g = (warp - kWarpEpi0) >> 2;     // accumulator group this warp drains
+        const int half = (warp - kWarpEpi0) >> 2;
         uint8_t* epi_stage = smem + C::kOffEpi + (warp - kWarpEpi0) * C::kNB * C::kStageBytes;
         uint32_t nstore = 0;
         int j = 0;
@@ -514,40 +518,42 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
             unit(un, t, kb0, kb1);
             int t_blk, w_blk;
             tile_coords(t, p.num_w, t_blk, w_blk);
-            // Row scales of the tile's tokens, fetched before the accumulators are ready:
-            // rs[c] belongs to token t_blk*BT + 32c + lane.
-            float rs[BT / 32];
+            // Row scales of this warp's tokens, fetched before the accumulators are ready:
+            // rs[c] belongs to token t_blk*BT + 32*(kHalf*half + c) + lane.
+            float rs[kHalf];
 #pragma unroll
-            for (int c = 0; c < BT / 32; ++c) {
-                const int m = t_blk * BT + 32 * c + lane;
+            for (int c = 0; c < kHalf; ++c) {
+                const int m = t_blk * BT + 32 * (kHalf * half + c) + lane;
                 rs[c] = (m < p.M) ? p.rowscale[m] : 0.0f;
             }
             const bool got = ptx::mbar_wait(&acc_full[0], j & 1, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
             ptx::tc_fence_after_sync();
-            {
+#pragma unroll 1
+            for (int g = 0; g < NG; ++g) {
                 const int n_base = w_blk * BW + g * BWG + quarter * 32;   // this warp's 32 output columns
-                const uint32_t taddr = tmem_base + kAccCol + static_cast<uint32_t>(g * BT) +
+                const uint32_t taddr = tmem_base + kAccCol + static_cast<uint32_t>(g * BT + 32 * kHalf * half) +
                                        (static_cast<uint32_t>(quarter * 32) << 16);
                 // Two register buffers: the TMEM load of chunk c+1 is in flight while chunk c is stored.
                 uint32_t r[2][32];
                 ptx::tmem_ld_32x32b_x32(taddr, r[0]);
 #pragma unroll
-                for (int chunk = 0; chunk < BT / 32; ++chunk) {
+                for (int c = 0; c < kHalf; ++c) {
+                    const int chunk = kHalf * half + c;
                     ptx::tmem_wait_ld();
-                    if (chunk + 1 < BT / 32) ptx::tmem_ld_32x32b_x32(taddr + (chunk + 1) * 32, r[(chunk + 1) & 1]);
-                    const uint32_t* v = r[chunk & 1];
+                    if (c + 1 < kHalf) ptx::tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r[(c + 1) & 1]);
+                    const uint32_t* v = r[c & 1];
                     // staging block [32 tokens][32 columns], C::kNB of them per warp
                     uint8_t* stage = epi_stage + (nstore % C::kNB) * C::kStageBytes;
                     if (lane == 0) ptx::bulk_wait_group_read<C::kNB - 1>();   // the store that used this buffer has read it
                     __syncwarp();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const float val = __uint_as_float(v[c]) * __shfl_sync(0xFFFFFFFFu, rs[chunk], c);
+                    for (int k = 0; k < 32; ++k) {
+                        const float val = __uint_as_float(v[k]) * __shfl_sync(0xFFFFFFFFu, rs[c], k);
                         if constexpr (kBf16Out) {
-                            reinterpret_cast<__nv_bfloat16*>(stage)[c * 32 + lane] = __float2bfloat16_rn(val);
+                            reinterpret_cast<__nv_bfloat16*>(stage)[k * 32 + lane] = __float2bfloat16_rn(val);
                         } else {
-                            reinterpret_cast<float*>(stage)[c * 32 + lane] = val;
+                            reinterpret_cast<float*>(stage)[k * 32 + lane] = val;
                         }
                     }
                     ptx::fence_proxy_async_smem();
