@@ -371,3 +371,28 @@ def test_full_mlp_down():
 @pytest.mark.parametrize("name", ["canvas2048_n4608", "canvas2048_n13824"])
 def test_full_canvas2048(name):
     _full_case(name)
+
+
+@pytest.mark.parametrize("name,M,split", [("qkv", None, 0), ("text_proj", 512, 0), ("text_proj", 32, 0),
+                                          ("mlp_down", None, 0)])
+def test_full_size_repeatable_with_poisoned_workspace(name, M, split):
+    """Three calls on the same input, the workspace filled with 0xFF bytes (NaN in every f16 and fp32 slot,
+    0xFFFFFFFF in every count) before each: the same bytes every time, and no NaN.  The calls' pipelines
+    (TMA rings, TMEM stages, accumulator hand-offs, split-K partials, stream-K segments) run at full size
+    with every CTA busy, where an ordering race between roles or CTAs shows up as differing tiles."""
+    w = S.WORKLOADS[name]
+    M = w.M if M is None else M
+    codes, s, b = w.w()
+    xd = to_dev_bf16(w.x(M))
+    cd, sd, bd = _dev(codes, s, b)
+    ws = torch.empty(max(ql.workspace_size(M, w.K, w.N, ql.PATH_AUTO, split), 16), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(3):
+        ws.fill_(0xFF)
+        y = ql.forward(xd, cd, sd, bd, workspace=ws, split_k=split)
+        assert ql.device_status() == 0
+        outs.append(bf16_bits(y))
+    assert not np.any((outs[0] & 0x7F80) == 0x7F80), "NaN or infinity in the output"
+    for o in outs[1:]:
+        diff = np.flatnonzero(o != outs[0])
+        assert diff.size == 0, (name, M, diff.size, diff[:8])
