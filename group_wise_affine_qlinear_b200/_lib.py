@@ -104,6 +104,8 @@ def load_library(path: str) -> ctypes.CDLL:
     L.qlinear_test_stall.restype = ctypes.c_int
     L.qlinear_test_ring_depth.argtypes = [i32]
     L.qlinear_test_ring_depth.restype = ctypes.c_int
+    L.qlinear_test_delay.argtypes = [i32, ctypes.c_uint64]
+    L.qlinear_test_delay.restype = ctypes.c_int
     return L
 
 

@@ -879,6 +879,22 @@ ql_status qlinear_test_stall(int32_t kernel_mask, uint64_t wait_limit_ns) {
 #endif
 }
 
+ql_status qlinear_test_delay(int32_t role_mask, uint64_t max_ns) {
+#ifdef QL_BOUNDS_CHECK
+    constexpr int kAll = kDelayActivations | kDelayCodes | kDelayDequant | kDelayMma | kDelayEpilogue;
+    if (role_mask < 0 || (role_mask & ~kAll) != 0 || max_ns > 1000000) return QL_ERR_INVALID_ARG;
+    const unsigned long long ns = max_ns;
+    if (cudaMemcpyToSymbol(g_delay_mask, &role_mask, sizeof(role_mask)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_delay_ns, &ns, sizeof(ns)) != cudaSuccess)
+        return QL_ERR_CUDA;
+    return QL_OK;
+#else
+    (void)role_mask;
+    (void)max_ns;
+    return QL_ERR_UNSUPPORTED;
+#endif
+}
+
 ql_status qlinear_test_ring_depth(int32_t variant) {
 #ifdef QL_BOUNDS_CHECK
     if (variant < 0 || variant >= QL_TEST_RING_VARIANTS) return QL_ERR_INVALID_ARG;

@@ -62,6 +62,28 @@ __device__ __forceinline__ constexpr uint64_t wait_limit_ns() { return kWaitLimi
 __device__ __forceinline__ constexpr bool stalled(int) { return false; }
 #endif
 
+// Roles of the tensor-core kernels that the checked build can hold back at their start (qlinear_test_delay):
+// the activation producer, the code producer, the dequantizers (builders), the MMA issuers and the
+// epilogue (drain) warps.
+constexpr int kDelayActivations = 1, kDelayCodes = 2, kDelayDequant = 4, kDelayMma = 8, kDelayEpilogue = 16;
+
+#ifdef QL_BOUNDS_CHECK
+// Test hook of the checked build: a role in the mask spins at its start for a CTA- and warp-dependent
+// part (0/7 .. 7/7) of g_delay_ns, bounded by the time read, so that every hand-off between roles meets
+// other orders of arrival; a race between roles then shows up as differing output bytes.
+static __device__ int g_delay_mask;
+static __device__ unsigned long long g_delay_ns;
+__device__ __forceinline__ void test_delay(int role_bit) {
+    if ((g_delay_mask & role_bit) == 0) return;
+    const uint64_t d = g_delay_ns * ((blockIdx.x * 7u + (threadIdx.x >> 5) * 3u) % 8u) / 7u;
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < d) {
+    }
+}
+#else
+__device__ __forceinline__ void test_delay(int) {}
+#endif
+
 __device__ __forceinline__ uint32_t bits_of(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 half2_of(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 

@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
 
     if (warp < kDequantWarps) {
         // ---------------------------------------------------------------- dequantizers
+        test_delay(kDelayDequant);   // the checked build can hold this role back (qlinear_test_delay)
         const int grp = warp >> 2;                 // weight-row group
         const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
         const int r = grp * BWG + quarter * 32 + lane;   // weight row within the tile
@@ -306,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         }
     } else if (warp == kWarpTmaX) {
         // ---------------------------------------------------------------- TMA producer of activation tiles
+        test_delay(kDelayActivations);   // the checked build can hold this role back (qlinear_test_delay)
         if (lane == 0) {
             uint32_t i = 0;
             bool ok = true;
@@ -331,6 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         }
     } else if (warp == kWarpTmaC) {
         // ---------------------------------------------------------------- TMA producer of codes and parameters
+        test_delay(kDelayCodes);   // the checked build can hold this role back (qlinear_test_delay)
         // (the checked build's stall hook holds it back: no code or parameter load)
         if (lane == 0 && !stalled(kStallFused)) {
             // one code stage: kS K-steps of a tile's 256 rows (in SwiGLU mode 128 gate rows, then the same
@@ -396,6 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         }
     } else if (warp == kWarpMma || warp == kWarpMma2) {
         // ---------------------------------------------------------------- MMA issuers, one per group
+        test_delay(kDelayMma);   // the checked build can hold this role back (qlinear_test_delay)
         const int gsel = warp == kWarpMma ? 0 : 1;
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_f16(BWG, BT, false);
@@ -439,6 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         }
     } else if (kSwiGLU && warp >= kWarpEpi0) {
         // ---------------------------------------------------------------- SwiGLU epilogue
+        test_delay(kDelayEpilogue);   // the checked build can hold this role back (qlinear_test_delay)
         // Warp (quarter, half) reads the gate and up accumulators of TMEM lanes 32*quarter .. +31 (its
         // 32 intermediate columns) for the token chunks kHalfChunks*half .. +kHalfChunks-1.
         constexpr int kHalfChunks = BT / 32 / 2;
@@ -504,6 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
         if (lane == 0) ptx::bulk_wait_group_all();   // every store has completed before the CTA exits
     } else if (warp >= kWarpEpi0) {
         // ---------------------------------------------------------------- epilogue
+        test_delay(kDelayEpilogue);   // the checked build can hold this role back (qlinear_test_delay)
         // All 8 warps drain group 0's accumulator first, then group 1's: warp (quarter, half) takes TMEM
         // lanes 32*quarter .. +31 and the token chunks kHalf*half .. +kHalf-1 of each group, so group 0 is
         // released after half a drain and its MMAs of the next unit run while group 1 is drained.

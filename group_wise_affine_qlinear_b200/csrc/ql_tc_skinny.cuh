@@ -294,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
 
     if (warp == kWarpTmaC) {
         // ---------------------------------------------------------------- code + parameter producer
+        test_delay(kDelayCodes);   // the checked build can hold this role back (qlinear_test_delay)
         // (codes and parameters do not depend on the prepass: no dependency wait; the checked build's
         // stall hook holds this producer back: no code or parameter load at all)
         if (lane == 0 && !stalled(kStallSkinny)) {
@@ -323,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
         }
     } else if (warp == kWarpTmaX) {
         // ---------------------------------------------------------------- activation producer
+        test_delay(kDelayActivations);   // the checked build can hold this role back (qlinear_test_delay)
         if (lane == 0) {
             ptx::grid_dependency_wait();              // the activations come from the prepass
             uint32_t xi = 0;
@@ -341,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
         }
     } else if (warp < kWarpMma0 + kMmaCopies) {
         // ---------------------------------------------------------------- MMA issuers (even / odd pairs)
+        test_delay(kDelayMma);   // the checked build can hold this role back (qlinear_test_delay)
         // The whole warp runs the loop; one elected lane issues the MMAs and the commits.
         const int copy = warp - kWarpMma0;
         const bool leader = ptx::elect_one();
@@ -404,6 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
         ptx::mbar_wait(&drain[copy], 0, nullptr);
     } else if (warp < kWarpDrain0) {
         // ---------------------------------------------------------------- A builders (four copies)
+        test_delay(kDelayDequant);   // the checked build can hold this role back (qlinear_test_delay)
         const int copy = (warp - kWarpBuild0) >> 2;
         const int quarter = warp & 3;                      // TMEM lanes 32*quarter.. belong to this warp
         const int r = quarter * 32 + lane;
@@ -498,6 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const __grid_consta
         }
     } else {
         // ---------------------------------------------------------------- drain (tile segment ends)
+        test_delay(kDelayEpilogue);   // the checked build can hold this role back (qlinear_test_delay)
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;

@@ -198,6 +198,18 @@ QL_API ql_status qlinear_test_stall(int32_t kernel_mask, uint64_t wait_limit_ns)
 QL_API ql_status qlinear_test_ring_depth(int32_t variant);
 
 /*
+ * Test hook of the checked build (libqlinear_bounds.so); the pages have no counterpart.  Holds back the
+ * roles of the tensor-core kernels in role_mask at their start, each CTA's and warp's by a different part
+ * (0/7 .. 7/7) of max_ns, so that every hand-off between roles (TMA rings, tensor-memory stages,
+ * accumulators, partials) meets other orders of arrival; the output must not change.  Bits: 1 the
+ * activation producer, 2 the code producer, 4 the dequantizers, 8 the MMA issuers, 16 the epilogue or
+ * drain warps.  role_mask 0 turns it off.  Synchronous (two small host-to-device copies on the legacy
+ * stream).  The shipped library returns QL_ERR_UNSUPPORTED; QL_ERR_INVALID_ARG for an unknown bit or
+ * max_ns above 1 ms.
+ */
+QL_API ql_status qlinear_test_delay(int32_t role_mask, uint64_t max_ns);
+
+/*
  * Allocation-free forward for small M.  The pages have no counterpart of this
  * call; it exists for callers that cannot allocate device memory where they
  * run the layer (a plugin living inside another engine's fixed memory pool, a

@@ -244,3 +244,4 @@ def test_test_hooks_are_inert_in_the_shipped_library(L):
     assert L.qlinear_test_stall(1, 20_000_000) == 3              # QL_ERR_UNSUPPORTED
     assert L.qlinear_test_ring_depth(1) == 3
     assert L.qlinear_test_ring_depth(0) == 3
+    assert L.qlinear_test_delay(31, 10_000) == 3
