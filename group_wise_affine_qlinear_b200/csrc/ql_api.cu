@@ -387,6 +387,20 @@ cudaError_t ring_smem_attr() {
 }
 #endif
 
+// The activation conversion in front of the fused kernel: 128-thread CTAs for rows that fit their
+// registers (K <= 5120), 256-thread CTAs for longer rows (the two shapes of convert_x_kernel).
+void launch_convert_x(int bits, const __nv_bfloat16* x, __half* xh, float* rs, int64_t M, int64_t K, cudaStream_t st) {
+    const unsigned rows = static_cast<unsigned>(M);
+    const int k = static_cast<int>(K);
+    if (K <= 128 * 5 * 8) {
+        if (bits == 4) convert_x_kernel<4, 128, 5><<<rows, 128, 0, st>>>(x, xh, rs, k);
+        else convert_x_kernel<8, 128, 5><<<rows, 128, 0, st>>>(x, xh, rs, k);
+    } else {
+        if (bits == 4) convert_x_kernel<4, 256, 4><<<rows, 256, 0, st>>>(x, xh, rs, k);
+        else convert_x_kernel<8, 256, 4><<<rows, 256, 0, st>>>(x, xh, rs, k);
+    }
+}
+
 ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const void* scales, const void* biases,
                     void* y, bool bf16_out, int64_t M, int64_t K, int64_t N, void* ws, cudaStream_t st,
                     int sm_count) {
@@ -424,12 +438,7 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
         return s;
     }
 
-    if (bits == 4)
-        convert_x_kernel<4><<<static_cast<unsigned>(M), kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), xh,
-                                                                              rs, static_cast<int>(K));
-    else
-        convert_x_kernel<8><<<static_cast<unsigned>(M), kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), xh,
-                                                                              rs, static_cast<int>(K));
+    launch_convert_x(bits, static_cast<const __nv_bfloat16*>(x), xh, rs, M, K, st);
     if ((s = launch_status()) != QL_OK) return s;
     // the transpose, then the fused kernel, start under programmatic dependent launch (each waits
     // for the kernels before it where it reads their output)
@@ -641,8 +650,7 @@ ql_status run_swiglu(const SwigluPlan& pl, const void* x, const uint32_t* gc, co
     if ((s = encode_2d(&my, bf16_out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, h, I, M,
                        I * (bf16_out ? 2 : 4), 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
         return s;
-    convert_x_kernel<4><<<static_cast<unsigned>(M), kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), xh, rs,
-                                                                          static_cast<int>(K));
+    launch_convert_x(4, static_cast<const __nv_bfloat16*>(x), xh, rs, M, K, st);
     if ((s = launch_status()) != QL_OK) return s;
     const dim3 tgrid(static_cast<unsigned>((G + 31) / 32), static_cast<unsigned>(pl.ncols / 32));
     if ((s = launch_dependent(transpose_params_pair_kernel, tgrid, 256, 0, st, static_cast<const __half*>(gs),

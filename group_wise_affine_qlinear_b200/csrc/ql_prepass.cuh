@@ -20,12 +20,12 @@
 
 namespace ql {
 
-constexpr int kPrepThreads = 256;
-
-// One CTA per row.  Pass 1 reads the row for max|x|, keeping up to kConvCache 8-blocks per thread in
-// registers (all of a row of K <= 8192), pass 2 converts them (re-reading, from L2, only what did not
-// fit).  All of a thread's pass-1 loads are issued before the first is used.
-constexpr int kConvCache = 4;
+// One CTA of kThreads per row.  Pass 1 reads the row for max|x|, keeping up to kCache 8-blocks per
+// thread in registers, pass 2 converts them (re-reading, from L2, only what did not fit).  All of a
+// thread's pass-1 loads are issued before the first is used.  Two shapes: 128 threads x 5 blocks hold a
+// row of up to 5120 elements and let twice as many rows be in flight per SM as 256-thread CTAs (about 4 us
+// less on the QKV projection's 4608 x 4608 activations, 20 us on the 2048^2 canvas's 33792 x 4608, on a
+// B200); longer rows take 256 threads x 4 blocks, which measured faster there (K = 18432 and 53248).
 
 // The f16 8-block of a bf16 8-block scaled by inv, in the k order the dequantizer of kBits-bit codes
 // emits its pairs in.
@@ -64,28 +64,28 @@ __device__ __forceinline__ float absmax_bf16x8(const uint4 v, float amax) {
 }
 
 // kBits: width of the weight codes the activations will meet (4 or 8), which fixes the k order.
-template <int kBits>
-__global__ void __launch_bounds__(kPrepThreads) convert_x_kernel(const __nv_bfloat16* __restrict__ x,
-                                                                 __half* __restrict__ xh,
-                                                                 float* __restrict__ rowscale, int K) {
+template <int kBits, int kThreads, int kCache>
+__global__ void __launch_bounds__(kThreads) convert_x_kernel(const __nv_bfloat16* __restrict__ x,
+                                                             __half* __restrict__ xh,
+                                                             float* __restrict__ rowscale, int K) {
     ptx::launch_dependents();
-    __shared__ float red[kPrepThreads / 32];
+    __shared__ float red[kThreads / 32];
     __shared__ int row_exp;
     const int64_t m = blockIdx.x;
     const uint4* src = reinterpret_cast<const uint4*>(x + m * K);   // 8 bf16 per uint4
     uint4* dst = reinterpret_cast<uint4*>(xh + m * K);
     const int n8 = K / 8;
 
-    uint4 v[kConvCache];
+    uint4 v[kCache];
 #pragma unroll
-    for (int j = 0; j < kConvCache; ++j) {
-        const int i = threadIdx.x + j * kPrepThreads;
+    for (int j = 0; j < kCache; ++j) {
+        const int i = threadIdx.x + j * kThreads;
         v[j] = i < n8 ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
     }
     float amax = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kConvCache; ++j) amax = absmax_bf16x8(v[j], amax);
-    for (int i = threadIdx.x + kConvCache * kPrepThreads; i < n8; i += kPrepThreads)
+    for (int j = 0; j < kCache; ++j) amax = absmax_bf16x8(v[j], amax);
+    for (int i = threadIdx.x + kCache * kThreads; i < n8; i += kThreads)
         amax = absmax_bf16x8(__ldg(src + i), amax);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kPrepThreads) convert_x_kernel(const __nv_bflo
     __syncthreads();
     if (threadIdx.x == 0) {
         float a = red[0];
-        for (int i = 1; i < kPrepThreads / 32; ++i) a = fmaxf(a, red[i]);
+        for (int i = 1; i < kThreads / 32; ++i) a = fmaxf(a, red[i]);
         int e = 0;                         // zero, inf or nan rows: no scaling
         if (a > 0.0f && a <= 3.4028235e38f) {
             const int ea = static_cast<int>((__float_as_uint(a) >> 23) & 0xFF) - 127;   // floor(log2 a), a normal
@@ -105,11 +105,11 @@ __global__ void __launch_bounds__(kPrepThreads) convert_x_kernel(const __nv_bflo
     __syncthreads();
     const float inv = __uint_as_float(static_cast<uint32_t>(127 - row_exp) << 23);   // 2^-e, exact
 #pragma unroll
-    for (int j = 0; j < kConvCache; ++j) {
-        const int i = threadIdx.x + j * kPrepThreads;
+    for (int j = 0; j < kCache; ++j) {
+        const int i = threadIdx.x + j * kThreads;
         if (i < n8) dst[i] = convert8<kBits>(v[j], inv);
     }
-    for (int i = threadIdx.x + kConvCache * kPrepThreads; i < n8; i += kPrepThreads)
+    for (int i = threadIdx.x + kCache * kThreads; i < n8; i += kThreads)
         dst[i] = convert8<kBits>(__ldg(src + i), inv);
 }
 

@@ -6,6 +6,10 @@ import torch
 
 from group_wise_affine_qlinear_b200 import synthetic as S
 
+# Tokens per tile of the fused tensor-core kernel (its dispatch record says "... x 192t ..."); sampled
+# rows include both sides of every boundary between such tiles.
+FUSED_TILE_TOKENS = 192
+
 
 def to_dev_codes(codes: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(codes).view(np.int32)).cuda()

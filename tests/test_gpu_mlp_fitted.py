@@ -17,7 +17,7 @@ import group_wise_affine_qlinear_b200 as ql
 from group_wise_affine_qlinear_b200 import synthetic as S
 from oracle import qlinear_oracle as O
 
-from ._helpers import bf16_bits, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
+from ._helpers import FUSED_TILE_TOKENS, bf16_bits, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
 from ._oracle_pool import pack_imatrix_parallel
 
 pytestmark = pytest.mark.gpu
@@ -48,7 +48,7 @@ def test_mlp_up_gate_with_fitted_rows():
     codes[:R], s[:R], b[:R] = rc, rs, rb
     y = ql.forward(to_dev_bf16(x), to_dev_codes(codes), to_dev_f16(s), to_dev_f16(b))
     assert ql.last_dispatch().startswith("path=tc_fused")
-    rows = sample_rows(w.M, n_random=48, seed=2)
+    rows = sample_rows(w.M, n_random=48, seed=2, tile=FUSED_TILE_TOKENS)
     y_ref = O.forward_rows(x, codes, s, b, rows)
     got = O.decode_bf16(bf16_bits(y)[rows])
     t = O.tolerance(got, y_ref)

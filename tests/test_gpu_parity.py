@@ -13,7 +13,7 @@ import group_wise_affine_qlinear_b200 as ql
 from group_wise_affine_qlinear_b200 import synthetic as S
 from oracle import qlinear_oracle as O
 
-from ._helpers import bf16_bits, random_layer, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
+from ._helpers import FUSED_TILE_TOKENS, bf16_bits, random_layer, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
 
 pytestmark = pytest.mark.gpu
 
@@ -308,6 +308,7 @@ def test_dispatch_record():
     x, codes, s, b = random_layer(rng, 256, 256, 256)
     ql.forward(to_dev_bf16(x), *_dev(codes, s, b))
     assert ql.last_dispatch().startswith("path=tc_fused")
+    assert f" x {FUSED_TILE_TOKENS}t " in ql.last_dispatch()      # the tile the tests sample boundaries of
     ql.forward(to_dev_bf16(x[:1]), *_dev(codes, s, b))
     assert ql.last_dispatch().startswith("path=tc_skinny")
 
@@ -347,7 +348,7 @@ def _full_case(name, M=None, path=ql.PATH_AUTO, fitted=None):
     x = w.x(M)
     codes, s, b = w.w() if fitted is None else fitted
     y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=path)
-    rows = sample_rows(M, n_random=48, seed=M)
+    rows = sample_rows(M, n_random=48, seed=M, tile=FUSED_TILE_TOKENS)
     y_ref = O.forward_rows(x, codes, s, b, rows)
     got = bf16_bits(y)[rows]
     t = O.tolerance(O.decode_bf16(got), y_ref)

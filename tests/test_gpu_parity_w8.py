@@ -13,7 +13,7 @@ import group_wise_affine_qlinear_b200 as ql
 from group_wise_affine_qlinear_b200 import synthetic as S
 from oracle import qlinear_oracle as O
 
-from ._helpers import bf16_bits, random_layer8, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
+from ._helpers import FUSED_TILE_TOKENS, bf16_bits, random_layer8, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
 
 pytestmark = pytest.mark.gpu
 
@@ -255,7 +255,7 @@ def test_full_text_proj_w8(M):
     x = w.x(M)
     codes, s, b = w.w()
     y = ql.forward8(to_dev_bf16(x), *_dev(codes, s, b))
-    rows = sample_rows(M, n_random=48, seed=M)
+    rows = sample_rows(M, n_random=48, seed=M, tile=FUSED_TILE_TOKENS)
     y_ref = O.forward8_rows(x, codes, s, b, rows)
     t = O.tolerance(O.decode_bf16(bf16_bits(y)[rows]), y_ref)
     assert t["ok"], (M, t)

@@ -16,7 +16,7 @@ import torch
 import group_wise_affine_qlinear_b200 as ql
 from oracle import qlinear_oracle as O
 
-from ._helpers import bf16_bits, random_layer, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
+from ._helpers import FUSED_TILE_TOKENS, bf16_bits, random_layer, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
 
 pytestmark = pytest.mark.gpu
 
@@ -64,7 +64,7 @@ def test_every_ring_depth_writes_the_same_bytes(M, K, N):
     for v in range(1, VARIANTS):
         diff = np.flatnonzero(outs[v] != outs[0])
         assert diff.size == 0, (v, diff[:8])
-    rows = sample_rows(M, n_random=24, seed=M, tile=192)
+    rows = sample_rows(M, n_random=24, seed=M, tile=FUSED_TILE_TOKENS)
     t = O.tolerance(O.decode_bf16(outs[0][rows]), O.forward_rows(x, codes, s, b, rows))
     assert t["ok"], t
 

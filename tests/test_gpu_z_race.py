@@ -16,7 +16,7 @@ import torch
 import group_wise_affine_qlinear_b200 as ql
 from oracle import qlinear_oracle as O
 
-from ._helpers import bf16_bits, random_layer, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
+from ._helpers import FUSED_TILE_TOKENS, bf16_bits, random_layer, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
 
 pytestmark = pytest.mark.gpu
 
@@ -55,7 +55,7 @@ def test_outputs_do_not_depend_on_role_timing(M, K, N, path, split):
 
     assert Lc.qlinear_test_delay(0, 0) == 0
     ref = call()
-    rows = sample_rows(M, n_random=16, seed=M)
+    rows = sample_rows(M, n_random=16, seed=M, tile=FUSED_TILE_TOKENS)
     t = O.tolerance(O.decode_bf16(ref[rows]), O.forward_rows(x, codes, s, b, rows))
     assert t["ok"], t
     try:

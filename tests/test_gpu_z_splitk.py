@@ -15,7 +15,7 @@ import group_wise_affine_qlinear_b200 as ql
 from group_wise_affine_qlinear_b200 import synthetic as S
 from oracle import qlinear_oracle as O
 
-from ._helpers import bf16_bits, random_layer, random_layer8, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
+from ._helpers import FUSED_TILE_TOKENS, bf16_bits, random_layer, random_layer8, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
 
 pytestmark = pytest.mark.gpu
 
@@ -66,6 +66,6 @@ def test_fused_split_k_text_proj_m512():
     x = w.x(512)
     codes, s, b = w.w()
     y = ql.forward(to_dev_bf16(x), *_dev(codes, s, b), path=ql.PATH_TC_FUSED, split_k=8)
-    rows = sample_rows(512, n_random=32, seed=512, tile=192)
+    rows = sample_rows(512, n_random=32, seed=512, tile=FUSED_TILE_TOKENS)
     t = O.tolerance(O.decode_bf16(bf16_bits(y)[rows]), O.forward_rows(x, codes, s, b, rows))
     assert t["ok"], t

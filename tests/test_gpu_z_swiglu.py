@@ -16,7 +16,7 @@ import group_wise_affine_qlinear_b200 as ql
 from group_wise_affine_qlinear_b200 import synthetic as S
 from oracle import qlinear_oracle as O
 
-from ._helpers import bf16_bits, random_layer, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
+from ._helpers import FUSED_TILE_TOKENS, bf16_bits, random_layer, sample_rows, to_dev_bf16, to_dev_codes, to_dev_f16
 
 pytestmark = pytest.mark.gpu
 
@@ -109,10 +109,10 @@ def test_swiglu_deterministic():
 
 
 def test_swiglu_full_mlp_width():
-    """The pages' MLP: K = 4608, I = 12288, 4608 tokens; sampled rows (every 192-token tile boundary)."""
+    """The pages' MLP: K = 4608, I = 12288, 4608 tokens; sampled rows (both sides of every fused-tile boundary)."""
     w = S.WORKLOADS["mlp_gate_up_12288"]
     x = w.x()
     gate, up = w.w_pair()
     h = ql.swiglu(to_dev_bf16(x), _dev(*gate), _dev(*up))
-    rows = sample_rows(w.M, n_random=24, seed=5, tile=192)
+    rows = sample_rows(w.M, n_random=24, seed=5, tile=FUSED_TILE_TOKENS)
     _check(h, x, gate, up, rows=rows)
