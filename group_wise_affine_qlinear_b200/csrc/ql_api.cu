@@ -387,18 +387,18 @@ cudaError_t ring_smem_attr() {
 }
 #endif
 
-// The activation conversion in front of the fused kernel: 128-thread CTAs for rows that fit their
-// registers (K <= 5120), 256-thread CTAs for longer rows (the two shapes of convert_x_kernel).
-void launch_convert_x(int bits, const __nv_bfloat16* x, __half* xh, float* rs, int64_t M, int64_t K, cudaStream_t st) {
-    const unsigned rows = static_cast<unsigned>(M);
+// The activation conversion in front of the fused kernel, launched behind the parameter transpose
+// under programmatic dependent launch: 128-thread CTAs for rows that fit their registers (K <= 5120),
+// 256-thread CTAs for longer rows (the two shapes of convert_x_kernel).
+ql_status launch_convert_x(int bits, const __nv_bfloat16* x, __half* xh, float* rs, int64_t M, int64_t K,
+                           cudaStream_t st) {
+    const dim3 rows(static_cast<unsigned>(M));
     const int k = static_cast<int>(K);
-    if (K <= 128 * 5 * 8) {
-        if (bits == 4) convert_x_kernel<4, 128, 5><<<rows, 128, 0, st>>>(x, xh, rs, k);
-        else convert_x_kernel<8, 128, 5><<<rows, 128, 0, st>>>(x, xh, rs, k);
-    } else {
-        if (bits == 4) convert_x_kernel<4, 256, 4><<<rows, 256, 0, st>>>(x, xh, rs, k);
-        else convert_x_kernel<8, 256, 4><<<rows, 256, 0, st>>>(x, xh, rs, k);
-    }
+    if (K <= 128 * 5 * 8)
+        return bits == 4 ? launch_dependent(convert_x_kernel<4, 128, 5>, rows, 128, 0, st, x, xh, rs, k)
+                         : launch_dependent(convert_x_kernel<8, 128, 5>, rows, 128, 0, st, x, xh, rs, k);
+    return bits == 4 ? launch_dependent(convert_x_kernel<4, 256, 4>, rows, 256, 0, st, x, xh, rs, k)
+                     : launch_dependent(convert_x_kernel<8, 256, 4>, rows, 256, 0, st, x, xh, rs, k);
 }
 
 ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const void* scales, const void* biases,
@@ -438,14 +438,15 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
         return s;
     }
 
-    launch_convert_x(bits, static_cast<const __nv_bfloat16*>(x), xh, rs, M, K, st);
-    if ((s = launch_status()) != QL_OK) return s;
-    // the transpose, then the fused kernel, start under programmatic dependent launch (each waits
-    // for the kernels before it where it reads their output)
+    // The parameter transpose first (a plain launch: it follows the caller's earlier work), then the
+    // conversion and the fused kernel under programmatic dependent launch: the conversion runs beside the
+    // transpose, its last CTA waits for it, and the fused kernel waits for the conversion where it reads
+    // the outputs of both.
     const dim3 tgrid(static_cast<unsigned>((G + 31) / 32), static_cast<unsigned>((N + 31) / 32));
-    if ((s = launch_dependent(transpose_params_kernel, tgrid, 256, 0, st, static_cast<const __half*>(scales),
-                              static_cast<const __half*>(biases), sb, static_cast<int>(N), static_cast<int>(G))) != QL_OK)
-        return s;
+    transpose_params_kernel<<<tgrid, 256, 0, st>>>(static_cast<const __half*>(scales), static_cast<const __half*>(biases),
+                                                   sb, static_cast<int>(N), static_cast<int>(G));
+    if ((s = launch_status()) != QL_OK) return s;
+    if ((s = launch_convert_x(bits, static_cast<const __nv_bfloat16*>(x), xh, rs, M, K, st)) != QL_OK) return s;
     fused::Params p;
     p.rowscale = rs;
     p.y = y;
@@ -650,14 +651,14 @@ ql_status run_swiglu(const SwigluPlan& pl, const void* x, const uint32_t* gc, co
     if ((s = encode_2d(&my, bf16_out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, h, I, M,
                        I * (bf16_out ? 2 : 4), 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
         return s;
-    launch_convert_x(4, static_cast<const __nv_bfloat16*>(x), xh, rs, M, K, st);
-    if ((s = launch_status()) != QL_OK) return s;
+    // pair transpose, then conversion and fused kernel under programmatic dependent launch (as run_fused)
     const dim3 tgrid(static_cast<unsigned>((G + 31) / 32), static_cast<unsigned>(pl.ncols / 32));
-    if ((s = launch_dependent(transpose_params_pair_kernel, tgrid, 256, 0, st, static_cast<const __half*>(gs),
-                              static_cast<const __half*>(gb), static_cast<const __half*>(us),
-                              static_cast<const __half*>(ub), sb, static_cast<int>(I), static_cast<int>(G),
-                              static_cast<int>(pl.ncols))) != QL_OK)
-        return s;
+    transpose_params_pair_kernel<<<tgrid, 256, 0, st>>>(static_cast<const __half*>(gs), static_cast<const __half*>(gb),
+                                                        static_cast<const __half*>(us), static_cast<const __half*>(ub),
+                                                        sb, static_cast<int>(I), static_cast<int>(G),
+                                                        static_cast<int>(pl.ncols));
+    if ((s = launch_status()) != QL_OK) return s;
+    if ((s = launch_convert_x(4, static_cast<const __nv_bfloat16*>(x), xh, rs, M, K, st)) != QL_OK) return s;
     fused::Params p;
     p.rowscale = rs;
     p.y = h;

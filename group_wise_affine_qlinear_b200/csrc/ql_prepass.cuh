@@ -111,11 +111,14 @@ __global__ void __launch_bounds__(kThreads) convert_x_kernel(const __nv_bfloat16
     }
     for (int i = threadIdx.x + kCache * kThreads; i < n8; i += kThreads)
         dst[i] = convert8<kBits>(__ldg(src + i), inv);
+    // Launched behind the parameter transpose under programmatic dependent launch, this kernel runs beside
+    // it; its last CTA waits for it before finishing, so that this kernel's completion implies both.
+    if (blockIdx.x == gridDim.x - 1) ptx::grid_dependency_wait();
 }
 
-// sb[g][n] = (scale[n][g], bias[n][g]); 32x32 tiles through shared memory.  Launched behind
-// convert_x_kernel under programmatic dependent launch: it does not read that kernel's output, so it
-// runs alongside it, and waits for it only before finishing, so that its own completion implies both.
+// sb[g][n] = (scale[n][g], bias[n][g]); 32x32 tiles through shared memory.  The first kernel of a
+// fused-path call: it lets the activation conversion start at once (programmatic dependent launch),
+// which runs beside it and waits for it only in its last CTA.
 __global__ void __launch_bounds__(256) transpose_params_kernel(const __half* __restrict__ scales,
                                                                const __half* __restrict__ biases,
                                                                uint32_t* __restrict__ sb, int N, int G) {
@@ -138,14 +141,13 @@ __global__ void __launch_bounds__(256) transpose_params_kernel(const __half* __r
         const int g = g0 + r, n = n0 + tx;
         if (g < G && n < N) sb[static_cast<int64_t>(g) * N + n] = tile[tx][r];
     }
-    ptx::grid_dependency_wait();
 }
 
 // SwiGLU pair: sb[g][256 w + r] = (scale, bias) of gate row 128 w + r for r < 128, of up row
 // 128 w + (r - 128) for r >= 128 (zeros past row I-1), so that one K-step's parameters of tile w are
 // one contiguous run of 256 pairs in the fused kernel's row order.  32x32 tiles as above; a tile's 32
 // destination columns never straddle a 128-row half, so they come from 32 consecutive rows of one
-// weight.  grid: (ceil(G / 32), num_w * 8).
+// weight.  grid: (ceil(G / 32), num_w * 8).  Launched first, like transpose_params_kernel.
 __global__ void __launch_bounds__(256) transpose_params_pair_kernel(const __half* __restrict__ gate_scales,
                                                                     const __half* __restrict__ gate_biases,
                                                                     const __half* __restrict__ up_scales,
@@ -175,7 +177,6 @@ __global__ void __launch_bounds__(256) transpose_params_pair_kernel(const __half
         const int g = g0 + r, c = c0 + tx;
         if (g < G && c < ncols) sb[static_cast<int64_t>(g) * ncols + c] = tile[tx][r];
     }
-    ptx::grid_dependency_wait();
 }
 
 }  // namespace ql
