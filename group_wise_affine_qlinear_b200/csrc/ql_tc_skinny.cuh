@@ -120,9 +120,6 @@ __host__ __device__ __forceinline__ int64_t run_first(int64_t units, int P, int 
     return units * c / P;
 }
 
-// Activation prepass, two kernels over a grid of (slice, row): one thread per 8-block of k, 256 per
-// CTA, so every 8-block of a row is read in parallel.
-
 // The activation prepass in one launch, one cluster of kPrepCluster CTAs per row t: each CTA takes
 // 1/kPrepCluster of the row's 8-blocks, the CTAs' maxima meet in distributed shared memory, then
 // e_t puts max_k |x[t][k]| in [2^14, 2^15) (0 for a zero or non-finite row);
