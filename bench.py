@@ -596,6 +596,33 @@ class Case:
         main_ms = [a.elapsed_time(b) for a, b in evm]
         return sum(step_ms) / steps, sum(main_ms) / steps
 
+    def timed_graph(self, steps):
+        """Per-step device time of the same call replayed from a CUDA graph, L2 flushed before every step.
+
+        A serving loop captures a decode-sized layer once and replays it: the kernels then start without
+        the host launching each of them.  The capture records the call's launches (programmatic dependent
+        launch edges included) with this case's buffers.
+        """
+        torch = self.torch
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.step()
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            self.flush.fill_(i & 0xFF)
+            ev[i][0].record()
+            g.replay()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+        del g
+        return sum(ms) / steps
+
     def algorithmic_bytes(self):
         """Bytes a weight-streaming pass must move: packed W + x + y."""
         return self.w.weight_bytes * self.N // self.w.N + self.M * self.K * 2 + self.M * self.N * 2
@@ -698,11 +725,13 @@ def main():
             c = Case(ql, torch, tp, Ms, 0, dev, flush)
             c.warm(3)
             st, mn = c.timed(max(10, a.steps))
+            sg = c.timed_graph(max(10, a.steps))
             c.flush = dirty
             st_d, _ = c.timed(max(10, a.steps))
             out.append({"M": Ms, "dispatch": c.dispatch, "step_us": st * 1e3, "kernel_us": mn * 1e3,
                         "weight_GBps": tp.weight_bytes / (st * 1e-3) / 1e9,
                         "algorithmic_GBps": c.algorithmic_bytes() / (st * 1e-3) / 1e9,
+                        "graph_step_us": sg * 1e3, "graph_weight_GBps": tp.weight_bytes / (sg * 1e-3) / 1e9,
                         "step_us_dirty_l2": st_d * 1e3,
                         "traffic": recorded_traffic(c.dispatch.split()[0], f"{name}:M={Ms}")})
             del c
