@@ -58,7 +58,8 @@
 // interleaved the same way by the parameter prepass.  The two accumulators then
 // hold g and u for the same 128 intermediate columns and 192 tokens, and each of
 // the 8 epilogue warps reads both for its lane quarter and half of the tokens and
-// writes h = silu(g) * u = g / (1 + e^-g) * u in fp32, rounded once.
+// writes h = silu(g) * u = g / (1 + e^-g) * u in fp32 (the exponential and the
+// division through the SFU's exp2 and reciprocal), rounded once.
 #pragma once
 
 #include "ql_ptx.cuh"
@@ -488,7 +489,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_gemm_kernel(
                     const float sc = __shfl_sync(0xFFFFFFFFu, rs[c], k);
                     const float gv = __uint_as_float(rg[k]) * sc;
                     const float uv = __uint_as_float(ru[k]) * sc;
-                    const float h = gv / (1.0f + expf(-gv)) * uv;
+                    // the hardware exponential and reciprocal (a few fp32 ulps, far inside the bf16
+                    // rounding that follows); -inf gives NaN and large negative g gives -0 as before
+                    const float h = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
                     if constexpr (kBf16Out) {
                         reinterpret_cast<__nv_bfloat16*>(stage)[k * 32 + lane] = __float2bfloat16_rn(h);
                     } else {
