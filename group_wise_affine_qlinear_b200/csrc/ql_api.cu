@@ -442,7 +442,7 @@ ql_status run_fused(const Plan& pl, const void* x, const uint32_t* codes, const 
     // conversion and the fused kernel under programmatic dependent launch: the conversion runs beside the
     // transpose, its last CTA waits for it, and the fused kernel waits for the conversion where it reads
     // the outputs of both.
-    const dim3 tgrid(static_cast<unsigned>((G + 31) / 32), static_cast<unsigned>((N + 31) / 32));
+    const dim3 tgrid(static_cast<unsigned>((G + 31) / 32), static_cast<unsigned>((N + kTransposeCols - 1) / kTransposeCols));
     transpose_params_kernel<<<tgrid, 256, 0, st>>>(static_cast<const __half*>(scales), static_cast<const __half*>(biases),
                                                    sb, static_cast<int>(N), static_cast<int>(G));
     if ((s = launch_status()) != QL_OK) return s;
@@ -652,7 +652,7 @@ ql_status run_swiglu(const SwigluPlan& pl, const void* x, const uint32_t* gc, co
                        I * (bf16_out ? 2 : 4), 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) != QL_OK)
         return s;
     // pair transpose, then conversion and fused kernel under programmatic dependent launch (as run_fused)
-    const dim3 tgrid(static_cast<unsigned>((G + 31) / 32), static_cast<unsigned>(pl.ncols / 32));
+    const dim3 tgrid(static_cast<unsigned>((G + 31) / 32), static_cast<unsigned>(pl.ncols / kTransposeCols));
     transpose_params_pair_kernel<<<tgrid, 256, 0, st>>>(static_cast<const __half*>(gs), static_cast<const __half*>(gb),
                                                         static_cast<const __half*>(us), static_cast<const __half*>(ub),
                                                         sb, static_cast<int>(I), static_cast<int>(G),

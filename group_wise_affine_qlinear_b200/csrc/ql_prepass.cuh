@@ -116,66 +116,87 @@ __global__ void __launch_bounds__(kThreads) convert_x_kernel(const __nv_bfloat16
     if (blockIdx.x == gridDim.x - 1) ptx::grid_dependency_wait();
 }
 
-// sb[g][n] = (scale[n][g], bias[n][g]); 32x32 tiles through shared memory.  The first kernel of a
+// sb[g][n] = (scale[n][g], bias[n][g]) through shared memory, one CTA per 32 groups x kTransposeCols
+// rows: each thread issues all of its loads (kTransposeCols / 8 rows, scale and bias each) before the
+// first is used, so a CTA waits for memory once instead of once per 32 x 32 tile.  The first kernel of a
 // fused-path call: it lets the activation conversion start at once (programmatic dependent launch),
-// which runs beside it and waits for it only in its last CTA.
+// which runs beside it and waits for it only in its last CTA.  grid: (ceil(G / 32), ceil(N / kTransposeCols)).
+constexpr int kTransposeCols = 128;
+
 __global__ void __launch_bounds__(256) transpose_params_kernel(const __half* __restrict__ scales,
                                                                const __half* __restrict__ biases,
                                                                uint32_t* __restrict__ sb, int N, int G) {
     ptx::launch_dependents();
-    __shared__ uint32_t tile[32][33];
-    const int g0 = blockIdx.x * 32, n0 = blockIdx.y * 32;
+    __shared__ uint32_t tile[kTransposeCols][33];
+    const int g0 = blockIdx.x * 32, n0 = blockIdx.y * kTransposeCols;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;     // 8 rows per pass
-    for (int r = ty; r < 32; r += 8) {
-        const int n = n0 + r, g = g0 + tx;
-        uint32_t v = 0;
+    uint32_t v[kTransposeCols / 8];
+#pragma unroll
+    for (int j = 0; j < kTransposeCols / 8; ++j) {
+        const int n = n0 + ty + 8 * j, g = g0 + tx;
+        v[j] = 0;
         if (n < N && g < G) {
             const int64_t i = static_cast<int64_t>(n) * G + g;
-            v = static_cast<uint32_t>(__half_as_ushort(scales[i])) |
-                (static_cast<uint32_t>(__half_as_ushort(biases[i])) << 16);
+            v[j] = static_cast<uint32_t>(__half_as_ushort(scales[i])) |
+                   (static_cast<uint32_t>(__half_as_ushort(biases[i])) << 16);
         }
-        tile[r][tx] = v;
     }
+#pragma unroll
+    for (int j = 0; j < kTransposeCols / 8; ++j) tile[ty + 8 * j][tx] = v[j];
     __syncthreads();
     for (int r = ty; r < 32; r += 8) {
-        const int g = g0 + r, n = n0 + tx;
-        if (g < G && n < N) sb[static_cast<int64_t>(g) * N + n] = tile[tx][r];
+        const int g = g0 + r;
+        if (g >= G) break;
+#pragma unroll
+        for (int c = tx; c < kTransposeCols; c += 32) {
+            const int n = n0 + c;
+            if (n < N) sb[static_cast<int64_t>(g) * N + n] = tile[c][r];
+        }
     }
 }
 
 // SwiGLU pair: sb[g][256 w + r] = (scale, bias) of gate row 128 w + r for r < 128, of up row
 // 128 w + (r - 128) for r >= 128 (zeros past row I-1), so that one K-step's parameters of tile w are
-// one contiguous run of 256 pairs in the fused kernel's row order.  32x32 tiles as above; a tile's 32
-// destination columns never straddle a 128-row half, so they come from 32 consecutive rows of one
-// weight.  grid: (ceil(G / 32), num_w * 8).  Launched first, like transpose_params_kernel.
+// one contiguous run of 256 pairs in the fused kernel's row order.  As above, with kTransposeCols = 128
+// destination columns per CTA: exactly one 128-row half, so they come from 128 consecutive rows of one
+// weight.  grid: (ceil(G / 32), num_w * 2).  Launched first, like transpose_params_kernel.
 __global__ void __launch_bounds__(256) transpose_params_pair_kernel(const __half* __restrict__ gate_scales,
                                                                     const __half* __restrict__ gate_biases,
                                                                     const __half* __restrict__ up_scales,
                                                                     const __half* __restrict__ up_biases,
                                                                     uint32_t* __restrict__ sb, int I, int G,
                                                                     int ncols) {
+    static_assert(kTransposeCols == 128, "one CTA per 128-row half of a 256-column tile group");
     ptx::launch_dependents();
-    __shared__ uint32_t tile[32][33];
-    const int g0 = blockIdx.x * 32, c0 = blockIdx.y * 32;     // c0: first destination column
-    const int w = c0 >> 8, rr = c0 & 255;
-    const bool up = rr >= 128;
-    const int n0 = w * 128 + (rr & 127);                      // first source row
+    __shared__ uint32_t tile[kTransposeCols][33];
+    const int g0 = blockIdx.x * 32, c0 = blockIdx.y * kTransposeCols;     // c0: first destination column
+    const int w = c0 >> 8;
+    const bool up = (c0 & 255) >= 128;
+    const int n0 = w * 128;                                                // first source row
     const __half* sc = up ? up_scales : gate_scales;
     const __half* bi = up ? up_biases : gate_biases;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-    for (int r = ty; r < 32; r += 8) {
-        const int n = n0 + r, g = g0 + tx;
-        uint32_t v = 0;
+    uint32_t v[kTransposeCols / 8];
+#pragma unroll
+    for (int j = 0; j < kTransposeCols / 8; ++j) {
+        const int n = n0 + ty + 8 * j, g = g0 + tx;
+        v[j] = 0;
         if (n < I && g < G) {
             const int64_t i = static_cast<int64_t>(n) * G + g;
-            v = static_cast<uint32_t>(__half_as_ushort(sc[i])) | (static_cast<uint32_t>(__half_as_ushort(bi[i])) << 16);
+            v[j] = static_cast<uint32_t>(__half_as_ushort(sc[i])) | (static_cast<uint32_t>(__half_as_ushort(bi[i])) << 16);
         }
-        tile[r][tx] = v;
     }
+#pragma unroll
+    for (int j = 0; j < kTransposeCols / 8; ++j) tile[ty + 8 * j][tx] = v[j];
     __syncthreads();
     for (int r = ty; r < 32; r += 8) {
-        const int g = g0 + r, c = c0 + tx;
-        if (g < G && c < ncols) sb[static_cast<int64_t>(g) * ncols + c] = tile[tx][r];
+        const int g = g0 + r;
+        if (g >= G) break;
+#pragma unroll
+        for (int c = tx; c < kTransposeCols; c += 32) {
+            const int col = c0 + c;
+            if (col < ncols) sb[static_cast<int64_t>(g) * ncols + col] = tile[c][r];
+        }
     }
 }
 
