@@ -73,4 +73,6 @@ def test_ring_depth_hook_rejects_unknown_variants():
     Lc = _checked_library()
     assert Lc.qlinear_test_ring_depth(-1) == 1          # QL_ERR_INVALID_ARG
     assert Lc.qlinear_test_ring_depth(VARIANTS) == 1
-    assert ql.lib().qlinear_test_ring_depth(1) == 3     # the shipped library: QL_ERR_UNSUPPORTED
+    from group_wise_affine_qlinear_b200 import build as qb
+    shipped = ql.load_library(qb.build())               # by path: QL_LIBRARY may select the checked build
+    assert shipped.qlinear_test_ring_depth(1) == 3      # the shipped library: QL_ERR_UNSUPPORTED
